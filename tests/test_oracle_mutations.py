@@ -1,0 +1,114 @@
+"""Planted mistakes in the oracle must be caught by its pins.
+
+Each case monkeypatches one oracle function with a plausible bug (dropped
+term, wrong sign, transposed operand, swapped index) and runs the pin tests
+that should catch it; at least one of them must fail.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from oracle import rib_oracle as R
+import tests.test_oracle_pins as P
+
+
+def _scores_bias_sign(qc, kc, qp, kp, scale):
+    return scale * (R._f64(qc) @ R._f64(kc).T - R._f64(qp) @ R._f64(kp).T)
+
+
+def _scores_no_bias(qc, kc, qp, kp, scale):
+    return scale * (R._f64(qc) @ R._f64(kc).T)
+
+
+def _fourier_swapped(y, x, freqs):
+    w = R._f64(freqs).reshape(1, -1)
+    ax = np.asarray(x, dtype=np.float64).reshape(-1, 1) * w
+    ay = np.asarray(y, dtype=np.float64).reshape(-1, 1) * w
+    return np.concatenate([np.sin(ay), np.cos(ay), np.sin(ax), np.cos(ax)], 1)
+
+
+def _coords_no_endpoint(M):
+    lin = -1.0 + 2.0 * np.arange(M, dtype=np.float64) / M
+    return np.repeat(lin, M), np.tile(lin, M)
+
+
+def _gelu_tanh(z):
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1 + np.tanh(np.sqrt(2 / np.pi) * (z + 0.044715 * z ** 3)))
+
+
+def _partition_wrong_roll(x, M, s):
+    return _orig_partition(np.roll(np.asarray(x), shift=(s, s), axis=(1, 2)), M, 0)
+
+
+_orig_partition = R.window_partition
+
+
+def _bwd_missing_rowsum(qc, kc, v, qp, kp, scale, dout):
+    qc, kc, v, qp, kp, do = map(R._f64, (qc, kc, v, qp, kp, dout))
+    s = R.unit_scores(qc, kc, qp, kp, scale)
+    p, _ = R._softmax_rows(s)
+    dp = do @ v.T
+    ds = p * dp
+    return (scale * ds @ kc, scale * ds.T @ qc, p.T @ do, scale * ds @ kp,
+            scale * ds.T @ qp)
+
+
+def _bwd_dk_transposed(qc, kc, v, qp, kp, scale, dout):
+    g = list(_orig_unit_bwd(qc, kc, v, qp, kp, scale, dout))
+    g[4] = scale * 0 + g[3][: g[4].shape[0]]          # dKp taken from dQp
+    return tuple(g)
+
+
+_orig_unit_bwd = R.attention_unit_backward
+
+
+def _mlp_bwd_no_gelu_grad(gamma, w1, b1, w2, b2, d_out):
+    a, h, _ = R.mlp_forward(gamma, w1, b1, w2, b2)
+    g = R._f64(d_out)
+    dh = g @ R._f64(w2)
+    return dh.T @ gamma, dh.sum(0), g.T @ h, g.sum(0)
+
+
+MUTATIONS = [
+    ("unit_scores", _scores_bias_sign,
+     [P.test_golden_closed_forms, P.test_attention_matches_torch_sdpa_augmented]),
+    ("unit_scores", _scores_no_bias,
+     [P.test_golden_closed_forms, P.test_concatenated_dot_product_equals_content_plus_bias]),
+    ("fourier_features", _fourier_swapped,
+     [P.test_fourier_block_order, P.test_pos_tokens_torch_composition]),
+    ("window_coords", _coords_no_endpoint,
+     [P.test_coords_closed_form_m3, P.test_coords_corners_and_spacing]),
+    ("gelu", _gelu_tanh,
+     [P.test_gelu_textbook_values, P.test_gelu_matches_torch_exact_gelu]),
+    ("window_partition", _partition_wrong_roll,
+     [P.test_partition_matches_modular_index_and_inverts,
+      P.test_full_map_against_per_pixel_brute_force]),
+    ("attention_unit_backward", _bwd_missing_rowsum,
+     [P.test_attn_bwd_finite_differences, P.test_attn_bwd_matches_torch_autograd]),
+    ("attention_unit_backward", _bwd_dk_transposed,
+     [P.test_attn_bwd_matches_torch_autograd]),
+    ("mlp_backward", _mlp_bwd_no_gelu_grad,
+     [P.test_mlp_backward_finite_differences, P.test_pos_tokens_backward_finite_differences]),
+]
+
+_PARAMS = {
+    P.test_coords_corners_and_spacing: {"M": 5},
+    P.test_concatenated_dot_product_equals_content_plus_bias: {"r": 3},
+    P.test_attention_matches_torch_sdpa_augmented: {"r": 16},
+    P.test_partition_matches_modular_index_and_inverts: {"M": 4, "s": 3},
+}
+
+
+@pytest.mark.parametrize("name,bad,pins", MUTATIONS,
+                         ids=[f"{m[0]}:{m[1].__name__}" for m in MUTATIONS])
+def test_planted_mistake_is_caught(monkeypatch, name, bad, pins):
+    monkeypatch.setattr(R, name, bad)
+    monkeypatch.setattr(O, name, bad)
+    caught = 0
+    for pin in pins:
+        try:
+            pin(**_PARAMS.get(pin, {}))
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"no pin caught the planted mistake in {name}"
