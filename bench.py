@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Throughput benchmark of RIB window attention on B200.
+
+One step = the whole hot path over one batch of the 96x96-window training
+workload (B=4, 192x192 map, 6 heads, d=32, rank 16, shift 48, MLP
+64->128->96): position tokens -> forward -> backward with position-MLP
+gradients (+ an all-reduce of those gradients across ranks when N > 1).
+Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rib|reference]
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RIB window-attention TFLOP/s and tokens/s (fwd, fwd+bwd) at 96×96 windows"
+D_QK, D_V = 48, 32
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="rib", choices=["rib", "reference"])
+    ap.add_argument("--workload", default="w96train")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def flops(w, layer=0):
+    """Algorithmic FLOPs of one layer: fwd 2N^2(d_qk+d_v), bwd 2N^2(3d_qk+2d_v)
+    per (batch, window, head) unit (the backward counts the score recompute)."""
+    M = w.windows[layer]
+    N = M * M
+    units = w.units(layer)
+    return units * 2.0 * N * N * (D_QK + D_V), units * 2.0 * N * N * (3 * D_QK + 2 * D_V)
+
+
+def workload_desc(w):
+    return (f"{w.name}: B={w.batch} {w.height}x{w.width} map, {w.windows[0]}x{w.windows[0]} windows, "
+            f"shift {w.shifts[0]}, {w.heads} heads, d={w.head_dim}, rank {w.rank}, "
+            f"MLP {4 * w.n_freq}->{w.hidden}->{w.heads * w.rank}, fwd+bwd with MLP grads")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons every 200 ms."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.device_id, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons, pw = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+                pw.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- peaks
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_hash():
+    """Hash of the kernel sources, to tell whether stored ncu counters still
+    describe the kernels being timed."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "windowed_attention_implicit_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it still
+    matches the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- oracle leg
+
+def oracle_sample(w, inputs, rows, unit=(0, 0, 0)):
+    """fp64 oracle fwd+bwd of `rows` query rows of one unit; returns
+    (seconds, algorithmic FLOPs of the sample)."""
+    import numpy as np
+    import oracle as O
+    M, s = w.windows[0], w.shifts[0]
+    b, win, h = unit
+    qp, kp = O.pos_tokens(inputs["freqs"], inputs["mlp_q"], inputs["mlp_k"], M, w.heads, w.rank)
+    qc, kc, v, qpf, kpf = O.gather_unit(inputs["qkv"][b:b + 1], qp, kp, M, s, 0, win, h)
+    dout = O.window_partition(inputs["dout"][b:b + 1].float().numpy(), M, s)[0, win, :, h]
+    sl = slice(0, rows)
+    tau = O.default_scale(w.head_dim, w.rank)
+    t0 = time.perf_counter()
+    O.attention_unit_rows(qc, kc, v, qpf, kpf, tau, rows=sl)
+    g = O.attention_unit_backward(qc[sl], kc, v, qpf[sl], kpf, tau, dout[sl])
+    dt = time.perf_counter() - t0
+    del g
+    N = M * M
+    return dt, 2.0 * rows * N * (D_QK + D_V) + 2.0 * rows * N * (3 * D_QK + 2 * D_V)
+
+
+def oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import rib_inputs as I
+    inputs = I.make_layer_inputs(w, 0)
+    N = w.windows[0] ** 2
+    # size the per-step sample so the whole run stays within a few minutes
+    t256, _ = oracle_sample(w, inputs, 256)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows = int(max(256, min(N, 256 * int(budget / max(t256, 1e-3)))))
+    units = [(b, win, h) for b in range(w.batch) for win in range((w.height // w.windows[0]) *
+                                                                   (w.width // w.windows[0]))
+             for h in range(w.heads)]
+    for i in range(args.warmup):
+        oracle_sample(w, inputs, rows, units[i % len(units)])
+    tot_t = tot_f = 0.0
+    for i in range(args.steps):
+        dt, f = oracle_sample(w, inputs, rows, units[(args.warmup + i) % len(units)])
+        tot_t += dt
+        tot_f += f
+    value = tot_f / tot_t / 1e12
+    cores = oracle_cores()
+    sample = f"{rows} of {N} query rows of one unit per step (fwd+bwd), fp64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "global_batch": w.batch, "window": w.windows[0],
+                   "shift": w.shifts[0], "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def run_rib(args, w):
+    import torch
+    import torch.distributed as dist
+    import rib_inputs as I
+    import windowed_attention_implicit_b200 as R
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    R.library()
+
+    M, s = w.windows[0], w.shifts[0]
+    # each rank trains on its own batch: seeds differ per rank (weak scaling)
+    wr = I.get_workload(w.name, seed=w.seed + 7919 * rank)
+    host = I.make_layer_inputs(wr, 0)
+    mlp = R.PositionMLP.from_params(host["freqs"], host["mlp_q"], host["mlp_k"], w.heads, w.rank,
+                                    device=dev)
+    qkv = host["qkv"].to(dev)
+    dout = host["dout"].to(dev)
+    B, H, W, heads, d = w.batch, w.height, w.width, w.heads, w.head_dim
+    pshape = (heads, M, M, w.rank)
+    qp = torch.empty(pshape, device=dev)
+    kp = torch.empty(pshape, device=dev)
+    q16 = torch.empty(pshape, device=dev, dtype=torch.bfloat16)
+    k16 = torch.empty(pshape, device=dev, dtype=torch.bfloat16)
+    out = torch.empty((B, H, W, heads, d), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((B, heads, H, W), device=dev)
+    dqkv = torch.empty_like(qkv)
+    dqp = torch.empty(pshape, device=dev)
+    dkp = torch.empty(pshape, device=dev)
+    shapes = [t.shape for t in (mlp.q_w1, mlp.q_b1, mlp.q_w2, mlp.q_b2,
+                                mlp.k_w1, mlp.k_b1, mlp.k_w2, mlp.k_b2)]
+    flat = torch.empty(sum(int(torch.Size(sh).numel()) for sh in shapes), device=dev)
+    views, off = [], 0
+    for sh in shapes:
+        n = int(torch.Size(sh).numel())
+        views.append(flat[off:off + n].view(sh))
+        off += n
+    dmlp = R.PositionMLPGrad(*views)
+    ws = torch.empty(R.rib_window_attn_bwd_workspace(B, H, W, heads, d, M, w.rank, mlp),
+                     device=dev, dtype=torch.uint8)
+
+    def step():
+        R.rib_pos_tokens(mlp, M, qp, kp, q16, k16)
+        R.rib_window_attn_fwd(qkv, M, s, q16, k16, out=out, lse=lse)
+        R.rib_window_attn_bwd(qkv, out, dout, lse, M, s, q16, k16, mlp=mlp, dqkv=dqkv,
+                              dqp=dqp, dkp=dkp, dmlp=dmlp, workspace=ws)
+        if world > 1:
+            dist.all_reduce(flat)
+
+    def fwd_only():
+        R.rib_window_attn_fwd(qkv, M, s, q16, k16, out=out, lse=lse)
+
+    def timed(fn, steps, trace=False, sampler=None):
+        stream = torch.cuda.current_stream()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        if trace:
+            R.rib_trace_enable(True)
+        if sampler:
+            sampler.start()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop() if sampler else None
+        kern = R.rib_trace_collect() if trace else None
+        if trace:
+            R.rib_trace_enable(False)
+        ms = a.elapsed_time(b)
+        if world > 1:
+            dist.barrier()
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms, kern, clocks
+
+    for _ in range(args.warmup):
+        step()
+    code, site = R.rib_last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
+    ms, kern, clocks = timed(step, args.steps, trace=True, sampler=sampler)
+    ms_step = ms / args.steps
+    f_fwd, f_bwd = flops(w)
+    value = world * (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
+    tokens_s = world * w.tokens() / (ms_step * 1e-3)
+
+    for _ in range(args.warmup):
+        fwd_only()
+    ms_f, kern_f, _ = timed(fwd_only, args.steps, trace=True)
+    ms_fwd = ms_f / args.steps
+    code, site = R.rib_last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
+
+    pk = peaks()
+    peak = pk["bf16_tflops_sustained"]
+    launches = sum(n for n, _ in kern.values())
+    per_kernel = {k: {"launches": n, "total_ms": t, "avg_ms": t / n,
+                      "share": t / sum(x for _, x in kern.values())} for k, (n, t) in kern.items()}
+    top = max(per_kernel, key=lambda k: per_kernel[k]["total_ms"])
+    kflops = {"attn_bwd_kernel": f_bwd, "attn_fwd_kernel": f_fwd}
+    roof = None
+    if top in kflops:
+        ach = kflops[top] / (per_kernel[top]["avg_ms"] * 1e-3) / 1e12
+        roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "traffic": stored_traffic(top, w.name),
+                "peak_source": f"{pk['source']} bf16_tflops_sustained (kernel inside a long step)"}
+    fwd_k = kern_f.get("attn_fwd_kernel", (1, ms_f))
+    fwd_ach = f_fwd / (fwd_k[1] / fwd_k[0] * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        # same step with the inputs copied from pinned host memory and the
+        # results read back, all inside the timed region
+        h_qkv = host["qkv"].pin_memory()
+        h_dout = host["dout"].pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_dqkv = torch.empty(dqkv.shape, dtype=dqkv.dtype).pin_memory()
+        h_flat = torch.empty(flat.shape, dtype=flat.dtype).pin_memory()
+
+        def e2e_step():
+            qkv.copy_(h_qkv, non_blocking=True)
+            dout.copy_(h_dout, non_blocking=True)
+            step()
+            h_out.copy_(out, non_blocking=True)
+            h_dqkv.copy_(dqkv, non_blocking=True)
+            h_flat.copy_(flat, non_blocking=True)
+
+        for _ in range(max(3, args.warmup // 2)):
+            e2e_step()
+        ms_e, _, _ = timed(e2e_step, args.steps)
+        e_step = ms_e / args.steps
+        nb = lambda t: t.numel() * t.element_size()
+        e2e = {"value": world * (f_fwd + f_bwd) / (e_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_step,
+               "tokens_per_s": world * w.tokens() / (e_step * 1e-3),
+               "h2d_bytes_per_step": nb(h_qkv) + nb(h_dout),
+               "d2h_bytes_per_step": nb(h_out) + nb(h_dqkv) + nb(h_flat)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        N = M * M
+        dt, f = oracle_sample(w, host, N)
+        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_cores(),
+               "kind": "oracle", "seconds": dt,
+               "sample": f"1 of {w.units()} units (batch 0, window 0, head 0), all {N} rows, "
+                         "fwd+bwd, fp64 numpy oracle"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) features and upstream grads, N(0,0.02) MLP weights)",
+        "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
+                   "map": [w.height, w.width], "window": M, "shift": s, "heads": heads,
+                   "head_dim": d, "rank": w.rank, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (qkv 170 MB + dout 57 MB per rank)"},
+        "tokens_per_s": tokens_s,
+        "fwd": {"tflops": world * f_fwd / (ms_fwd * 1e-3) / 1e12, "ms": ms_fwd,
+                "tokens_per_s": world * w.tokens() / (ms_fwd * 1e-3),
+                "kernel_tflops": fwd_ach, "kernel_frac": fwd_ach / peak},
+        "roofline": roof,
+        "kernels": per_kernel,
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "peaks": pk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    import rib_inputs as I
+    w = I.get_workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_rib(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,252 @@
+/*
+ * rib.h -- C ABI of librib.so: RIB windowed attention on NVIDIA B200 (sm_100a).
+ *
+ * RIB (Rank-factorized Implicit Neural Bias) is windowed multi-head
+ * self-attention over image feature maps whose positional bias is the
+ * low-rank product Qp Kp^T.  Qp and Kp come from a Fourier-feature MLP on
+ * window coordinates and are concatenated channel-wise with the content
+ * tokens, so the score [Qc,Qp][Kc,Kp]^T = Qc Kc^T + Qp Kp^T is one dot
+ * product and attention runs flash-style without an N x N score or bias
+ * matrix.  Sources: "Rank-Factorized Implicit Neural Bias: Scaling
+ * Super-Resolution Transformer with FlashAttention" (arXiv 2603.06738) --
+ * its abstract, and the gist.science summaries (English: Technical Summary
+ * §2.A "Rank-Factorized Implicit Neural Bias (RIB)", steps 1-4 and the score
+ * equation; German: Methodik §A; Chinese: 核心方法论 §A).
+ *
+ * Conventions for every entry point
+ *   - Pointers are caller-owned.  Tensor arguments are DEVICE pointers on the
+ *     current CUDA device unless stated otherwise; the library allocates no
+ *     device memory: scratch comes from the caller's workspace.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: a return of RIB_OK means "validated and
+ *     launched".  Faults seen inside kernels (a bounded wait that ran out)
+ *     are recorded in a per-device status word read by rib_last_status().
+ *   - Arguments are validated before anything is launched; on error nothing
+ *     is enqueued and a negative RIB_ERR_* code is returned.  No C++
+ *     exception crosses this boundary.
+ *   - Layouts are row-major, innermost index last.  bf16 = IEEE bfloat16
+ *     stored as 16-bit words; conversion is round-to-nearest-even.
+ *   - Device buffers must be 16-byte aligned (TMA); violations return
+ *     RIB_ERR_ALIGN.
+ *
+ * Notation: B batch, H x W feature map, M window side, N = M*M tokens per
+ * window, nW = (H/M)(W/M) windows, h heads, d = 32 content head dim,
+ * r = 16 (or 0) rank, F Fourier frequencies, s cyclic shift.  A "unit" is
+ * one (batch, window, head) attention problem.
+ *
+ * Window partition with cyclic shift (no region mask): token (i, j) of
+ * window (wy, wx) is map pixel ((wy*M + i + s) mod H, (wx*M + j + s) mod W),
+ * i.e. a roll of the map by -s followed by a partition; outputs are written
+ * back to the same pixels (the inverse roll).
+ */
+#ifndef RIB_H_
+#define RIB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RIB_OK               0
+#define RIB_ERR_ARG         -1  /* null pointer, negative size, bad scalar */
+#define RIB_ERR_SHAPE       -2  /* H % M != 0, W % M != 0, shift outside [0, M) */
+#define RIB_ERR_UNSUPPORTED -3  /* valid but not built: d != 32, r not in {0,16},
+                                   M % 16 != 0, s % 8 != 0, ... */
+#define RIB_ERR_WORKSPACE   -4  /* workspace missing or smaller than required */
+#define RIB_ERR_CUDA        -5  /* a CUDA runtime/driver call failed */
+#define RIB_ERR_TIMEOUT     -6  /* a kernel's bounded wait ran out (status word) */
+#define RIB_ERR_ALIGN       -7  /* a device pointer is not 16-byte aligned */
+
+/* Position-MLP weights (device, fp32, PyTorch Linear layout weight[out][in]).
+ * d_in = 4*n_freq (features [sin(w x), cos(w x), sin(w y), cos(w y)]),
+ * hidden = d_hidden, d_out = heads*rank (output column o = head*rank + r).
+ * Two MLPs of the same shape: q_* gives Qp, k_* gives Kp; passing the same
+ * pointers for both ties them.  freqs[n_freq] are angular frequencies. */
+typedef struct {
+    int n_freq;
+    const float* freqs;
+    int d_hidden;
+    int heads;
+    int rank;
+    const float *q_w1, *q_b1, *q_w2, *q_b2;   /* [hid][4F], [hid], [h*r][hid], [h*r] */
+    const float *k_w1, *k_b1, *k_w2, *k_b2;
+} rib_mlp_t;
+
+/* Gradients of the position MLPs (device, fp32, same shapes as rib_mlp_t). */
+typedef struct {
+    float *q_dw1, *q_db1, *q_dw2, *q_db2;
+    float *k_dw1, *k_db1, *k_dw2, *k_db2;
+} rib_mlp_grad_t;
+
+/* ------------------------------------------------------------------------
+ * rib_pos_tokens -- positional tokens for one window geometry.
+ *
+ * English summary §2.A steps 1-2 (German §A step 1: normalised 2D coordinate
+ * in [-1, 1]; Fourier feature map; lightweight MLP -> low-rank Qp, Kp).
+ * Coordinates are local to the window with endpoints included:
+ * y_i = -1 + 2i/(M-1), x_j = -1 + 2j/(M-1) (M = 1 gives 0).  Hidden layer:
+ * GELU (erf form).  Qp/Kp depend only on the geometry (Chinese summary §A:
+ * precomputed and cached), so one call serves every window, batch entry and
+ * layer with this M and these weights.
+ *
+ *   mlp      : host pointer to the weight struct (device weight pointers)
+ *   window   : M, 1 <= M <= 128
+ *   qp, kp   : out, fp32 [heads][M][M][rank]
+ *   qp_bf16, kp_bf16 : out, bf16 copies of the same shape (may be NULL)
+ * Computes in fp32 (coordinate Fourier features in fp64, rounded to fp32).
+ * ------------------------------------------------------------------------ */
+int rib_pos_tokens(const rib_mlp_t* mlp, int window, float* qp, float* kp,
+                   void* qp_bf16, void* kp_bf16, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rib_pos_tokens_bwd -- backward of rib_pos_tokens: gradients of the two
+ * position MLPs given dL/dQp and dL/dKp (the chain rule through Linear ->
+ * GELU(erf) -> Linear, with the Fourier features recomputed).  Sums over the
+ * M*M tokens run in a fixed order (per-chunk partials, then a chunk sum), so
+ * the result is deterministic.
+ *
+ *   dqp, dkp : fp32 [heads][M][M][rank]
+ *   dmlp     : host pointer to device gradient buffers (fp32, weight shapes)
+ *   workspace: device scratch of rib_pos_tokens_bwd_workspace() bytes,
+ *              256-byte aligned
+ * ------------------------------------------------------------------------ */
+size_t rib_pos_tokens_bwd_workspace(const rib_mlp_t* mlp, int window);
+int rib_pos_tokens_bwd(const rib_mlp_t* mlp, int window, const float* dqp,
+                       const float* dkp, const rib_mlp_grad_t* dmlp,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rib_window_attn_fwd -- RIB window attention forward.
+ *
+ * English summary §2.A steps 3-4 and the score equation; the paper's
+ * abstract (channel-wise concatenation turns the bias addition into a dot
+ * product so FlashAttention-style kernels apply).  Per unit:
+ *   S = scale * [Qc,Qp][Kc,Kp]^T,  P = softmax_rows(S),  O = P V,
+ *   lse = ln sum_k exp(S[:,k]),
+ * computed flash-style (online softmax on tcgen05/TMEM), never forming S.
+ *
+ *   qkv      : bf16 [B][H][W][3][heads][head_dim]  (Qc, Kc, V)
+ *   qp_bf16, kp_bf16 : bf16 [heads][M][M][rank] from rib_pos_tokens
+ *                      (ignored when rank == 0)
+ *   rank     : 0 or 16
+ *   scale    : softmax scale; <= 0 selects 1/sqrt(head_dim + rank)
+ *   out      : bf16 [B][H][W][heads][head_dim]
+ *   lse      : fp32 [B][heads][H][W] (natural log), needed by the backward
+ * Supported: head_dim == 32, M % 16 == 0, 16 <= M <= 128, s % 8 == 0.
+ * ------------------------------------------------------------------------ */
+int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads,
+                        int head_dim, int window, int shift,
+                        const void* qp_bf16, const void* kp_bf16, int rank,
+                        float scale, void* out, float* lse, void* stream);
+
+/* Bytes of device workspace rib_window_attn_bwd needs for these sizes;
+ * `mlp` (host pointer, may be NULL) adds the MLP-gradient scratch. */
+size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads,
+                                     int head_dim, int window, int rank,
+                                     const rib_mlp_t* mlp);
+
+/* ------------------------------------------------------------------------
+ * rib_window_attn_bwd -- RIB window attention backward (+ MLP gradients).
+ *
+ * Gradients of sum(out * dout) for the forward above (training, per the
+ * abstract's training-time claim).  With D = rowsum(dO * O):
+ *   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
+ *   d[Qc,Qp] = scale dS [Kc,Kp],  d[Kc,Kp] = scale dS^T [Qc,Qp].
+ * dqp/dkp are summed over batch entries and windows (the tokens are shared
+ * by every window).  If mlp and dmlp are both non-NULL the position-MLP
+ * weight gradients are computed from dqp/dkp as well (sums over tokens in a
+ * fixed order).
+ *
+ *   qkv, out, lse : as produced for / by rib_window_attn_fwd
+ *   dout     : bf16 [B][H][W][heads][head_dim]
+ *   dqkv     : out, bf16 [B][H][W][3][heads][head_dim]
+ *   dqp, dkp : out, fp32 [heads][M][M][rank] (may be NULL when rank == 0)
+ *   mlp      : host pointer (may be NULL), must match heads/rank
+ *   dmlp     : host pointer to device gradient buffers (may be NULL)
+ *   workspace: device scratch of at least rib_window_attn_bwd_workspace()
+ *              bytes, 256-byte aligned; contents need not be initialised
+ * dQ is accumulated with fp32 atomics across key tiles, so dqkv's query
+ * part and dqp may differ in the last bits between runs.
+ * ------------------------------------------------------------------------ */
+int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout,
+                        const float* lse, int B, int H, int W, int heads,
+                        int head_dim, int window, int shift,
+                        const void* qp_bf16, const void* kp_bf16, int rank,
+                        float scale, void* dqkv, float* dqp, float* dkp,
+                        const rib_mlp_t* mlp, const rib_mlp_grad_t* dmlp,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rib_window_gather / rib_window_scatter -- the window partition with cyclic
+ * shift as a standalone copy (the same rolled TMA tile addressing the
+ * attention kernels use), for bit-exact checks and for callers that want
+ * window-contiguous tensors.
+ *
+ *   x   : [B][H][W][C] elements of elem_bytes (1, 2 or 4) each
+ *   xw  : [B][nW][M*M][C], window index wy*(W/M)+wx, token index i*M+j
+ * gather: xw[b][w][i*M+j] = x[b][(wy*M+i+s) % H][(wx*M+j+s) % W];
+ * scatter writes the inverse.  Requires C*elem_bytes % 16 == 0,
+ * M % 8 == 0, s % 8 == 0.  Pure copies: bit-exact.
+ * ------------------------------------------------------------------------ */
+int rib_window_gather(const void* x, int B, int H, int W, int C,
+                      int elem_bytes, int window, int shift, void* xw,
+                      void* stream);
+int rib_window_scatter(const void* xw, int B, int H, int W, int C,
+                       int elem_bytes, int window, int shift, void* x,
+                       void* stream);
+
+/* ------------------------------------------------------------------------
+ * Status and failure detection.
+ * Every wait inside the kernels (mbarrier phases of the TMA / tensor-core
+ * pipelines) is bounded by a time limit; when it runs out the kernel records
+ * RIB_ERR_TIMEOUT in a per-device status word, drains its in-flight copies
+ * and tensor-core work, frees its tensor memory and returns.
+ * ------------------------------------------------------------------------ */
+
+/* Human-readable name of a status code (static string). */
+const char* rib_status_string(int status);
+
+/* Synchronises the current device, returns the first error recorded by a
+ * kernel since the previous call (RIB_OK if none) and clears it.  If `site`
+ * is non-NULL it receives a code naming the wait that gave up. */
+int rib_last_status(int* site);
+
+/* Time limit, in nanoseconds, of every bounded wait in kernels launched
+ * after this call (process-wide; default 1e9 = 1 s; 0 restores it). */
+int rib_set_wait_limit_ns(unsigned long long limit_ns);
+
+/* Test hook for the failure path: launches one CTA that waits on an
+ * mbarrier nothing will arrive on, with the given limit, using the same
+ * bounded-wait routine as the attention kernels.  The wait runs out and the
+ * kernel records RIB_ERR_TIMEOUT; nothing faults and the context stays
+ * usable. */
+int rib_debug_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Tracing: per-kernel device time measured with CUDA events recorded on
+ * the launch stream around every kernel the library launches.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    const char* kernel;   /* static name */
+    int launches;
+    double total_ms;
+} rib_trace_entry_t;
+
+/* Turns tracing on (1) or off (0) for later launches (process-wide).
+ * Turning it on discards records not yet collected. */
+int rib_trace_enable(int on);
+
+/* Waits for the traced launches, aggregates them per kernel into
+ * entries[0 .. *n_entries) (at most max_entries) and clears the records. */
+int rib_trace_collect(rib_trace_entry_t* entries, int max_entries, int* n_entries);
+
+/* Library version, e.g. "rib-b200 0.1 sm_100a". */
+const char* rib_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RIB_H_ */

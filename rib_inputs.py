@@ -17,10 +17,12 @@ Workloads (the five shapes the benchmark and the parity tests run):
             forward only, one MLP shared by every layer
 
 Recipe: torch CPU generator, randn in fp32, then cast.  Features and upstream
-gradients ~ N(0,1); MLP weights ~ N(0, 0.02), biases 0 (the benchmark recipe);
-a "strong" variant (weights N(0, 0.5), biases N(0, 0.5)) makes the positional
-bias visible against the content scores.  Fourier frequencies default to
-pi*(k+1), k < 16.  Seed: 0 for tiny, the workload's index otherwise, plus
+gradients ~ N(0,1); MLP weights ~ N(0, 0.02), biases 0 (the benchmark recipe).
+With those weights the bias logits are ~1e-4 and invisible, so parity tests
+also use a "strong" variant: weights N(0, (1.5/sqrt(fan_in))^2), biases
+N(0, 0.1^2), which gives Qp/Kp entries of std ~1 and bias logits of std
+~0.65 (max ~6), the size of the content logits (std ~0.8 for N(0,1)
+features, d=32).  Fourier frequencies default to pi*(k+1), k < 16.  Seed: 0 for tiny, the workload's index otherwise, plus
 1000 per layer.
 """
 from __future__ import annotations
@@ -134,15 +136,17 @@ def make_mlp(n_freq, hidden, heads, rank, seed, which, strong=False):
     """Weights of the q (which=0) or k (which=1) position MLP, fp32.
 
     d_in = 4*n_freq, d_out = heads*rank.  Default: weights N(0, 0.02),
-    biases 0.  strong=True: weights and biases N(0, 0.5^2)."""
+    biases 0.  strong=True: weights N(0, (1.5/sqrt(fan_in))^2), biases
+    N(0, 0.1^2)."""
     g = _gen(seed, _TAG_MLPQ if which == 0 else _TAG_MLPK)
     d_in, d_out = 4 * n_freq, heads * rank
-    std = 0.5 if strong else 0.02
-    w1 = torch.randn((hidden, d_in), generator=g) * std
-    w2 = torch.randn((d_out, hidden), generator=g) * std
+    s1 = 1.5 / math.sqrt(d_in) if strong else 0.02
+    s2 = 1.5 / math.sqrt(hidden) if strong else 0.02
+    w1 = torch.randn((hidden, d_in), generator=g) * s1
+    w2 = torch.randn((d_out, hidden), generator=g) * s2
     if strong:
-        b1 = torch.randn((hidden,), generator=g) * std
-        b2 = torch.randn((d_out,), generator=g) * std
+        b1 = torch.randn((hidden,), generator=g) * 0.1
+        b2 = torch.randn((d_out,), generator=g) * 0.1
     else:
         b1 = torch.zeros(hidden)
         b2 = torch.zeros(d_out)

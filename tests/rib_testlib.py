@@ -1,0 +1,94 @@
+"""Shared helpers of the parity tests: inputs, oracle runs, comparisons.
+
+Inputs come from rib_inputs (seeded); expected values only from oracle/.
+The attention parity cases feed both sides the same bf16-rounded Qp/Kp (the
+oracle computes them in fp64, the host rounds them), so each kernel is
+compared on exactly the values it consumes.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+import rib_inputs as I
+
+MAX_ABS = 2e-2     # outputs and gradients, bf16 in / fp32 accumulate
+MEAN_ABS = 2e-3
+POS_REL = 1e-5     # Qp/Kp fp32: max|d| / max|ref|
+
+
+def stats(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    d = np.abs(got - ref)
+    return float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0
+
+
+def check_close(got, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS, normalize=False):
+    """Returns an error message ('' if within bounds).  normalize=True divides
+    the errors by max(1, max|ref|) first (used for fp32 sums whose magnitude
+    grows with the number of tokens summed)."""
+    mx, mn = stats(got, ref)
+    scale = max(1.0, float(np.abs(np.asarray(ref, dtype=np.float64)).max())) if normalize else 1.0
+    ok = mx / scale <= max_abs and mn / scale <= mean_abs
+    msg = (f"{what}: max|d|={mx:.3e}, mean|d|={mn:.3e}, max|ref|="
+           f"{float(np.abs(np.asarray(ref, dtype=np.float64)).max()):.3e}"
+           f"{' (normalised by %.3e)' % scale if normalize else ''} bounds {max_abs}/{mean_abs}")
+    print(msg)
+    return "" if ok else msg
+
+
+def assert_close(got, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS, normalize=False):
+    msg = check_close(got, ref, what, max_abs, mean_abs, normalize)
+    assert not msg, msg
+
+
+def assert_all(checks):
+    """checks: list of messages from check_close; fails listing every miss."""
+    bad = [c for c in checks if c]
+    assert not bad, "; ".join(bad)
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def bf16_round(a) -> torch.Tensor:
+    return torch.as_tensor(np.asarray(a), dtype=torch.float64).to(torch.bfloat16)
+
+
+class Case:
+    """One attention problem: host inputs, their device copies and the
+    oracle's position tokens."""
+
+    def __init__(self, B, H, W, heads, M, s, rank=16, hidden=64, F=16, seed=0,
+                 strong=True, qkv_std=1.0):
+        self.B, self.H, self.W, self.heads, self.M, self.s, self.rank = B, H, W, heads, M, s, rank
+        self.d = 32
+        self.qkv = I.make_qkv(B, H, W, heads, 32, seed, std=qkv_std)
+        self.dout = I.make_dout(B, H, W, heads, 32, seed)
+        self.freqs = I.default_freqs(F)
+        r = max(rank, 1)
+        self.mlp_q = I.make_mlp(F, hidden, heads, r, seed, 0, strong=strong)
+        self.mlp_k = I.make_mlp(F, hidden, heads, r, seed, 1, strong=strong)
+        if rank > 0:
+            qp, kp = O.pos_tokens(self.freqs, self.mlp_q, self.mlp_k, M, heads, rank)
+            self.qp16, self.kp16 = bf16_round(qp), bf16_round(kp)
+        else:
+            self.qp16 = torch.zeros((heads, M, M, 0), dtype=torch.bfloat16)
+            self.kp16 = torch.zeros((heads, M, M, 0), dtype=torch.bfloat16)
+        self.scale = O.default_scale(32, rank)
+
+    def device(self):
+        dev = "cuda"
+        return dict(qkv=self.qkv.to(dev), dout=self.dout.to(dev),
+                    qp16=self.qp16.to(dev) if self.rank else None,
+                    kp16=self.kp16.to(dev) if self.rank else None)
+
+    def oracle_fwd(self):
+        return O.attn_fwd(self.qkv, self.M, self.s, self.qp16, self.kp16, self.scale)
+
+    def oracle_bwd(self, units=None):
+        return O.attn_bwd(self.qkv, self.dout, self.M, self.s, self.qp16, self.kp16,
+                          self.scale, units=units)

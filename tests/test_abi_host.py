@@ -1,0 +1,130 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import windowed_attention_implicit_b200 as R
+from windowed_attention_implicit_b200 import _abi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "rib.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rib_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("rib_pos_tokens", "rib_window_attn_fwd", "rib_window_attn_bwd",
+              "rib_window_attn_bwd_workspace", "rib_last_status", "rib_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = R.library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _abi._SIGS, f"{name} has no ctypes signature"
+
+
+def test_status_strings():
+    lib = R.library()
+    for code, name in ((0, "RIB_OK"), (-1, "RIB_ERR_ARG"), (-2, "RIB_ERR_SHAPE"),
+                       (-3, "RIB_ERR_UNSUPPORTED"), (-4, "RIB_ERR_WORKSPACE"),
+                       (-5, "RIB_ERR_CUDA"), (-6, "RIB_ERR_TIMEOUT"), (-7, "RIB_ERR_ALIGN")):
+        assert lib.rib_status_string(code).decode() == name
+    assert R.rib_version().startswith("rib-b200")
+
+
+FAKE = 1 << 20        # 16-byte-aligned non-null stand-in; never dereferenced
+
+
+def fwd(**kw):
+    a = dict(qkv=FAKE, B=1, H=64, W=64, heads=2, d=32, M=16, s=0, qp=FAKE, kp=FAKE, r=16,
+             scale=0.0, out=FAKE, lse=FAKE)
+    a.update(kw)
+    return R.library().rib_window_attn_fwd(
+        a["qkv"], a["B"], a["H"], a["W"], a["heads"], a["d"], a["M"], a["s"], a["qp"],
+        a["kp"], a["r"], a["scale"], a["out"], a["lse"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qkv=None), _abi.RIB_ERR_ARG),
+    (dict(B=0), _abi.RIB_ERR_ARG),
+    (dict(H=0), _abi.RIB_ERR_ARG),
+    (dict(H=72), _abi.RIB_ERR_SHAPE),
+    (dict(W=40), _abi.RIB_ERR_SHAPE),
+    (dict(s=16), _abi.RIB_ERR_SHAPE),
+    (dict(s=-8), _abi.RIB_ERR_SHAPE),
+    (dict(d=64), _abi.RIB_ERR_UNSUPPORTED),
+    (dict(r=8), _abi.RIB_ERR_UNSUPPORTED),
+    (dict(M=8, H=64, W=64), _abi.RIB_ERR_UNSUPPORTED),
+    (dict(s=4), _abi.RIB_ERR_UNSUPPORTED),
+    (dict(qp=None), _abi.RIB_ERR_ARG),
+    (dict(out=FAKE + 8), _abi.RIB_ERR_ALIGN),
+    (dict(scale=float("nan")), _abi.RIB_ERR_ARG),
+])
+def test_fwd_validation(kw, code):
+    assert fwd(**kw) == code
+
+
+def test_fwd_rank0_needs_no_position_tokens():
+    # rank 0 with null Qp/Kp passes validation; stop it at the alignment check
+    assert fwd(r=0, qp=None, kp=None, lse=FAKE + 4) == _abi.RIB_ERR_ALIGN
+
+
+def test_bwd_workspace_sizes():
+    ws = R.rib_window_attn_bwd_workspace
+    B, H, W, h = 4, 192, 192, 6
+    pix = B * h * H * W
+    a = lambda x: (x + 255) // 256 * 256
+    expect = a(pix * 4) * 2 + a(pix * 48 * 4) + a(pix * 16 * 4)
+    assert ws(B, H, W, h, 32, 96, 16) == expect
+    assert ws(B, H, W, h, 32, 96, 0) == a(pix * 4) * 2 + a(pix * 48 * 4)
+    assert ws(B, H, W, h, 64, 96, 16) == 0          # unsupported -> 0
+    assert ws(B, 100, W, h, 32, 96, 16) == 0        # bad shape -> 0
+
+
+def test_bwd_validation():
+    lib = R.library()
+    def call(ws_bytes=1 << 40, **kw):
+        a = dict(M=16, s=0, r=16, d=32, dqp=FAKE, ws=FAKE * 256)
+        a.update(kw)
+        return lib.rib_window_attn_bwd(FAKE, FAKE, FAKE, FAKE, 1, 64, 64, 2, a["d"], a["M"],
+                                       a["s"], FAKE, FAKE, a["r"], 0.0, FAKE, a["dqp"], FAKE,
+                                       None, None, a["ws"], ws_bytes, None)
+    assert call(ws_bytes=16) == _abi.RIB_ERR_WORKSPACE
+    assert call(ws=None) == _abi.RIB_ERR_WORKSPACE
+    assert call(dqp=None) == _abi.RIB_ERR_ARG
+    assert call(M=24) == _abi.RIB_ERR_SHAPE
+    assert call(d=16) == _abi.RIB_ERR_UNSUPPORTED
+    assert call(ws=FAKE * 256 + 16) == _abi.RIB_ERR_ALIGN
+
+
+def test_gather_validation():
+    lib = R.library()
+    g = lambda **kw: lib.rib_window_gather(
+        kw.get("x", FAKE), 1, kw.get("H", 64), kw.get("W", 64), kw.get("C", 8), kw.get("eb", 2),
+        kw.get("M", 16), kw.get("s", 0), FAKE, None)
+    assert g(x=None) == _abi.RIB_ERR_ARG
+    assert g(eb=3) == _abi.RIB_ERR_ARG
+    assert g(H=40) == _abi.RIB_ERR_SHAPE
+    assert g(C=4) == _abi.RIB_ERR_UNSUPPORTED        # 8 bytes per pixel row
+    assert g(s=4) == _abi.RIB_ERR_UNSUPPORTED
+    assert g(M=12, H=48, W=48) == _abi.RIB_ERR_UNSUPPORTED
+
+
+def test_pos_tokens_validation():
+    lib = R.library()
+    m = _abi.rib_mlp_t(16, FAKE, 64, 3, 16, *([FAKE] * 8))
+    assert lib.rib_pos_tokens(None, 16, FAKE, FAKE, None, None, None) == _abi.RIB_ERR_ARG
+    assert lib.rib_pos_tokens(ctypes.byref(m), 0, FAKE, FAKE, None, None, None) == _abi.RIB_ERR_ARG
+    assert lib.rib_pos_tokens(ctypes.byref(m), 16, None, FAKE, None, None, None) == _abi.RIB_ERR_ARG
+    m.n_freq = 0
+    assert lib.rib_pos_tokens(ctypes.byref(m), 16, FAKE, FAKE, None, None, None) == _abi.RIB_ERR_ARG

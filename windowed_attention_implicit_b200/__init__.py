@@ -1,0 +1,314 @@
+"""RIB windowed attention on B200 (sm_100a): Python binding of librib.so.
+
+Every function here has the name of a C entry point of include/rib.h and only
+marshals arguments: it checks devices / dtypes / contiguity, allocates
+missing outputs with torch (PyTorch is the device-memory and stream
+provider), passes raw pointers and the current CUDA stream, and raises
+RibError on a non-zero status.  All arithmetic runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback.
+
+"Rank-Factorized Implicit Neural Bias: Scaling Super-Resolution Transformer
+with FlashAttention" (arXiv 2603.06738): position tokens from a Fourier-
+feature MLP on window coordinates are concatenated with the content tokens so
+that the positional bias Qp Kp^T comes out of the attention dot product.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Dict, Optional, Tuple
+
+import torch
+
+from . import _abi
+
+__all__ = [
+    "RibError", "PositionMLP", "PositionMLPGrad", "PosTokenCache", "rib_pos_tokens",
+    "rib_pos_tokens_bwd", "rib_pos_tokens_bwd_workspace",
+    "rib_window_attn_fwd", "rib_window_attn_bwd", "rib_window_attn_bwd_workspace",
+    "rib_window_gather", "rib_window_scatter", "rib_last_status", "rib_status_string",
+    "rib_set_wait_limit_ns", "rib_debug_wait_timeout", "rib_version", "library",
+    "rib_trace_enable", "rib_trace_collect",
+]
+
+
+class RibError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {rib_status_string(code)} ({code})")
+
+
+def library() -> ctypes.CDLL:
+    return _abi.load()
+
+
+def _check(code: int, where: str) -> None:
+    if code != _abi.RIB_OK:
+        raise RibError(code, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def rib_status_string(code: int) -> str:
+    return library().rib_status_string(int(code)).decode()
+
+
+def rib_version() -> str:
+    return library().rib_version().decode()
+
+
+# ---------------------------------------------------------------- MLP weights
+
+@dataclass
+class PositionMLP:
+    """Device fp32 weights of the two position MLPs (Linear layout [out][in])."""
+    freqs: torch.Tensor
+    q_w1: torch.Tensor
+    q_b1: torch.Tensor
+    q_w2: torch.Tensor
+    q_b2: torch.Tensor
+    k_w1: torch.Tensor
+    k_b1: torch.Tensor
+    k_w2: torch.Tensor
+    k_b2: torch.Tensor
+    heads: int
+    rank: int
+
+    @property
+    def n_freq(self) -> int:
+        return self.freqs.numel()
+
+    @property
+    def hidden(self) -> int:
+        return self.q_w1.shape[0]
+
+    @classmethod
+    def from_params(cls, freqs, mlp_q, mlp_k, heads, rank, device="cuda"):
+        """From host tensors (anything with w1, b1, w2, b2)."""
+        f = lambda t: t.detach().to(device=device, dtype=torch.float32).contiguous()
+        return cls(f(freqs), f(mlp_q.w1), f(mlp_q.b1), f(mlp_q.w2), f(mlp_q.b2),
+                   f(mlp_k.w1), f(mlp_k.b1), f(mlp_k.w2), f(mlp_k.b2), heads, rank)
+
+    def c_struct(self) -> _abi.rib_mlp_t:
+        p = lambda t, n: _ptr(t, torch.float32, n)
+        return _abi.rib_mlp_t(
+            self.n_freq, p(self.freqs, "freqs"), self.hidden, self.heads, self.rank,
+            p(self.q_w1, "q_w1"), p(self.q_b1, "q_b1"), p(self.q_w2, "q_w2"),
+            p(self.q_b2, "q_b2"), p(self.k_w1, "k_w1"), p(self.k_b1, "k_b1"),
+            p(self.k_w2, "k_w2"), p(self.k_b2, "k_b2"))
+
+    def key(self) -> Tuple[int, ...]:
+        return tuple(t.data_ptr() for t in (self.freqs, self.q_w1, self.q_w2, self.k_w1,
+                                            self.k_w2))
+
+
+@dataclass
+class PositionMLPGrad:
+    q_dw1: torch.Tensor
+    q_db1: torch.Tensor
+    q_dw2: torch.Tensor
+    q_db2: torch.Tensor
+    k_dw1: torch.Tensor
+    k_db1: torch.Tensor
+    k_dw2: torch.Tensor
+    k_db2: torch.Tensor
+
+    @classmethod
+    def empty_like(cls, mlp: PositionMLP):
+        e = torch.empty_like
+        return cls(e(mlp.q_w1), e(mlp.q_b1), e(mlp.q_w2), e(mlp.q_b2),
+                   e(mlp.k_w1), e(mlp.k_b1), e(mlp.k_w2), e(mlp.k_b2))
+
+    def c_struct(self) -> _abi.rib_mlp_grad_t:
+        return _abi.rib_mlp_grad_t(*[_ptr(getattr(self, n), torch.float32, n) for n in (
+            "q_dw1", "q_db1", "q_dw2", "q_db2", "k_dw1", "k_db1", "k_dw2", "k_db2")])
+
+    def tensors(self) -> Dict[str, torch.Tensor]:
+        return dict(self.__dict__)
+
+
+# ---------------------------------------------------------------- entry points
+
+def rib_pos_tokens(mlp: PositionMLP, window: int, qp=None, kp=None, qp_bf16=None,
+                   kp_bf16=None, stream=None, with_bf16: bool = True):
+    """Qp, Kp fp32 [heads][M][M][rank] (+ bf16 copies) for one window size."""
+    shape = (mlp.heads, window, window, mlp.rank)
+    dev = mlp.freqs.device
+    qp = torch.empty(shape, device=dev, dtype=torch.float32) if qp is None else qp
+    kp = torch.empty(shape, device=dev, dtype=torch.float32) if kp is None else kp
+    if with_bf16:
+        qp_bf16 = torch.empty(shape, device=dev, dtype=torch.bfloat16) if qp_bf16 is None else qp_bf16
+        kp_bf16 = torch.empty(shape, device=dev, dtype=torch.bfloat16) if kp_bf16 is None else kp_bf16
+    c = mlp.c_struct()
+    _check(library().rib_pos_tokens(
+        ctypes.byref(c), int(window), _ptr(qp, torch.float32, "qp"), _ptr(kp, torch.float32, "kp"),
+        _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
+        _stream(stream)), "rib_pos_tokens")
+    return qp, kp, qp_bf16, kp_bf16
+
+
+def rib_pos_tokens_bwd_workspace(mlp: PositionMLP, window: int) -> int:
+    c = mlp.c_struct()
+    return int(library().rib_pos_tokens_bwd_workspace(ctypes.byref(c), int(window)))
+
+
+def rib_pos_tokens_bwd(mlp: PositionMLP, window: int, dqp: torch.Tensor, dkp: torch.Tensor,
+                       dmlp: Optional["PositionMLPGrad"] = None, workspace=None, stream=None):
+    """Position-MLP gradients from dL/dQp, dL/dKp ([heads][M][M][rank] fp32)."""
+    dmlp = PositionMLPGrad.empty_like(mlp) if dmlp is None else dmlp
+    need = rib_pos_tokens_bwd_workspace(mlp, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=dqp.device, dtype=torch.uint8)
+    c, cg = mlp.c_struct(), dmlp.c_struct()
+    _check(library().rib_pos_tokens_bwd(
+        ctypes.byref(c), int(window), _ptr(dqp, torch.float32, "dqp"),
+        _ptr(dkp, torch.float32, "dkp"), ctypes.byref(cg), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "rib_pos_tokens_bwd")
+    return dmlp
+
+
+def rib_window_attn_fwd(qkv: torch.Tensor, window: int, shift: int, qp_bf16=None,
+                        kp_bf16=None, rank: int = 16, scale: float = 0.0, out=None, lse=None,
+                        stream=None):
+    """out bf16 [B][H][W][heads][d], lse fp32 [B][heads][H][W]."""
+    B, H, W, three, heads, d = qkv.shape
+    if three != 3:
+        raise ValueError("qkv must be [B][H][W][3][heads][head_dim]")
+    out = torch.empty((B, H, W, heads, d), device=qkv.device, dtype=torch.bfloat16) if out is None else out
+    lse = torch.empty((B, heads, H, W), device=qkv.device, dtype=torch.float32) if lse is None else lse
+    _check(library().rib_window_attn_fwd(
+        _ptr(qkv, torch.bfloat16, "qkv"), B, H, W, heads, d, int(window), int(shift),
+        _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
+        int(rank), float(scale), _ptr(out, torch.bfloat16, "out"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream)), "rib_window_attn_fwd")
+    return out, lse
+
+
+def rib_window_attn_bwd_workspace(B, H, W, heads, head_dim, window, rank,
+                                  mlp: Optional[PositionMLP] = None) -> int:
+    c = mlp.c_struct() if mlp is not None else None
+    return int(library().rib_window_attn_bwd_workspace(
+        B, H, W, heads, head_dim, int(window), int(rank),
+        ctypes.byref(c) if c is not None else None))
+
+
+def rib_window_attn_bwd(qkv, out, dout, lse, window: int, shift: int, qp_bf16=None,
+                        kp_bf16=None, rank: int = 16, scale: float = 0.0,
+                        mlp: Optional[PositionMLP] = None, dqkv=None, dqp=None, dkp=None,
+                        dmlp: Optional[PositionMLPGrad] = None, workspace=None, stream=None):
+    """Returns dict(dqkv, dqp, dkp, dmlp).  dmlp is computed when mlp is given."""
+    B, H, W, _, heads, d = qkv.shape
+    dev = qkv.device
+    dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
+    if rank > 0:
+        pshape = (heads, window, window, rank)
+        dqp = torch.empty(pshape, device=dev, dtype=torch.float32) if dqp is None else dqp
+        dkp = torch.empty(pshape, device=dev, dtype=torch.float32) if dkp is None else dkp
+    if mlp is not None and dmlp is None:
+        dmlp = PositionMLPGrad.empty_like(mlp)
+    need = rib_window_attn_bwd_workspace(B, H, W, heads, d, window, rank, mlp)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
+    c_mlp = mlp.c_struct() if mlp is not None else None
+    c_dmlp = dmlp.c_struct() if (mlp is not None and dmlp is not None) else None
+    _check(library().rib_window_attn_bwd(
+        _ptr(qkv, torch.bfloat16, "qkv"), _ptr(out, torch.bfloat16, "out"),
+        _ptr(dout, torch.bfloat16, "dout"), _ptr(lse, torch.float32, "lse"),
+        B, H, W, heads, d, int(window), int(shift),
+        _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
+        int(rank), float(scale), _ptr(dqkv, torch.bfloat16, "dqkv"),
+        _ptr(dqp, torch.float32, "dqp"), _ptr(dkp, torch.float32, "dkp"),
+        ctypes.byref(c_mlp) if c_mlp is not None else None,
+        ctypes.byref(c_dmlp) if c_dmlp is not None else None,
+        _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "rib_window_attn_bwd")
+    return {"dqkv": dqkv, "dqp": dqp, "dkp": dkp, "dmlp": dmlp}
+
+
+def rib_window_gather(x: torch.Tensor, window: int, shift: int, out=None, stream=None):
+    """x [B][H][W][C] -> [B][nW][M*M][C] (roll by -shift, partition)."""
+    B, H, W, C = x.shape
+    nW = (H // window) * (W // window)
+    out = torch.empty((B, nW, window * window, C), device=x.device, dtype=x.dtype) if out is None else out
+    _check(library().rib_window_gather(
+        _ptr(x, None, "x"), B, H, W, C, x.element_size(), int(window), int(shift),
+        _ptr(out, x.dtype, "out"), _stream(stream)), "rib_window_gather")
+    return out
+
+
+def rib_window_scatter(xw: torch.Tensor, H: int, W: int, window: int, shift: int, out=None,
+                       stream=None):
+    """Inverse of rib_window_gather."""
+    B, nW, N, C = xw.shape
+    out = torch.empty((B, H, W, C), device=xw.device, dtype=xw.dtype) if out is None else out
+    _check(library().rib_window_scatter(
+        _ptr(xw, None, "xw"), B, H, W, C, xw.element_size(), int(window), int(shift),
+        _ptr(out, xw.dtype, "out"), _stream(stream)), "rib_window_scatter")
+    return out
+
+
+def rib_last_status() -> Tuple[int, int]:
+    site = ctypes.c_int(0)
+    code = library().rib_last_status(ctypes.byref(site))
+    return int(code), int(site.value)
+
+
+def rib_set_wait_limit_ns(limit_ns: int) -> None:
+    _check(library().rib_set_wait_limit_ns(int(limit_ns)), "rib_set_wait_limit_ns")
+
+
+def rib_debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(library().rib_debug_wait_timeout(int(limit_ns), _stream(stream)),
+           "rib_debug_wait_timeout")
+
+
+def rib_trace_enable(on: bool = True) -> None:
+    _check(library().rib_trace_enable(1 if on else 0), "rib_trace_enable")
+
+
+def rib_trace_collect() -> Dict[str, Tuple[int, float]]:
+    """{kernel: (launches, total_ms)} of the launches traced since enabling."""
+    entries = (_abi.rib_trace_entry_t * 32)()
+    n = ctypes.c_int(0)
+    _check(library().rib_trace_collect(ctypes.cast(entries, ctypes.c_void_p), 32,
+                                       ctypes.byref(n)), "rib_trace_collect")
+    return {entries[i].kernel.decode(): (int(entries[i].launches), float(entries[i].total_ms))
+            for i in range(n.value)}
+
+
+# ---------------------------------------------------------------- geometry cache
+
+class PosTokenCache:
+    """Qp/Kp per window geometry, computed once and reused across windows,
+    batch entries and layers (they depend only on the geometry and the MLP)."""
+
+    def __init__(self):
+        self._cache = {}
+
+    def get(self, mlp: PositionMLP, window: int, stream=None):
+        k = (mlp.key(), int(window))
+        if k not in self._cache:
+            self._cache[k] = rib_pos_tokens(mlp, window, stream=stream)
+        return self._cache[k]
+
+    def clear(self):
+        self._cache.clear()
+
+    def __len__(self):
+        return len(self._cache)

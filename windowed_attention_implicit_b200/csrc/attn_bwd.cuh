@@ -1,0 +1,569 @@
+// attn_bwd.cuh -- RIB window attention backward on tcgen05 tensor cores.
+//
+// Gradients of the forward in attn_fwd.cuh (the augmented score of the
+// English summary §2.A, score equation).  With P = softmax(S),
+// S = tau [Qc,Qp][Kc,Kp]^T and D = rowsum(dO * O):
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
+//   d[Qc,Qp] = tau dS [Kc,Kp],  d[Kc,Kp] = tau dS^T [Qc,Qp].
+// The positional parts dQp, dKp are summed over batch entries and windows
+// because one Qp/Kp set serves every window of the geometry.
+//
+// Kernels, in launch order:
+//   bwd_preprocess   D and lse*log2(e) per pixel and head; zeroes dQ acc
+//   attn_bwd_kernel  one CTA per (key tile, unit): keeps K, V, Kp of its 128
+//                    keys in shared memory and streams the unit's query
+//                    tiles; dK, dV accumulate in TMEM; dQ partials go to an
+//                    fp32 accumulator with vector atomics
+//   dq_finalize      dQ content channels -> bf16 dqkv at the rolled pixels
+//   posgrad_reduce   fixed-order sums over (batch, window) of dQp, dKp
+//
+// attn_bwd_kernel, 320 threads:
+//   warps 0-7  compute: thread = key row (TMEM lane), warps 0-3 take query
+//              columns 0-63 and warps 4-7 columns 64-127 of each tile
+//   warp  8    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 2 stages)
+//   warp  9    TMEM allocator and MMA issuer
+// Per query tile i:  S^T = K_aug Q_aug^T and dP^T = V dO^T (MMA, TMEM) ->
+// compute warps form P^T (to TMEM) and dS^T (to shared memory, core-matrix
+// layout readable both K-major and MN-major) -> MMA: dV += P^T dO (A from
+// TMEM), dK_aug += dS^T Q_aug, dQ_aug = dS K_aug (double-buffered TMEM) ->
+// compute warps drain dQ with red.global.add.v4.f32.
+// S/dP of tile i+1 are issued as soon as the compute warps have pulled tile
+// i into registers, so the MMAs overlap the exponentials.
+#pragma once
+
+#include "geom.cuh"
+#include "ptx.cuh"
+
+namespace rib {
+
+constexpr int kBwdStages = 2;
+constexpr int kBwdThreads = 320;
+constexpr uint32_t kBwdTmemCols = 512;
+// TMEM columns
+constexpr uint32_t kBColS = 0, kBColDP = 128, kBColP = 256, kBColDV = 320, kBColDKc = 352,
+                   kBColDQc = 384 /* +32 per buffer */, kBColDKp = 448,
+                   kBColDQp = 464 /* +16 per buffer */;
+constexpr uint64_t kBwdDrainNs = 200ull * 1000ull * 1000ull;
+
+struct BwdParams {
+  int B, H, W, heads, M, s, rank, nWx, nW, tiles_x, n_tiles;
+  float scale;       // tau
+  float scale_log2;  // tau * log2(e)
+  __nv_bfloat16* dqkv;
+  float* dq_acc;     // [units][n_tiles][128][48]
+  float* dkp_part;   // [units][n_tiles][128][16]
+  uint64_t wait_limit_ns;
+};
+
+struct __align__(1024) BwdSmem {
+  uint8_t kc[8192];                // key tile, content, 64B swizzle
+  uint8_t v[8192];
+  uint8_t ds[32768];               // dS^T [128 keys x 128 queries] bf16, core matrices
+  uint8_t qc[kBwdStages][8192];
+  uint8_t dO[kBwdStages][8192];
+  uint8_t kp[4096];                // key tile, positional, 32B swizzle
+  uint8_t qp[kBwdStages][4096];
+  float lse2[kBwdStages][128];     // lse * log2(e), tile row order
+  float dd[kBwdStages][128];       // D = rowsum(dO * O), tile row order
+  uint64_t k_full;
+  uint64_t q_full[kBwdStages], q_empty[kBwdStages];
+  uint64_t s_full, s_free, ds_full, ds_free;
+  uint64_t dq_full[2], dq_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t kBwdSmemBytes = sizeof(BwdSmem) + 1024;
+
+constexpr uint32_t kIdescBS = make_idesc_bf16(128, 128, false, false);   // S^T, dP^T
+constexpr uint32_t kIdescBN32 = make_idesc_bf16(128, 32, false, true);   // dV, dKc
+constexpr uint32_t kIdescBN16 = make_idesc_bf16(128, 16, false, true);   // dKp
+constexpr uint32_t kIdescBQ32 = make_idesc_bf16(128, 32, true, true);    // dQc
+constexpr uint32_t kIdescBQ16 = make_idesc_bf16(128, 16, true, true);    // dQp
+
+// Byte offset of element (key k, query q) of dS^T: 8 x 8 core matrices of
+// 128 contiguous bytes; key groups of 8 every 128 B, query groups of 8
+// every 2048 B.
+__device__ __forceinline__ uint32_t ds_offset(int k, int q) {
+  return static_cast<uint32_t>((q >> 3) * 2048 + (k >> 3) * 128 + (k & 7) * 16 + (q & 7) * 2);
+}
+
+__device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
+                                             const CUtensorMap* tdo, const CUtensorMap* tqp,
+                                             const CUtensorMap* tkp, const CUtensorMap* tlse2,
+                                             const CUtensorMap* tdd, const BwdParams& p,
+                                             const UnitCoord& u, int kt) {
+  volatile int* ab = &sm.abort_flag;
+  const int hh = u.head;
+  const int by = u.wy * p.M + p.s, bx = u.wx * p.M + p.s;
+  const bool pos = p.rank > 0;
+  {
+    int i0, j0;
+    tile_origin(kt, p.tiles_x, i0, j0);
+    const int y = wrap_once(by + i0, p.H);
+    mbar_arrive_expect_tx(&sm.k_full, 2u * 8192u + (pos ? 4096u : 0u));
+    for (int c = 0; c < 2; ++c) {
+      const int x = wrap_once(bx + j0 + 8 * c, p.W);
+      tma_load_5d(sm.kc + c * 4096, tq, &sm.k_full, 0, p.heads + hh, x, y, u.b);
+      tma_load_5d(sm.v + c * 4096, tq, &sm.k_full, 0, 2 * p.heads + hh, x, y, u.b);
+      if (pos) tma_load_4d(sm.kp + c * 2048, tkp, &sm.k_full, 0, j0 + 8 * c, i0, hh);
+    }
+  }
+  const uint32_t q_bytes = 2u * 8192u + (pos ? 4096u : 0u) + 2u * 512u;
+  int i = 0;
+  for (; i < p.n_tiles; ++i) {
+    const int st = i % kBwdStages, use = i / kBwdStages;
+    if (use > 0 &&
+        !mbar_wait(&sm.q_empty[st], (use - 1) & 1, ab, p.wait_limit_ns, SITE_BWD_PRODUCER))
+      break;
+    mbar_arrive_expect_tx(&sm.q_full[st], q_bytes);
+    int i0, j0;
+    tile_origin(i, p.tiles_x, i0, j0);
+    const int y = wrap_once(by + i0, p.H);
+    for (int c = 0; c < 2; ++c) {
+      const int x = wrap_once(bx + j0 + 8 * c, p.W);
+      tma_load_5d(sm.qc[st] + c * 4096, tq, &sm.q_full[st], 0, hh, x, y, u.b);
+      tma_load_5d(sm.dO[st] + c * 4096, tdo, &sm.q_full[st], 0, hh, x, y, u.b);
+      if (pos) tma_load_4d(sm.qp[st] + c * 2048, tqp, &sm.q_full[st], 0, j0 + 8 * c, i0, hh);
+      tma_load_4d(&sm.lse2[st][c * 64], tlse2, &sm.q_full[st], x, y, hh, u.b);
+      tma_load_4d(&sm.dd[st][c * 64], tdd, &sm.q_full[st], x, y, hh, u.b);
+    }
+  }
+  if (*ab) {
+    volatile int no_abort = 0;
+    mbar_wait(&sm.k_full, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
+    for (int ii = i - 1; ii >= 0 && ii >= i - kBwdStages; --ii)
+      mbar_wait(&sm.q_full[ii % kBwdStages], (ii / kBwdStages) & 1, &no_abort, kBwdDrainNs,
+                SITE_BWD_DRAIN);
+  }
+}
+
+__device__ __forceinline__ void bwd_mma(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
+  volatile int* ab = &sm.abort_flag;
+  const uint64_t lim = p.wait_limit_ns;
+  const bool pos = p.rank > 0;
+  const int n = p.n_tiles;
+  const uint32_t kc = smem_u32(sm.kc), v = smem_u32(sm.v), kp = smem_u32(sm.kp),
+                 ds = smem_u32(sm.ds);
+  auto issue_s_dp = [&](int st) {
+    // S^T = K_aug Q_aug^T  (M = keys, N = queries, K = 32 + 16)
+    const uint64_t a = make_sdesc(kc, 16, 512, kLayoutSW64);
+    const uint64_t b = make_sdesc(smem_u32(sm.qc[st]), 16, 512, kLayoutSW64);
+    umma_ss(tmem + kBColS, a, b, kIdescBS, 0u);
+    umma_ss(tmem + kBColS, a + 2, b + 2, kIdescBS, 1u);
+    if (pos)
+      umma_ss(tmem + kBColS, make_sdesc(kp, 16, 256, kLayoutSW32),
+              make_sdesc(smem_u32(sm.qp[st]), 16, 256, kLayoutSW32), kIdescBS, 1u);
+    // dP^T = V dO^T  (M = keys, N = queries, K = 32)
+    const uint64_t av = make_sdesc(v, 16, 512, kLayoutSW64);
+    const uint64_t bo = make_sdesc(smem_u32(sm.dO[st]), 16, 512, kLayoutSW64);
+    umma_ss(tmem + kBColDP, av, bo, kIdescBS, 0u);
+    umma_ss(tmem + kBColDP, av + 2, bo + 2, kIdescBS, 1u);
+    umma_commit(&sm.s_full);
+  };
+  bool ok = mbar_wait(&sm.k_full, 0, ab, lim, SITE_BWD_MMA) &&
+            mbar_wait(&sm.q_full[0], 0, ab, lim, SITE_BWD_MMA);
+  if (ok) {
+    tc_fence_after();
+    issue_s_dp(0);
+  }
+  for (int i = 0; ok && i < n; ++i) {
+    const int st = i % kBwdStages;
+    if (i + 1 < n) {
+      const int st1 = (i + 1) % kBwdStages;
+      ok = mbar_wait(&sm.q_full[st1], ((i + 1) / kBwdStages) & 1, ab, lim, SITE_BWD_MMA) &&
+           mbar_wait(&sm.s_free, i & 1, ab, lim, SITE_BWD_MMA);
+      if (!ok) break;
+      tc_fence_after();
+      issue_s_dp(st1);
+    }
+    if (!(ok = mbar_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
+    tc_fence_after();
+    const uint32_t qc = smem_u32(sm.qc[st]), qp = smem_u32(sm.qp[st]),
+                   dO = smem_u32(sm.dO[st]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {  // K = queries, 16 per step
+      const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+      // dV += P^T dO
+      umma_ts(tmem + kBColDV, tmem + kBColP + k * 8,
+              make_sdesc(dO + k * 1024, 16, 512, kLayoutSW64), kIdescBN32, acc);
+      // dK_aug += dS^T Q_aug ; A = dS^T K-major (core matrices)
+      const uint64_t a = make_sdesc(ds + k * 4096, 2048, 128, kLayoutNone);
+      umma_ss(tmem + kBColDKc, a, make_sdesc(qc + k * 1024, 16, 512, kLayoutSW64), kIdescBN32,
+              acc);
+      if (pos)
+        umma_ss(tmem + kBColDKp, a, make_sdesc(qp + k * 512, 16, 256, kLayoutSW32), kIdescBN16,
+                acc);
+    }
+    const int bq = i & 1;
+    if (i >= 2 && !(ok = mbar_wait(&sm.dq_free[bq], ((i >> 1) - 1) & 1, ab, lim, SITE_BWD_MMA)))
+      break;
+    tc_fence_after();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {  // K = keys, 16 per step
+      const uint32_t acc = k > 0 ? 1u : 0u;
+      // dQ_aug = dS K_aug ; A = dS MN-major (same core matrices)
+      const uint64_t a = make_sdesc(ds + k * 256, 128, 2048, kLayoutNone);
+      umma_ss(tmem + kBColDQc + bq * 32, a, make_sdesc(kc + k * 1024, 16, 512, kLayoutSW64),
+              kIdescBQ32, acc);
+      if (pos)
+        umma_ss(tmem + kBColDQp + bq * 16, a, make_sdesc(kp + k * 512, 16, 256, kLayoutSW32),
+                kIdescBQ16, acc);
+    }
+    umma_commit(&sm.ds_free);
+    umma_commit(&sm.dq_full[bq]);
+    umma_commit(&sm.q_empty[st]);
+  }
+  umma_commit(&sm.drain);
+  volatile int no_abort = 0;
+  mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
+}
+
+// Drains dQ of query tile `it` (buffer it & 1) from TMEM into the fp32
+// accumulator.  Group 0 takes columns 0-23, group 1 columns 24-47.
+__device__ __forceinline__ bool bwd_drain_dq(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
+                                             int unit, int it, int g, int wq, bool pos) {
+  volatile int* ab = &sm.abort_flag;
+  const int lane = threadIdx.x & 31;
+  const int bq = it & 1;
+  if (!warp_wait(&sm.dq_full[bq], (it >> 1) & 1, ab, p.wait_limit_ns, SITE_BWD_COMPUTE))
+    return false;
+  tc_fence_after();
+  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  uint32_t r16[16], r8[8];
+  if (g == 0) {
+    tmem_ld_x16(tmem + lane_off + kBColDQc + bq * 32, r16);
+    tmem_ld_x8(tmem + lane_off + kBColDQc + bq * 32 + 16, r8);
+  } else {
+    tmem_ld_x8(tmem + lane_off + kBColDQc + bq * 32 + 24, r8);
+    if (pos) tmem_ld_x16(tmem + lane_off + kBColDQp + bq * 16, r16);
+  }
+  tmem_wait_ld();
+  reg_fence_x16(r16);
+  reg_fence_x8(r8);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sm.dq_free[bq]);
+  const int row = wq * 32 + lane;
+  float* dst = p.dq_acc + ((static_cast<size_t>(unit) * p.n_tiles + it) * 128 + row) * 48;
+  auto f = [](uint32_t x) { return __uint_as_float(x); };
+  if (g == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      red_add_v4(dst + 4 * q, f(r16[4 * q]), f(r16[4 * q + 1]), f(r16[4 * q + 2]),
+                 f(r16[4 * q + 3]));
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      red_add_v4(dst + 16 + 4 * q, f(r8[4 * q]), f(r8[4 * q + 1]), f(r8[4 * q + 2]),
+                 f(r8[4 * q + 3]));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      red_add_v4(dst + 24 + 4 * q, f(r8[4 * q]), f(r8[4 * q + 1]), f(r8[4 * q + 2]),
+                 f(r8[4 * q + 3]));
+    if (pos) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        red_add_v4(dst + 32 + 4 * q, f(r16[4 * q]), f(r16[4 * q + 1]), f(r16[4 * q + 2]),
+                   f(r16[4 * q + 3]));
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
+                                            const UnitCoord& u, int unit, int kt, int g,
+                                            int wq) {
+  volatile int* ab = &sm.abort_flag;
+  const uint64_t lim = p.wait_limit_ns;
+  const int lane = threadIdx.x & 31;
+  const bool pos = p.rank > 0;
+  const int n = p.n_tiles;
+  const int key = wq * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  const float sl = p.scale_log2;
+  uint8_t* ds_row = sm.ds;
+  bool ok = true;
+  for (int i = 0; i < n; ++i) {
+    const int st = i % kBwdStages;
+    if (!(ok = warp_wait(&sm.s_full, i & 1, ab, lim, SITE_BWD_COMPUTE))) break;
+    tc_fence_after();
+    uint32_t s[2][32], dp[2][32];
+    tmem_ld_x32(tmem + lane_off + kBColS + 64 * g, s[0]);
+    tmem_ld_x32(tmem + lane_off + kBColS + 64 * g + 32, s[1]);
+    tmem_ld_x32(tmem + lane_off + kBColDP + 64 * g, dp[0]);
+    tmem_ld_x32(tmem + lane_off + kBColDP + 64 * g + 32, dp[1]);
+    tmem_wait_ld();
+    reg_fence_x32(s[0]);
+    reg_fence_x32(s[1]);
+    reg_fence_x32(dp[0]);
+    reg_fence_x32(dp[1]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.s_free);
+    // lse*log2e and D of this query tile (written by TMA)
+    if (!(ok = warp_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_COMPUTE)))
+      break;
+    const float* lse2 = sm.lse2[st] + 64 * g;
+    const float* dd = sm.dd[st] + 64 * g;
+    uint32_t pk[2][16], dk[2][16];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int q0 = 32 * c + 2 * e;
+        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e]), sl, -lse2[q0]));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e + 1]), sl, -lse2[q0 + 1]));
+        const float d0 = p0 * (__uint_as_float(dp[c][2 * e]) - dd[q0]);
+        const float d1 = p1 * (__uint_as_float(dp[c][2 * e + 1]) - dd[q0 + 1]);
+        pk[c][e] = pack_bf16x2(p0, p1);
+        dk[c][e] = pack_bf16x2(d0, d1);
+      }
+    }
+    // P^T and dS^T buffers are free once the MMAs of tile i-1 completed.
+    if (i > 0 && !(ok = warp_wait(&sm.ds_free, (i - 1) & 1, ab, lim, SITE_BWD_COMPUTE))) break;
+    tc_fence_after();
+    tmem_st_x16(tmem + lane_off + kBColP + 32 * g, pk[0]);
+    tmem_st_x16(tmem + lane_off + kBColP + 32 * g + 16, pk[1]);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int h8 = 0; h8 < 4; ++h8) {
+        const int q = 64 * g + 32 * c + 8 * h8;
+        *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) =
+            make_uint4(dk[c][4 * h8], dk[c][4 * h8 + 1], dk[c][4 * h8 + 2], dk[c][4 * h8 + 3]);
+      }
+    tmem_wait_st();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.ds_full);
+    if (i > 0 && !(ok = bwd_drain_dq(sm, tmem, p, unit, i - 1, g, wq, pos))) break;
+  }
+  if (!ok) return;
+  if (!bwd_drain_dq(sm, tmem, p, unit, n - 1, g, wq, pos)) return;
+  // all MMAs of the last tile are complete (ds_free(n-1) is committed with dq_full)
+  if (!warp_wait(&sm.ds_free, (n - 1) & 1, ab, lim, SITE_BWD_COMPUTE)) return;
+  tc_fence_after();
+  int i0, j0, ii, jl;
+  tile_origin(kt, p.tiles_x, i0, j0);
+  tile_row_local(key, i0, j0, ii, jl);
+  const int y = wrap_once(u.wy * p.M + ii + p.s, p.H);
+  const int x = wrap_once(u.wx * p.M + jl + p.s, p.W);
+  const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
+  __nv_bfloat16* base = p.dqkv + pix * 3 * p.heads * 32;
+  uint32_t r[32];
+  if (g == 0) {  // dV
+    tmem_ld_x32(tmem + lane_off + kBColDV, r);
+    tmem_wait_ld();
+    reg_fence_x32(r);
+    uint4* dst = reinterpret_cast<uint4*>(base + (2 * p.heads + u.head) * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(
+          pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1])),
+          pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+          pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+          pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+    if (pos) {
+      uint32_t r16[16];
+      tmem_ld_x16(tmem + lane_off + kBColDKp, r16);
+      tmem_wait_ld();
+      reg_fence_x16(r16);
+      float4* dk = reinterpret_cast<float4*>(
+          p.dkp_part + ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + key) * 16);
+      const float t = p.scale;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dk[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
+                            __uint_as_float(r16[4 * q + 2]) * t,
+                            __uint_as_float(r16[4 * q + 3]) * t);
+    }
+  } else {  // dKc
+    tmem_ld_x32(tmem + lane_off + kBColDKc, r);
+    tmem_wait_ld();
+    reg_fence_x32(r);
+    const float t = p.scale;
+    uint4* dst = reinterpret_cast<uint4*>(base + (p.heads + u.head) * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(
+          pack_bf16x2(__uint_as_float(r[8 * q + 0]) * t, __uint_as_float(r[8 * q + 1]) * t),
+          pack_bf16x2(__uint_as_float(r[8 * q + 2]) * t, __uint_as_float(r[8 * q + 3]) * t),
+          pack_bf16x2(__uint_as_float(r[8 * q + 4]) * t, __uint_as_float(r[8 * q + 5]) * t),
+          pack_bf16x2(__uint_as_float(r[8 * q + 6]) * t, __uint_as_float(r[8 * q + 7]) * t));
+  }
+}
+
+// grid (n_tiles, units), block kBwdThreads, dynamic smem kBwdSmemBytes.
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+                    const __grid_constant__ CUtensorMap tm_dout,
+                    const __grid_constant__ CUtensorMap tm_qp,
+                    const __grid_constant__ CUtensorMap tm_kp,
+                    const __grid_constant__ CUtensorMap tm_lse2,
+                    const __grid_constant__ CUtensorMap tm_dd, const BwdParams p) {
+  extern __shared__ uint8_t sm_raw_bwd[];
+  BwdSmem& sm = *align1024<BwdSmem>(sm_raw_bwd);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int unit = blockIdx.y;
+  const UnitCoord u = decode_unit(unit, p.heads, p.nW, p.nWx);
+  const int kt = blockIdx.x;
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.k_full, 1);
+    for (int st = 0; st < kBwdStages; ++st) {
+      mbar_init(&sm.q_full[st], 1);
+      mbar_init(&sm.q_empty[st], 1);
+    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_free, 8);
+    mbar_init(&sm.ds_full, 8);
+    mbar_init(&sm.ds_free, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.dq_full[b], 1);
+      mbar_init(&sm.dq_free[b], 8);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_dout);
+    tma_prefetch_desc(&tm_lse2);
+    tma_prefetch_desc(&tm_dd);
+  }
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, kBwdTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (warp < 8) {
+    bwd_compute(sm, tmem, p, u, unit, kt, warp >> 2, warp & 3);
+  } else if (warp == 8) {
+    if (lane == 0) bwd_producer(sm, &tm_qkv, &tm_dout, &tm_qp, &tm_kp, &tm_lse2, &tm_dd, p, u, kt);
+  } else {
+    if (lane == 0) bwd_mma(sm, tmem, p);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- helpers
+
+struct BwdAuxParams {
+  int B, H, W, heads, M, s, nWx, nW, tiles_x, n_tiles, rank;
+  float scale;
+  const __nv_bfloat16* out;
+  const __nv_bfloat16* dout;
+  const float* lse;
+  float* lse2;      // [B][heads][H][W]
+  float* dd;        // [B][heads][H][W]
+  float* dq_acc;    // [units][n_tiles][128][48]
+  const float* dkp_part;
+  size_t dq_acc_floats;
+  __nv_bfloat16* dqkv;
+  float* dqp;       // [heads][M][M][rank]
+  float* dkp;
+};
+
+// One thread per (b, head, y, x): D = sum_c dO*O, lse2 = lse*log2(e); the
+// grid also zeroes the dQ accumulator.
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdAuxParams p) {
+  const size_t n = static_cast<size_t>(p.B) * p.heads * p.H * p.W;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n;
+       idx += stride) {
+    const int x = static_cast<int>(idx % p.W);
+    size_t r = idx / p.W;
+    const int y = static_cast<int>(r % p.H);
+    r /= p.H;
+    const int h = static_cast<int>(r % p.heads);
+    const int b = static_cast<int>(r / p.heads);
+    const size_t row = (((static_cast<size_t>(b) * p.H + y) * p.W + x) * p.heads + h) * 32;
+    const uint4* o4 = reinterpret_cast<const uint4*>(p.out + row);
+    const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + row);
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 a = o4[q], c = g4[q];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+        const float2 fc = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+        acc = fmaf(fa.x, fc.x, acc);
+        acc = fmaf(fa.y, fc.y, acc);
+      }
+    }
+    p.dd[idx] = acc;
+    p.lse2[idx] = p.lse[idx] * 1.4426950408889634f;
+  }
+  float4* z = reinterpret_cast<float4*>(p.dq_acc);
+  const size_t nz = p.dq_acc_floats / 4;
+  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < nz;
+       idx += stride)
+    z[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// One thread per (unit, tile row): dQc * tau -> bf16 at the rolled pixel.
+__global__ void __launch_bounds__(256) dq_finalize_kernel(const BwdAuxParams p) {
+  const size_t n = static_cast<size_t>(p.B) * p.nW * p.heads * p.n_tiles * 128;
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  const int row = static_cast<int>(idx & 127);
+  const size_t ut = idx >> 7;
+  const int tile = static_cast<int>(ut % p.n_tiles);
+  const int unit = static_cast<int>(ut / p.n_tiles);
+  const UnitCoord u = decode_unit(unit, p.heads, p.nW, p.nWx);
+  int i0, j0, i, j;
+  tile_origin(tile, p.tiles_x, i0, j0);
+  tile_row_local(row, i0, j0, i, j);
+  const int y = wrap_once(u.wy * p.M + i + p.s, p.H);
+  const int x = wrap_once(u.wx * p.M + j + p.s, p.W);
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + idx * 48);
+  const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
+  uint4* dst = reinterpret_cast<uint4*>(p.dqkv + (pix * 3 * p.heads + u.head) * 32);
+  const float t = p.scale;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 a = src[2 * q], b = src[2 * q + 1];
+    dst[q] = make_uint4(pack_bf16x2(a.x * t, a.y * t), pack_bf16x2(a.z * t, a.w * t),
+                        pack_bf16x2(b.x * t, b.y * t), pack_bf16x2(b.z * t, b.w * t));
+  }
+}
+
+// One thread per (head, window-local token, r): fixed-order sums over the
+// B*nW units of that head.
+__global__ void __launch_bounds__(256) posgrad_reduce_kernel(const BwdAuxParams p) {
+  const int N = p.M * p.M;
+  const size_t n = static_cast<size_t>(p.heads) * N * p.rank;
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  const int r = static_cast<int>(idx % p.rank);
+  const int tok = static_cast<int>((idx / p.rank) % N);
+  const int h = static_cast<int>(idx / (static_cast<size_t>(p.rank) * N));
+  const int i = tok / p.M, j = tok - i * p.M;
+  const int tile = (i >> 3) * p.tiles_x + (j >> 4);
+  const int row = ((j >> 3) & 1) * 64 + (i & 7) * 8 + (j & 7);
+  float aq = 0.f, ak = 0.f;
+  const int bw_units = p.B * p.nW;
+  for (int bw = 0; bw < bw_units; ++bw) {
+    const size_t unit = static_cast<size_t>(bw) * p.heads + h;
+    const size_t rr = (unit * p.n_tiles + tile) * 128 + row;
+    aq += p.dq_acc[rr * 48 + 32 + r];
+    ak += p.dkp_part[rr * 16 + r];
+  }
+  p.dqp[idx] = aq * p.scale;
+  p.dkp[idx] = ak;
+}
+
+}  // namespace rib

@@ -1,0 +1,200 @@
+// pos_tokens.cuh -- position tokens Qp, Kp of one window geometry and the
+// backward of the position MLPs.
+//
+// "Rank-Factorized Implicit Neural Bias" (gist.science English summary,
+// Technical Summary §2.A steps 1-2; German summary §A step 1): each token of
+// the window gets a normalised 2D coordinate in [-1, 1], expanded by a
+// Fourier feature map and fed to a lightweight MLP that outputs the low-rank
+// positional query / key tokens.  Here: coordinates local to the window with
+// endpoints included, features [sin(w x), cos(w x), sin(w y), cos(w y)],
+// Linear -> GELU(erf) -> Linear, one MLP per side.
+//
+// This is small FMA-pipe work (about 0.8 GFLOP at M = 96) computed once per
+// geometry and cached by the caller, so the kernels favour exactness: the
+// Fourier features are evaluated in fp64 and rounded once to fp32, the MLP
+// runs in fp32 with fp32 accumulation.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace rib {
+
+struct PosParams {
+  int M, N, F, hid, dout, rank;
+  const float* freqs;
+  const float* w1[2];
+  const float* b1[2];
+  const float* w2[2];
+  const float* b2[2];
+  float* out32[2];
+  __nv_bfloat16* out16[2];
+  // backward
+  const float* dtok[2];  // dL/dQp, dL/dKp fp32 [heads][N][rank]
+  float* partial;        // [2][n_chunks][n_params]
+  int n_chunks;
+  int n_params;          // hid*4F + hid + dout*hid + dout
+  float* grads[2][4];    // dw1, db1, dw2, db2 per side
+};
+
+constexpr int kPosTok = 32;      // tokens per CTA, forward
+constexpr int kMlpBwdTok = 64;   // tokens per CTA, backward partial sums
+constexpr int kPosThreads = 256;
+
+// Fourier features of tokens [t0, t0 + T) into g[T][4F] (fp64 math, fp32 store).
+__device__ __forceinline__ void fourier_tile(const PosParams& p, int t0, int T, float* g) {
+  const int F = p.F;
+  for (int idx = threadIdx.x; idx < T * F; idx += blockDim.x) {
+    const int t = idx / F, k = idx - t * F;
+    const int tok = t0 + t;
+    float* row = g + t * 4 * F;
+    if (tok < p.N) {
+      const int i = tok / p.M, j = tok - i * p.M;
+      const double den = p.M > 1 ? static_cast<double>(p.M - 1) : 1.0;
+      const double y = p.M > 1 ? -1.0 + 2.0 * i / den : 0.0;
+      const double x = p.M > 1 ? -1.0 + 2.0 * j / den : 0.0;
+      const double w = static_cast<double>(__ldg(p.freqs + k));
+      double sx, cx, sy, cy;
+      sincos(w * x, &sx, &cx);
+      sincos(w * y, &sy, &cy);
+      row[k] = static_cast<float>(sx);
+      row[F + k] = static_cast<float>(cx);
+      row[2 * F + k] = static_cast<float>(sy);
+      row[3 * F + k] = static_cast<float>(cy);
+    } else {
+      row[k] = row[F + k] = row[2 * F + k] = row[3 * F + k] = 0.f;
+    }
+  }
+}
+
+__device__ __forceinline__ float gelu_erf(float a) {
+  return 0.5f * a * (1.f + erff(a * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ float gelu_erf_grad(float a) {
+  const float cdf = 0.5f * (1.f + erff(a * 0.70710678118654752f));
+  const float pdf = 0.39894228040143268f * expf(-0.5f * a * a);
+  return cdf + a * pdf;
+}
+
+// grid (ceil(N / kPosTok), 2): blockIdx.y selects the q (0) or k (1) MLP.
+__global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
+  extern __shared__ float sm_pos[];
+  const int side = blockIdx.y;
+  const int t0 = blockIdx.x * kPosTok;
+  const int din = 4 * p.F;
+  float* g = sm_pos;                   // [kPosTok][din]
+  float* h = g + kPosTok * din;        // [kPosTok][hid]
+  fourier_tile(p, t0, kPosTok, g);
+  __syncthreads();
+  const float* w1 = p.w1[side];
+  const float* b1 = p.b1[side];
+  for (int idx = threadIdx.x; idx < kPosTok * p.hid; idx += blockDim.x) {
+    const int t = idx / p.hid, jh = idx - t * p.hid;
+    const float* wr = w1 + static_cast<size_t>(jh) * din;
+    const float* gr = g + t * din;
+    float acc = __ldg(b1 + jh);
+    for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
+    h[t * p.hid + jh] = gelu_erf(acc);
+  }
+  __syncthreads();
+  const float* w2 = p.w2[side];
+  const float* b2 = p.b2[side];
+  for (int idx = threadIdx.x; idx < kPosTok * p.dout; idx += blockDim.x) {
+    const int t = idx / p.dout, o = idx - t * p.dout;
+    const int tok = t0 + t;
+    if (tok >= p.N) continue;
+    const float* wr = w2 + static_cast<size_t>(o) * p.hid;
+    const float* hr = h + t * p.hid;
+    float acc = __ldg(b2 + o);
+    for (int k = 0; k < p.hid; ++k) acc = fmaf(__ldg(wr + k), hr[k], acc);
+    const int head = o / p.rank, r = o - head * p.rank;
+    const size_t off = (static_cast<size_t>(head) * p.N + tok) * p.rank + r;
+    p.out32[side][off] = acc;
+    if (p.out16[side]) p.out16[side][off] = __float2bfloat16_rn(acc);
+  }
+}
+
+// Partial sums over kMlpBwdTok tokens of the position-MLP weight gradients.
+// grid (n_chunks, 2).  partial[side][chunk][:] = [dw1 | db1 | dw2 | db2].
+__global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams p) {
+  extern __shared__ float sm_pos[];
+  const int side = blockIdx.y;
+  const int chunk = blockIdx.x;
+  const int t0 = chunk * kMlpBwdTok;
+  const int din = 4 * p.F, hid = p.hid, dout = p.dout;
+  constexpr int T = kMlpBwdTok;
+  float* g = sm_pos;             // [T][din]  Fourier features
+  float* a = g + T * din;        // [T][hid]  pre-activation, then dL/da
+  float* h = a + T * hid;        // [T][hid]  GELU(a)
+  float* go = h + T * hid;       // [T][dout] dL/d(out)
+  fourier_tile(p, t0, T, g);
+  for (int idx = threadIdx.x; idx < T * dout; idx += blockDim.x) {
+    const int t = idx / dout, o = idx - t * dout;
+    const int tok = t0 + t;
+    const int head = o / p.rank, r = o - head * p.rank;
+    go[idx] = tok < p.N ? p.dtok[side][(static_cast<size_t>(head) * p.N + tok) * p.rank + r]
+                        : 0.f;
+  }
+  __syncthreads();
+  const float* w1 = p.w1[side];
+  const float* b1 = p.b1[side];
+  const float* w2 = p.w2[side];
+  for (int idx = threadIdx.x; idx < T * hid; idx += blockDim.x) {
+    const int t = idx / hid, jh = idx - t * hid;
+    const float* wr = w1 + static_cast<size_t>(jh) * din;
+    const float* gr = g + t * din;
+    float acc = __ldg(b1 + jh);
+    for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
+    float dh = 0.f;
+    for (int o = 0; o < dout; ++o) dh = fmaf(__ldg(w2 + static_cast<size_t>(o) * hid + jh),
+                                             go[t * dout + o], dh);
+    h[idx] = gelu_erf(acc);
+    a[idx] = dh * gelu_erf_grad(acc);  // tokens past N have go == 0, so dL/da == 0
+  }
+  __syncthreads();
+  float* out = p.partial + (static_cast<size_t>(side) * p.n_chunks + chunk) * p.n_params;
+  // dw1[jh][k] = sum_t da[t][jh] g[t][k]
+  for (int idx = threadIdx.x; idx < hid * din; idx += blockDim.x) {
+    const int jh = idx / din, k = idx - jh * din;
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc = fmaf(a[t * hid + jh], g[t * din + k], acc);
+    out[idx] = acc;
+  }
+  for (int jh = threadIdx.x; jh < hid; jh += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc += a[t * hid + jh];
+    out[hid * din + jh] = acc;
+  }
+  float* o2 = out + hid * din + hid;
+  // dw2[o][jh] = sum_t go[t][o] h[t][jh]
+  for (int idx = threadIdx.x; idx < dout * hid; idx += blockDim.x) {
+    const int o = idx / hid, jh = idx - o * hid;
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc = fmaf(go[t * dout + o], h[t * hid + jh], acc);
+    o2[idx] = acc;
+  }
+  for (int o = threadIdx.x; o < dout; o += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc += go[t * dout + o];
+    o2[dout * hid + o] = acc;
+  }
+}
+
+// Fixed-order sum of the chunk partials: grid (ceil(n_params / 256), 2).
+__global__ void __launch_bounds__(256) mlp_bwd_reduce_kernel(PosParams p) {
+  const int side = blockIdx.y;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= p.n_params) return;
+  const float* src = p.partial + static_cast<size_t>(side) * p.n_chunks * p.n_params + idx;
+  float acc = 0.f;
+  for (int c = 0; c < p.n_chunks; ++c) acc += src[static_cast<size_t>(c) * p.n_params];
+  const int din = 4 * p.F;
+  const int n_w1 = p.hid * din, n_b1 = p.hid, n_w2 = p.dout * p.hid;
+  if (idx < n_w1) p.grads[side][0][idx] = acc;
+  else if (idx < n_w1 + n_b1) p.grads[side][1][idx - n_w1] = acc;
+  else if (idx < n_w1 + n_b1 + n_w2) p.grads[side][2][idx - n_w1 - n_b1] = acc;
+  else p.grads[side][3][idx - n_w1 - n_b1 - n_w2] = acc;
+}
+
+}  // namespace rib
