@@ -34,12 +34,14 @@ D_QK, D_V = 48, 32
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="rib", choices=["rib", "reference"])
     ap.add_argument("--workload", default="w96train")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--step-only", action="store_true",
+                    help="run only warm-up + timed training steps (for profiler launch lists)")
     return ap.parse_args()
 
 
@@ -283,22 +285,19 @@ def run_rib(args, w):
     def fwd_only():
         R.rib_window_attn_fwd(qkv, M, s, q16, k16, out=out, lse=lse)
 
-    def timed(fn, steps, trace=False, sampler=None):
+    def timed(fn, steps, trace=False):
         stream = torch.cuda.current_stream()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         if trace:
             R.rib_trace_enable(True)
-        if sampler:
-            sampler.start()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(steps):
             fn()
         b.record(stream)
         torch.cuda.synchronize()
-        clocks = sampler.stop() if sampler else None
         kern = R.rib_trace_collect() if trace else None
         if trace:
             R.rib_trace_enable(False)
@@ -308,21 +307,31 @@ def run_rib(args, w):
             t = torch.tensor([ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ms = float(t.item())
-        return ms, kern, clocks
+        return ms, kern, None
 
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
+    if sampler:
+        sampler.start()       # samples cover warm-up and every timed loop below
     for _ in range(args.warmup):
         step()
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
-    props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
-    ms, kern, clocks = timed(step, args.steps, trace=True, sampler=sampler)
+    ms, kern, _ = timed(step, args.steps, trace=True)
     ms_step = ms / args.steps
     f_fwd, f_bwd = flops(w)
     value = world * (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
     tokens_s = world * w.tokens() / (ms_step * 1e-3)
 
+    if args.step_only:
+        if sampler:
+            sampler.stop()
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"step_only": True, "ms_per_step": ms_step, "kernels": kern}))
+        return 0
     for _ in range(args.warmup):
         fwd_only()
     ms_f, kern_f, _ = timed(fwd_only, args.steps, trace=True)
@@ -376,6 +385,7 @@ def run_rib(args, w):
                "h2d_bytes_per_step": nb(h_qkv) + nb(h_dout),
                "d2h_bytes_per_step": nb(h_out) + nb(h_dqkv) + nb(h_flat)}
 
+    clocks = sampler.stop() if sampler else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         N = M * M

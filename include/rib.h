@@ -242,6 +242,12 @@ int rib_trace_enable(int on);
  * entries[0 .. *n_entries) (at most max_entries) and clears the records. */
 int rib_trace_collect(rib_trace_entry_t* entries, int max_entries, int* n_entries);
 
+/* Test hook for the FMA-pipe exponential of the attention kernels:
+ * y[i] = 2^x[i] computed as the forward kernel computes it (Cody-Waite
+ * reduction + degree-3 minimax polynomial, inputs clamped at -125), for
+ * device arrays of n fp32 values (n even). */
+int rib_debug_exp2(const float* x, float* y, int n, void* stream);
+
 /* Library version, e.g. "rib-b200 0.1 sm_100a". */
 const char* rib_version(void);
 

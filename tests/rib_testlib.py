@@ -27,10 +27,16 @@ def stats(got, ref):
 
 def check_close(got, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS, normalize=False):
     """Returns an error message ('' if within bounds).  normalize=True divides
-    the errors by max(1, max|ref|) first (used for fp32 sums whose magnitude
-    grows with the number of tokens summed)."""
+    the errors by max(1, max|ref|) first, and a number divides them by
+    max(1, that number) (used for fp32 sums whose magnitude grows with the
+    number of tokens summed)."""
     mx, mn = stats(got, ref)
-    scale = max(1.0, float(np.abs(np.asarray(ref, dtype=np.float64)).max())) if normalize else 1.0
+    if normalize is True:
+        scale = max(1.0, float(np.abs(np.asarray(ref, dtype=np.float64)).max()))
+    elif normalize:
+        scale = max(1.0, float(normalize))
+    else:
+        scale = 1.0
     ok = mx / scale <= max_abs and mn / scale <= mean_abs
     msg = (f"{what}: max|d|={mx:.3e}, mean|d|={mn:.3e}, max|ref|="
            f"{float(np.abs(np.asarray(ref, dtype=np.float64)).max()):.3e}"
@@ -48,6 +54,20 @@ def assert_all(checks):
     """checks: list of messages from check_close; fails listing every miss."""
     bad = [c for c in checks if c]
     assert not bad, "; ".join(bad)
+
+
+def mlp_grad_checks(dmlp, ref_q, ref_k):
+    """Position-MLP weight grads of one side are judged on that side's common
+    scale, max(1, max|ref| over its four tensors): the key MLP's output-bias
+    gradient is a sum that cancels exactly (rows of dS sum to zero), so its
+    own magnitude says nothing about the size of the terms summed."""
+    checks = []
+    for side, ref in (("q", ref_q), ("k", ref_k)):
+        scale = max(float(np.abs(r).max()) for r in ref)
+        for name, r in zip(("dw1", "db1", "dw2", "db2"), ref):
+            checks.append(check_close(to_np(getattr(dmlp, f"{side}_{name}")), r,
+                                      f"{side}_{name}", normalize=scale))
+    return checks
 
 
 def to_np(t):

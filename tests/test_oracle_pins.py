@@ -434,6 +434,17 @@ def test_attn_bwd_matches_torch_autograd():
     assert abs(tau - 1 / math.sqrt(d + r)) < 1e-16
 
 
+def test_key_gradients_sum_to_zero():
+    """Rows of dS = P*(dP - rowsum(P*dP)) sum to zero, so sum_k dK[k] = 0 for
+    both the content and the positional key gradients."""
+    N, d, r = 40, 6, 3
+    g = O.attention_unit_backward(rnd(N, d), rnd(N, d), rnd(N, d), rnd(N, r), rnd(N, r), 0.7,
+                                  rnd(N, d))
+    dkc, dkp = g[1], g[4]
+    assert np.allclose(dkc.sum(0), 0, atol=1e-12 * np.abs(dkc).sum())
+    assert np.allclose(dkp.sum(0), 0, atol=1e-12 * np.abs(dkp).sum())
+
+
 def test_attn_bwd_unit_subset_equals_zero_upstream_elsewhere():
     qkv, qp, kp, g, M, s = _tiny_problem()
     keep = {(0, 1, 0), (0, 3, 1)}

@@ -28,7 +28,7 @@ __all__ = [
     "rib_window_attn_fwd", "rib_window_attn_bwd", "rib_window_attn_bwd_workspace",
     "rib_window_gather", "rib_window_scatter", "rib_last_status", "rib_status_string",
     "rib_set_wait_limit_ns", "rib_debug_wait_timeout", "rib_version", "library",
-    "rib_trace_enable", "rib_trace_collect",
+    "rib_trace_enable", "rib_trace_collect", "rib_debug_exp2",
 ]
 
 
@@ -271,6 +271,14 @@ def rib_last_status() -> Tuple[int, int]:
 
 def rib_set_wait_limit_ns(limit_ns: int) -> None:
     _check(library().rib_set_wait_limit_ns(int(limit_ns)), "rib_set_wait_limit_ns")
+
+
+def rib_debug_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x with the attention kernels' FMA-pipe exponential (test hook)."""
+    y = torch.empty_like(x)
+    _check(library().rib_debug_exp2(_ptr(x, torch.float32, "x"), _ptr(y, torch.float32, "y"),
+                                    x.numel(), _stream(stream)), "rib_debug_exp2")
+    return y
 
 
 def rib_debug_wait_timeout(limit_ns: int, stream=None) -> None:

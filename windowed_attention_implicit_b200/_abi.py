@@ -60,6 +60,7 @@ _SIGS = {
     "rib_last_status": (_i, [ctypes.POINTER(_i)]),
     "rib_set_wait_limit_ns": (_i, [ctypes.c_ulonglong]),
     "rib_debug_wait_timeout": (_i, [ctypes.c_ulonglong, _p]),
+    "rib_debug_exp2": (_i, [_p, _p, _i, _p]),
     "rib_version": (ctypes.c_char_p, []),
     "rib_trace_enable": (_i, [_i]),
     "rib_trace_collect": (_i, [ctypes.c_void_p, _i, ctypes.POINTER(_i)]),

@@ -20,15 +20,31 @@
 // attn_bwd_kernel, 320 threads:
 //   warps 0-7  compute: thread = key row (TMEM lane), warps 0-3 take query
 //              columns 0-63 and warps 4-7 columns 64-127 of each tile
-//   warp  8    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 2 stages)
-//   warp  9    TMEM allocator and MMA issuer
+//   warp  8    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 4 stages: the
+//              prefetch distance must cover the TMA latency of a tile)
+//   warp  9    TMEM allocator; issues the S^T / dP^T MMAs
+//   warp 10    issues the gradient MMAs (dV, dK_aug, dQ_aug)
+// Two issuing threads: a tcgen05.mma blocks its issuing thread for ~45
+// cycles, so with one issuer the scores of tile i+1 could only be issued
+// after the 24 gradient MMAs of tile i-1, serialising MMAs and
+// exponentials.
 // Per query tile i:  S^T = K_aug Q_aug^T and dP^T = V dO^T (MMA, TMEM) ->
-// compute warps form P^T (to TMEM) and dS^T (to shared memory, core-matrix
-// layout readable both K-major and MN-major) -> MMA: dV += P^T dO (A from
-// TMEM), dK_aug += dS^T Q_aug, dQ_aug = dS K_aug (double-buffered TMEM) ->
-// compute warps drain dQ with red.global.add.v4.f32.
-// S/dP of tile i+1 are issued as soon as the compute warps have pulled tile
-// i into registers, so the MMAs overlap the exponentials.
+// compute warps form P^T and dS^T (to TMEM) and dS (to shared memory,
+// core-matrix layout, double-buffered) -> MMA: dV += P^T dO and
+// dK_aug += dS^T [Qc|Qp] (A from TMEM), dQ_aug = dS [Kc|Kp] (A from shared
+// memory) -> compute warps drain dQ with red.global.add.v4.f32.
+// At d = 32 the MMAs are narrow: a tcgen05.mma of M=128, K=16 costs ~40-50
+// cycles however small N is, and with both operands in shared memory an
+// N <= 64 MMA moves more bytes than its flops cover.  So the A operand comes
+// from TMEM wherever the lane layout allows (P^T, dS^T), the positional
+// tiles are fetched zero-padded to 32 channels (TMA fills the out-of-bounds
+// half with zeros) so that [Qc|Qp] and [Kc|Kp] form one N=48 B operand of two
+// 64B-swizzle atoms, and dK_aug, dQ_aug are one MMA chain each (29 MMAs per
+// tile).  S/dP of tile i+1 are issued as soon as the compute warps have
+// pulled tile i into registers; P^T/dS^T are released right after the dV/dK
+// MMAs and dS is double-buffered, so the compute warps rarely wait on the
+// gradient MMAs of the previous tile.  Exponentials are split between MUFU
+// and the FMA pipe (exp2_fma2), with packed f32x2 arithmetic.
 #pragma once
 
 #include "geom.cuh"
@@ -36,13 +52,20 @@
 
 namespace rib {
 
-constexpr int kBwdStages = 2;
-constexpr int kBwdThreads = 320;
+constexpr int kBwdStages = 4;
+constexpr int kBwdThreads = 352;
 constexpr uint32_t kBwdTmemCols = 512;
-// TMEM columns
-constexpr uint32_t kBColS = 0, kBColDP = 128, kBColP = 256, kBColDV = 320, kBColDKc = 352,
-                   kBColDQc = 384 /* +32 per buffer */, kBColDKp = 448,
-                   kBColDQp = 464 /* +16 per buffer */;
+// TMEM columns (512): S^T, dP^T fp32; P^T, dS^T bf16; dV; dK = [dKc | dKp];
+// dQ = [dQc | dQp]
+constexpr uint32_t kBColS = 0, kBColDP = 128, kBColP = 256, kBColDST = 320, kBColDV = 384,
+                   kBColDK = 416, kBColDQ = 464;
+// Of every 8 element pairs, how many exponentials run on the FMA pipe.  The
+// backward is issue-bound rather than MUFU-bound (its MMA work per score is
+// 2.6x the forward's), so by default every exponential stays on MUFU.
+#ifndef RIB_BWD_POLY_PAIRS
+#define RIB_BWD_POLY_PAIRS 0
+#endif
+constexpr int kBwdPolyPairs = RIB_BWD_POLY_PAIRS;
 constexpr uint64_t kBwdDrainNs = 200ull * 1000ull * 1000ull;
 
 struct BwdParams {
@@ -56,31 +79,31 @@ struct BwdParams {
 };
 
 struct __align__(1024) BwdSmem {
-  uint8_t kc[8192];                // key tile, content, 64B swizzle
+  uint8_t kc[8192];                // key tile, content, [128 rows][64 B], 64B swizzle
+  uint8_t kp[8192];                // key tile, positional zero-padded to 32 ch (kc + 8 KB)
   uint8_t v[8192];
-  uint8_t ds[32768];               // dS^T [128 keys x 128 queries] bf16, core matrices
+  uint8_t ds[2][32768];            // dS^T [128 keys x 128 queries] bf16, core matrices
   uint8_t qc[kBwdStages][8192];
+  uint8_t qp[kBwdStages][8192];    // positional, zero-padded (qc + kBwdStages * 8 KB)
   uint8_t dO[kBwdStages][8192];
-  uint8_t kp[4096];                // key tile, positional, 32B swizzle
-  uint8_t qp[kBwdStages][4096];
-  float lse2[kBwdStages][128];     // lse * log2(e), tile row order
-  float dd[kBwdStages][128];       // D = rowsum(dO * O), tile row order
+  float lse2[kBwdStages][128];     // -lse * log2(e), tile row order
+  float dd[kBwdStages][128];       // -D = -rowsum(dO * O), tile row order
   uint64_t k_full;
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
-  uint64_t s_full, s_free, ds_full, ds_free;
-  uint64_t dq_full[2], dq_free[2];
+  uint64_t s_full, s_free, ds_full, pt_free /* P^T and dS^T in TMEM */, ds_free[2];
+  uint64_t dq_full, dq_free;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 constexpr size_t kBwdSmemBytes = sizeof(BwdSmem) + 1024;
+static_assert(kBwdSmemBytes <= 227 * 1024, "backward shared memory exceeds the per-CTA limit");
 
 constexpr uint32_t kIdescBS = make_idesc_bf16(128, 128, false, false);   // S^T, dP^T
-constexpr uint32_t kIdescBN32 = make_idesc_bf16(128, 32, false, true);   // dV, dKc
-constexpr uint32_t kIdescBN16 = make_idesc_bf16(128, 16, false, true);   // dKp
-constexpr uint32_t kIdescBQ32 = make_idesc_bf16(128, 32, true, true);    // dQc
-constexpr uint32_t kIdescBQ16 = make_idesc_bf16(128, 16, true, true);    // dQp
+constexpr uint32_t kIdescBV = make_idesc_bf16(128, 32, false, true);     // dV
+constexpr uint32_t kIdescBK = make_idesc_bf16(128, 48, false, true);     // dK_aug
+constexpr uint32_t kIdescBQ = make_idesc_bf16(128, 48, true, true);      // dQ_aug
 
 // Byte offset of element (key k, query q) of dS^T: 8 x 8 core matrices of
 // 128 contiguous bytes; key groups of 8 every 128 B, query groups of 8
@@ -102,15 +125,15 @@ __device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
     int i0, j0;
     tile_origin(kt, p.tiles_x, i0, j0);
     const int y = wrap_once(by + i0, p.H);
-    mbar_arrive_expect_tx(&sm.k_full, 2u * 8192u + (pos ? 4096u : 0u));
+    mbar_arrive_expect_tx(&sm.k_full, 2u * 8192u + (pos ? 8192u : 0u));
     for (int c = 0; c < 2; ++c) {
       const int x = wrap_once(bx + j0 + 8 * c, p.W);
       tma_load_5d(sm.kc + c * 4096, tq, &sm.k_full, 0, p.heads + hh, x, y, u.b);
       tma_load_5d(sm.v + c * 4096, tq, &sm.k_full, 0, 2 * p.heads + hh, x, y, u.b);
-      if (pos) tma_load_4d(sm.kp + c * 2048, tkp, &sm.k_full, 0, j0 + 8 * c, i0, hh);
+      if (pos) tma_load_4d(sm.kp + c * 4096, tkp, &sm.k_full, 0, j0 + 8 * c, i0, hh);
     }
   }
-  const uint32_t q_bytes = 2u * 8192u + (pos ? 4096u : 0u) + 2u * 512u;
+  const uint32_t q_bytes = 2u * 8192u + (pos ? 8192u : 0u) + 2u * 512u;
   int i = 0;
   for (; i < p.n_tiles; ++i) {
     const int st = i % kBwdStages, use = i / kBwdStages;
@@ -125,7 +148,7 @@ __device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
       const int x = wrap_once(bx + j0 + 8 * c, p.W);
       tma_load_5d(sm.qc[st] + c * 4096, tq, &sm.q_full[st], 0, hh, x, y, u.b);
       tma_load_5d(sm.dO[st] + c * 4096, tdo, &sm.q_full[st], 0, hh, x, y, u.b);
-      if (pos) tma_load_4d(sm.qp[st] + c * 2048, tqp, &sm.q_full[st], 0, j0 + 8 * c, i0, hh);
+      if (pos) tma_load_4d(sm.qp[st] + c * 4096, tqp, &sm.q_full[st], 0, j0 + 8 * c, i0, hh);
       tma_load_4d(&sm.lse2[st][c * 64], tlse2, &sm.q_full[st], x, y, hh, u.b);
       tma_load_4d(&sm.dd[st][c * 64], tdd, &sm.q_full[st], x, y, hh, u.b);
     }
@@ -139,80 +162,83 @@ __device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
   }
 }
 
-__device__ __forceinline__ void bwd_mma(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
+// Warp 9: S^T = K_aug Q_aug^T and dP^T = V dO^T of every query tile, each
+// issued as soon as the compute warps have pulled the previous one into
+// registers.
+__device__ __forceinline__ void bwd_mma_scores(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const bool pos = p.rank > 0;
   const int n = p.n_tiles;
-  const uint32_t kc = smem_u32(sm.kc), v = smem_u32(sm.v), kp = smem_u32(sm.kp),
-                 ds = smem_u32(sm.ds);
-  auto issue_s_dp = [&](int st) {
+  const uint32_t kc = smem_u32(sm.kc), kp = smem_u32(sm.kp), v = smem_u32(sm.v);
+  bool ok = mbar_wait(&sm.k_full, 0, ab, lim, SITE_BWD_MMA);
+  for (int i = 0; ok && i < n; ++i) {
+    const int st = i % kBwdStages;
+    ok = mbar_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_MMA) &&
+         (i == 0 || mbar_wait(&sm.s_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA));
+    if (!ok) break;
+    tc_fence_after();
     // S^T = K_aug Q_aug^T  (M = keys, N = queries, K = 32 + 16)
     const uint64_t a = make_sdesc(kc, 16, 512, kLayoutSW64);
     const uint64_t b = make_sdesc(smem_u32(sm.qc[st]), 16, 512, kLayoutSW64);
     umma_ss(tmem + kBColS, a, b, kIdescBS, 0u);
     umma_ss(tmem + kBColS, a + 2, b + 2, kIdescBS, 1u);
     if (pos)
-      umma_ss(tmem + kBColS, make_sdesc(kp, 16, 256, kLayoutSW32),
-              make_sdesc(smem_u32(sm.qp[st]), 16, 256, kLayoutSW32), kIdescBS, 1u);
+      umma_ss(tmem + kBColS, make_sdesc(kp, 16, 512, kLayoutSW64),
+              make_sdesc(smem_u32(sm.qp[st]), 16, 512, kLayoutSW64), kIdescBS, 1u);
     // dP^T = V dO^T  (M = keys, N = queries, K = 32)
     const uint64_t av = make_sdesc(v, 16, 512, kLayoutSW64);
     const uint64_t bo = make_sdesc(smem_u32(sm.dO[st]), 16, 512, kLayoutSW64);
     umma_ss(tmem + kBColDP, av, bo, kIdescBS, 0u);
     umma_ss(tmem + kBColDP, av + 2, bo + 2, kIdescBS, 1u);
     umma_commit(&sm.s_full);
-  };
-  bool ok = mbar_wait(&sm.k_full, 0, ab, lim, SITE_BWD_MMA) &&
-            mbar_wait(&sm.q_full[0], 0, ab, lim, SITE_BWD_MMA);
-  if (ok) {
-    tc_fence_after();
-    issue_s_dp(0);
   }
+  umma_commit(&sm.drain);
+  volatile int no_abort = 0;
+  mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
+}
+
+// Warp 10: dV += P^T dO, dK_aug += dS^T [Qc|Qp] (A from TMEM) and
+// dQ_aug = dS [Kc|Kp] (A from shared memory) of every query tile.
+__device__ __forceinline__ void bwd_mma_grads(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
+  volatile int* ab = &sm.abort_flag;
+  const uint64_t lim = p.wait_limit_ns;
+  const int n = p.n_tiles;
+  const uint32_t kc = smem_u32(sm.kc), kp = smem_u32(sm.kp);
+  const uint32_t lbo_q = smem_u32(sm.qp[0]) - smem_u32(sm.qc[0]);   // [Qc|Qp] atoms
+  const uint32_t lbo_k = kp - kc;                                   // [Kc|Kp] atoms
+  bool ok = true;
   for (int i = 0; ok && i < n; ++i) {
     const int st = i % kBwdStages;
-    if (i + 1 < n) {
-      const int st1 = (i + 1) % kBwdStages;
-      ok = mbar_wait(&sm.q_full[st1], ((i + 1) / kBwdStages) & 1, ab, lim, SITE_BWD_MMA) &&
-           mbar_wait(&sm.s_free, i & 1, ab, lim, SITE_BWD_MMA);
-      if (!ok) break;
-      tc_fence_after();
-      issue_s_dp(st1);
-    }
+    // ds_full(i) implies the stage's tiles have landed: the compute warps
+    // waited for them (q_full) before forming P^T and dS^T.
     if (!(ok = mbar_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
     tc_fence_after();
-    const uint32_t qc = smem_u32(sm.qc[st]), qp = smem_u32(sm.qp[st]),
-                   dO = smem_u32(sm.dO[st]);
+    const uint32_t qc = smem_u32(sm.qc[st]), dO = smem_u32(sm.dO[st]);
+    const uint32_t ds = smem_u32(sm.ds[i & 1]);
+    // dV += P^T dO   (K = queries, 16 per step; A from TMEM)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {  // K = queries, 16 per step
-      const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-      // dV += P^T dO
+    for (int k = 0; k < 8; ++k)
       umma_ts(tmem + kBColDV, tmem + kBColP + k * 8,
-              make_sdesc(dO + k * 1024, 16, 512, kLayoutSW64), kIdescBN32, acc);
-      // dK_aug += dS^T Q_aug ; A = dS^T K-major (core matrices)
-      const uint64_t a = make_sdesc(ds + k * 4096, 2048, 128, kLayoutNone);
-      umma_ss(tmem + kBColDKc, a, make_sdesc(qc + k * 1024, 16, 512, kLayoutSW64), kIdescBN32,
-              acc);
-      if (pos)
-        umma_ss(tmem + kBColDKp, a, make_sdesc(qp + k * 512, 16, 256, kLayoutSW32), kIdescBN16,
-                acc);
-    }
-    const int bq = i & 1;
-    if (i >= 2 && !(ok = mbar_wait(&sm.dq_free[bq], ((i >> 1) - 1) & 1, ab, lim, SITE_BWD_MMA)))
-      break;
+              make_sdesc(dO + k * 1024, 16, 512, kLayoutSW64), kIdescBV,
+              (i > 0 || k > 0) ? 1u : 0u);
+    // dK_aug += dS^T [Qc|Qp]   (A = dS^T from TMEM)
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      umma_ts(tmem + kBColDK, tmem + kBColDST + k * 8,
+              make_sdesc(qc + k * 1024, lbo_q, 512, kLayoutSW64), kIdescBK,
+              (i > 0 || k > 0) ? 1u : 0u);
+    umma_commit(&sm.pt_free);
+    // dQ_aug = dS [Kc|Kp]   (A = dS MN-major core matrices); the single dQ
+    // buffer is free once the compute warps drained tile i-1
+    if (i > 0 && !(ok = mbar_wait(&sm.dq_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA))) break;
     tc_fence_after();
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {  // K = keys, 16 per step
-      const uint32_t acc = k > 0 ? 1u : 0u;
-      // dQ_aug = dS K_aug ; A = dS MN-major (same core matrices)
-      const uint64_t a = make_sdesc(ds + k * 256, 128, 2048, kLayoutNone);
-      umma_ss(tmem + kBColDQc + bq * 32, a, make_sdesc(kc + k * 1024, 16, 512, kLayoutSW64),
-              kIdescBQ32, acc);
-      if (pos)
-        umma_ss(tmem + kBColDQp + bq * 16, a, make_sdesc(kp + k * 512, 16, 256, kLayoutSW32),
-                kIdescBQ16, acc);
-    }
-    umma_commit(&sm.ds_free);
-    umma_commit(&sm.dq_full[bq]);
+    for (int k = 0; k < 8; ++k)
+      umma_ss(tmem + kBColDQ, make_sdesc(ds + k * 256, 128, 2048, kLayoutNone),
+              make_sdesc(kc + k * 1024, lbo_k, 512, kLayoutSW64), kIdescBQ, k > 0 ? 1u : 0u);
+    umma_commit(&sm.ds_free[i & 1]);
+    umma_commit(&sm.dq_full);
     umma_commit(&sm.q_empty[st]);
   }
   umma_commit(&sm.drain);
@@ -220,31 +246,29 @@ __device__ __forceinline__ void bwd_mma(BwdSmem& sm, uint32_t tmem, const BwdPar
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
 }
 
-// Drains dQ of query tile `it` (buffer it & 1) from TMEM into the fp32
-// accumulator.  Group 0 takes columns 0-23, group 1 columns 24-47.
+// Drains dQ of query tile `it` from TMEM into the fp32 accumulator.
+// Group 0 takes columns 0-23, group 1 columns 24-47 (32-47 = dQp).
 __device__ __forceinline__ bool bwd_drain_dq(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
                                              int unit, int it, int g, int wq, bool pos) {
   volatile int* ab = &sm.abort_flag;
   const int lane = threadIdx.x & 31;
-  const int bq = it & 1;
-  if (!warp_wait(&sm.dq_full[bq], (it >> 1) & 1, ab, p.wait_limit_ns, SITE_BWD_COMPUTE))
-    return false;
+  if (!warp_wait(&sm.dq_full, it & 1, ab, p.wait_limit_ns, SITE_BWD_COMPUTE)) return false;
   tc_fence_after();
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-  uint32_t r16[16], r8[8];
+  uint32_t r16[16] = {0}, r8[8];
   if (g == 0) {
-    tmem_ld_x16(tmem + lane_off + kBColDQc + bq * 32, r16);
-    tmem_ld_x8(tmem + lane_off + kBColDQc + bq * 32 + 16, r8);
+    tmem_ld_x16(tmem + lane_off + kBColDQ, r16);
+    tmem_ld_x8(tmem + lane_off + kBColDQ + 16, r8);
   } else {
-    tmem_ld_x8(tmem + lane_off + kBColDQc + bq * 32 + 24, r8);
-    if (pos) tmem_ld_x16(tmem + lane_off + kBColDQp + bq * 16, r16);
+    tmem_ld_x8(tmem + lane_off + kBColDQ + 24, r8);
+    if (pos) tmem_ld_x16(tmem + lane_off + kBColDQ + 32, r16);
   }
   tmem_wait_ld();
   reg_fence_x16(r16);
   reg_fence_x8(r8);
   tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive(&sm.dq_free[bq]);
+  if (lane == 0) mbar_arrive(&sm.dq_free);
   const int row = wq * 32 + lane;
   float* dst = p.dq_acc + ((static_cast<size_t>(unit) * p.n_tiles + it) * 128 + row) * 48;
   auto f = [](uint32_t x) { return __uint_as_float(x); };
@@ -283,7 +307,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
   const int key = wq * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
   const float sl = p.scale_log2;
-  uint8_t* ds_row = sm.ds;
+  const uint64_t sl2 = pk2(sl, sl);
   bool ok = true;
   for (int i = 0; i < n; ++i) {
     const int st = i % kBwdStages;
@@ -305,35 +329,52 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     // lse*log2e and D of this query tile (written by TMA)
     if (!(ok = warp_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_COMPUTE)))
       break;
-    const float* lse2 = sm.lse2[st] + 64 * g;
-    const float* dd = sm.dd[st] + 64 * g;
-    uint32_t pk[2][16], dk[2][16];
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int q0 = 32 * c + 2 * e;
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e]), sl, -lse2[q0]));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e + 1]), sl, -lse2[q0 + 1]));
-        const float d0 = p0 * (__uint_as_float(dp[c][2 * e]) - dd[q0]);
-        const float d1 = p1 * (__uint_as_float(dp[c][2 * e + 1]) - dd[q0 + 1]);
-        pk[c][e] = pack_bf16x2(p0, p1);
-        dk[c][e] = pack_bf16x2(d0, d1);
-      }
-    }
-    // P^T and dS^T buffers are free once the MMAs of tile i-1 completed.
-    if (i > 0 && !(ok = warp_wait(&sm.ds_free, (i - 1) & 1, ab, lim, SITE_BWD_COMPUTE))) break;
+    // P^T and dS^T (TMEM) are free once dV(i-1), dK(i-1) completed; the dS
+    // buffer i&1 (shared memory) once tile i-2's dQ MMAs completed.
+    if (i > 0 && !(ok = warp_wait(&sm.pt_free, (i - 1) & 1, ab, lim, SITE_BWD_COMPUTE))) break;
+    if (i > 1 &&
+        !(ok = warp_wait(&sm.ds_free[i & 1], ((i >> 1) - 1) & 1, ab, lim, SITE_BWD_COMPUTE)))
+      break;
     tc_fence_after();
-    tmem_st_x16(tmem + lane_off + kBColP + 32 * g, pk[0]);
-    tmem_st_x16(tmem + lane_off + kBColP + 32 * g + 16, pk[1]);
+    uint8_t* ds_row = sm.ds[i & 1];
+    const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[st] + 64 * g);
+    const float4* dd4 = reinterpret_cast<const float4*>(sm.dd[st] + 64 * g);
+    // 16 query columns at a time: P^T and dS^T to TMEM, dS to shared memory.
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
+    for (int ch = 0; ch < 4; ++ch) {
+      const uint32_t* sc = &s[ch >> 1][(ch & 1) * 16];
+      const uint32_t* dc = &dp[ch >> 1][(ch & 1) * 16];
+      uint32_t pk[8], dk[8];
 #pragma unroll
-      for (int h8 = 0; h8 < 4; ++h8) {
-        const int q = 64 * g + 32 * c + 8 * h8;
-        *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) =
-            make_uint4(dk[c][4 * h8], dk[c][4 * h8 + 1], dk[c][4 * h8 + 2], dk[c][4 * h8 + 3]);
+      for (int v4 = 0; v4 < 4; ++v4) {
+        const float4 l = lse4[ch * 4 + v4];    // -lse*log2e
+        const float4 dv = dd4[ch * 4 + v4];    // -D
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int e = 4 * v4 + 2 * h2;       // element pair (e, e+1) of the chunk
+          const uint64_t nl = h2 ? pk2(l.z, l.w) : pk2(l.x, l.y);
+          const uint64_t nd = h2 ? pk2(dv.z, dv.w) : pk2(dv.x, dv.y);
+          const uint64_t x2 = ffma2(pk2(__uint_as_float(sc[e]), __uint_as_float(sc[e + 1])),
+                                    sl2, nl);
+          uint64_t p2;
+          if (2 * v4 + h2 < kBwdPolyPairs) {
+            p2 = exp2_fma2(x2);
+          } else {
+            p2 = pk2(ex2_approx(lo2(x2)), ex2_approx(hi2(x2)));
+          }
+          const uint64_t d2 = fmul2(p2, fadd2(pk2(__uint_as_float(dc[e]),
+                                                  __uint_as_float(dc[e + 1])), nd));
+          pk[e >> 1] = pack_bf16x2(lo2(p2), hi2(p2));
+          dk[e >> 1] = pack_bf16x2(lo2(d2), hi2(d2));
+        }
       }
+      tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, pk);
+      tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, dk);
+      const int q = 64 * g + 16 * ch;
+      *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+      *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q + 8)) =
+          make_uint4(dk[4], dk[5], dk[6], dk[7]);
+    }
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
@@ -342,9 +383,8 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     if (i > 0 && !(ok = bwd_drain_dq(sm, tmem, p, unit, i - 1, g, wq, pos))) break;
   }
   if (!ok) return;
+  // dq_full(n-1) is committed after every MMA of the kernel
   if (!bwd_drain_dq(sm, tmem, p, unit, n - 1, g, wq, pos)) return;
-  // all MMAs of the last tile are complete (ds_free(n-1) is committed with dq_full)
-  if (!warp_wait(&sm.ds_free, (n - 1) & 1, ab, lim, SITE_BWD_COMPUTE)) return;
   tc_fence_after();
   int i0, j0, ii, jl;
   tile_origin(kt, p.tiles_x, i0, j0);
@@ -368,7 +408,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
           pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
     if (pos) {
       uint32_t r16[16];
-      tmem_ld_x16(tmem + lane_off + kBColDKp, r16);
+      tmem_ld_x16(tmem + lane_off + kBColDK + 32, r16);
       tmem_wait_ld();
       reg_fence_x16(r16);
       float4* dk = reinterpret_cast<float4*>(
@@ -381,7 +421,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
                             __uint_as_float(r16[4 * q + 3]) * t);
     }
   } else {  // dKc
-    tmem_ld_x32(tmem + lane_off + kBColDKc, r);
+    tmem_ld_x32(tmem + lane_off + kBColDK, r);
     tmem_wait_ld();
     reg_fence_x32(r);
     const float t = p.scale;
@@ -419,12 +459,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.s_free, 8);
     mbar_init(&sm.ds_full, 8);
-    mbar_init(&sm.ds_free, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.dq_full[b], 1);
-      mbar_init(&sm.dq_free[b], 8);
-    }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.pt_free, 1);
+    mbar_init(&sm.ds_free[0], 1);
+    mbar_init(&sm.ds_free[1], 1);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dq_free, 8);
+    mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -446,8 +486,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_compute(sm, tmem, p, u, unit, kt, warp >> 2, warp & 3);
   } else if (warp == 8) {
     if (lane == 0) bwd_producer(sm, &tm_qkv, &tm_dout, &tm_qp, &tm_kp, &tm_lse2, &tm_dd, p, u, kt);
+  } else if (warp == 9) {
+    if (lane == 0) bwd_mma_scores(sm, tmem, p);
   } else {
-    if (lane == 0) bwd_mma(sm, tmem, p);
+    if (lane == 0) bwd_mma_grads(sm, tmem, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -475,8 +517,9 @@ struct BwdAuxParams {
   float* dkp;
 };
 
-// One thread per (b, head, y, x): D = sum_c dO*O, lse2 = lse*log2(e); the
-// grid also zeroes the dQ accumulator.
+// One thread per (b, head, y, x): -D = -sum_c dO*O and -lse*log2(e), stored
+// negated for the fused multiply-adds of the main kernel; the grid also
+// zeroes the dQ accumulator.
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdAuxParams p) {
   const size_t n = static_cast<size_t>(p.B) * p.heads * p.H * p.W;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
@@ -504,8 +547,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdAuxParams 
         acc = fmaf(fa.y, fc.y, acc);
       }
     }
-    p.dd[idx] = acc;
-    p.lse2[idx] = p.lse[idx] * 1.4426950408889634f;
+    p.dd[idx] = -acc;
+    p.lse2[idx] = -p.lse[idx] * 1.4426950408889634f;
   }
   float4* z = reinterpret_cast<float4*>(p.dq_acc);
   const size_t nz = p.dq_acc_floats / 4;

@@ -20,12 +20,20 @@
 //              3-stage shared-memory ring; boxes at rolled map coordinates
 //   warp  9    TMEM allocator and MMA issuer (one thread)
 // TMEM (512 columns): S_A, S_B fp32 [128 x 128]; P_A, P_B bf16 [128 x 128]
-// (64 packed columns each); O_A, O_B fp32 [128 x 32].
+// (64 packed columns each); [O|L]_A, [O|L]_B fp32 [128 x 48].
 // Per key tile j and group X: S_X(j) = Q_X K_j^T (MMA) -> online softmax in
-// registers -> P_X(j) to TMEM -> O_X += P_X(j) V_j (MMA, A from TMEM).
-// S_X(j+1) is issued as soon as group X has pulled S_X(j) into registers,
-// so score MMAs overlap the exponentials.  The running max is updated
-// lazily: O and l are rescaled only when the max grows by more than 2^8.
+// registers -> P_X(j) to TMEM -> [O|L]_X += P_X(j) [V_j | 1] (MMA, A from
+// TMEM): the second swizzle atom of the B operand is an all-ones tile, so the
+// tensor core also accumulates the softmax denominators L from the very bf16
+// P it multiplies with V.  S_X(j+1) is issued as soon as group X has pulled
+// S_X(j) into registers, so score MMAs overlap the exponentials.  The
+// running max is updated lazily: O and L are rescaled only when the max
+// grows by more than 2^8.
+//
+// The exponentials are the bottleneck of this kernel (16K per 128x128 tile
+// against 320 tensor-core cycles of MMA at d_qk=48, d_v=32), so a fixed
+// share of them (kPolyPairs of every 16 pairs) runs on the FMA pipe
+// (exp2_fma2) and the rest on MUFU ex2; scaling uses packed f32x2 FMAs.
 #pragma once
 
 #include "geom.cuh"
@@ -36,7 +44,13 @@ namespace rib {
 constexpr int kFwdStages = 3;
 constexpr int kFwdThreads = 320;
 constexpr uint32_t kFwdTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // O_X at kColO + 48 X, L at +32
+constexpr int kOCols = 48;
+// Of every 16 element pairs, how many exponentials run on the FMA pipe.
+#ifndef RIB_FWD_POLY_PAIRS
+#define RIB_FWD_POLY_PAIRS 6
+#endif
+constexpr int kPolyPairs = RIB_FWD_POLY_PAIRS;
 constexpr uint64_t kFwdDrainNs = 200ull * 1000ull * 1000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -52,6 +66,7 @@ struct __align__(1024) FwdSmem {
   uint8_t qc[2][8192];            // [128 rows][64 B], 64B swizzle
   uint8_t kc[kFwdStages][8192];
   uint8_t v[kFwdStages][8192];
+  uint8_t ones[8192];             // bf16 1.0 everywhere: B atom that yields the row sums
   uint8_t qp[2][4096];            // [128 rows][32 B], 32B swizzle
   uint8_t kp[kFwdStages][4096];
   uint64_t q_full;
@@ -64,9 +79,10 @@ struct __align__(1024) FwdSmem {
 };
 
 constexpr size_t kFwdSmemBytes = sizeof(FwdSmem) + 1024;  // + alignment slack
+static_assert(kFwdSmemBytes <= 227 * 1024, "forward shared memory exceeds the per-CTA limit");
 
 constexpr uint32_t kIdescS = make_idesc_bf16(128, 128, false, false);
-constexpr uint32_t kIdescPV = make_idesc_bf16(128, 32, false, true);
+constexpr uint32_t kIdescPV = make_idesc_bf16(128, kOCols, false, true);
 
 __device__ __forceinline__ void fwd_producer(FwdSmem& sm, const CUtensorMap* tq,
                                              const CUtensorMap* tqp, const CUtensorMap* tkp,
@@ -152,15 +168,17 @@ __device__ __forceinline__ void fwd_mma(FwdSmem& sm, uint32_t tmem, const FwdPar
       if (!ok) break;
     }
     const uint32_t vaddr = smem_u32(sm.v[st]);
+    // B = [V | ones]: two MN-major 64B-swizzle atoms, the second LBO bytes on
+    const uint32_t lbo = smem_u32(sm.ones) - vaddr;
     for (int X = 0; ok && X < 2; ++X) {
       ok = mbar_wait(&sm.p_full[X], j & 1, ab, lim, SITE_FWD_MMA);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t d = tmem + kColO + X * 32;
+      const uint32_t d = tmem + kColO + X * kOCols;
       const uint32_t a = tmem + kColP + X * 64;
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        umma_ts(d, a + k * 8, make_sdesc(vaddr + k * 1024, 16, 512, kLayoutSW64), kIdescPV,
+        umma_ts(d, a + k * 8, make_sdesc(vaddr + k * 1024, lbo, 512, kLayoutSW64), kIdescPV,
                 (j > 0 || k > 0) ? 1u : 0u);
       umma_commit(&sm.pv_done[X]);
     }
@@ -180,10 +198,11 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
   const uint32_t tS = tmem + lane_off + kColS + X * 128;
   const uint32_t tP = tmem + lane_off + kColP + X * 64;
-  const uint32_t tO = tmem + lane_off + kColO + X * 32;
+  const uint32_t tO = tmem + lane_off + kColO + X * kOCols;
   const float sl = p.scale_log2;
+  const uint64_t sl2 = pk2(sl, sl);
   const int n = p.n_tiles;
-  float m_run = 0.f, l_run = 0.f;
+  float m_run = 0.f;
   bool ok = true;
   for (int j = 0; j < n; ++j) {
     if (!(ok = warp_wait(&sm.s_full[X], j & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
@@ -206,7 +225,9 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+      for (int e = (c == 0 ? 1 : 0); e + 1 < 32; e += 2)
+        mx = fmax3(mx, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+    mx = fmaxf(mx, __uint_as_float(s[3][31]));
     const float m_tile = mx * sl;
     float m_new = m_run, alpha = 1.f;
     bool resc = false;
@@ -218,32 +239,44 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
       resc = true;
     }
     if (j > 0) {
-      // P_X and O_X are free once PV_X(j-1) has completed.
+      // P_X and [O|L]_X are free once PV_X(j-1) has completed.
       if (!(ok = warp_wait(&sm.pv_done[X], (j - 1) & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
       tc_fence_after();
-      if (__any_sync(0xffffffffu, resc)) {
-        uint32_t o[32];
-        tmem_ld_x32(tO, o);
-        tmem_wait_ld();
-        reg_fence_x32(o);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st_x32(tO, o);
-      }
     }
-    l_run *= alpha;
-    const float neg = -m_new;
+    const uint64_t neg2 = pk2(-m_new, -m_new);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e]), sl, neg));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][2 * e + 1]), sl, neg));
-        l_run += p0 + p1;
+        const uint64_t x2 = ffma2(pk2(__uint_as_float(s[c][2 * e]),
+                                      __uint_as_float(s[c][2 * e + 1])), sl2, neg2);
+        float p0, p1;
+        if (e < kPolyPairs) {
+          const uint64_t e2 = exp2_fma2(x2);
+          p0 = lo2(e2);
+          p1 = hi2(e2);
+        } else {
+          p0 = ex2_approx(lo2(x2));
+          p1 = ex2_approx(hi2(x2));
+        }
         pk[e] = pack_bf16x2(p0, p1);
       }
       tmem_st_x16(tP + c * 16, pk);
+    }
+    if (j > 0 && __any_sync(0xffffffffu, resc)) {
+      uint32_t o[32], l[16];
+      tmem_ld_x32(tO, o);
+      tmem_ld_x16(tO + 32, l);
+      tmem_wait_ld();
+      reg_fence_x32(o);
+      reg_fence_x16(l);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) l[e] = __float_as_uint(__uint_as_float(l[e]) * alpha);
+      tmem_st_x32(tO, o);
+      tmem_st_x16(tO + 32, l);
     }
     tmem_wait_st();
     tc_fence_before();
@@ -254,10 +287,13 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   if (!ok) return;
   if (!warp_wait(&sm.pv_done[X], (n - 1) & 1, ab, lim, SITE_FWD_SOFTMAX)) return;
   tc_fence_after();
-  uint32_t o[32];
+  uint32_t o[32], l[16];
   tmem_ld_x32(tO, o);
+  tmem_ld_x16(tO + 32, l);
   tmem_wait_ld();
   reg_fence_x32(o);
+  reg_fence_x16(l);
+  const float l_run = __uint_as_float(l[0]);
   const float inv = 1.f / l_run;
   uint32_t pk[16];
 #pragma unroll
@@ -301,6 +337,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
+  }
+  {
+    // all-ones B atom (bf16 1.0 = 0x3F80), read by the tensor core
+    uint4* ones = reinterpret_cast<uint4*>(sm.ones);
+    for (int i = threadIdx.x; i < 8192 / 16; i += blockDim.x)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_proxy_async_smem();
   }
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_qkv);

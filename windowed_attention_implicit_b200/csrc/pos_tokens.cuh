@@ -37,17 +37,24 @@ struct PosParams {
   float* grads[2][4];    // dw1, db1, dw2, db2 per side
 };
 
-constexpr int kPosTok = 32;      // tokens per CTA, forward
-constexpr int kMlpBwdTok = 64;   // tokens per CTA, backward partial sums
-constexpr int kPosThreads = 256;
+constexpr int kPosTok = 64;       // tokens per CTA (forward and backward partials)
+constexpr int kMlpBwdTok = kPosTok;
+constexpr int kPosThreads = 256;  // 4 threads per token
 
-// Fourier features of tokens [t0, t0 + T) into g[T][4F] (fp64 math, fp32 store).
-__device__ __forceinline__ void fourier_tile(const PosParams& p, int t0, int T, float* g) {
-  const int F = p.F;
-  for (int idx = threadIdx.x; idx < T * F; idx += blockDim.x) {
-    const int t = idx / F, k = idx - t * F;
+// Shared-memory layouts are token-major with rows padded by one float: a warp
+// covers 32 consecutive tokens at a fixed feature (conflict-free) or 32
+// consecutive features of one token (conflict-free), and weight rows are read
+// with the same address across the warp (broadcast).
+__host__ __device__ constexpr int pad1(int n) { return n + 1; }
+
+// Fourier features of tokens [t0, t0 + kPosTok) into g[kPosTok][pad1(4F)]
+// (fp64 math, fp32 store).
+__device__ __forceinline__ void fourier_tile(const PosParams& p, int t0, float* g) {
+  const int F = p.F, ld = pad1(4 * F);
+  for (int idx = threadIdx.x; idx < kPosTok * F; idx += blockDim.x) {
+    const int t = idx % kPosTok, k = idx / kPosTok;
     const int tok = t0 + t;
-    float* row = g + t * 4 * F;
+    float* row = g + t * ld;
     if (tok < p.N) {
       const int i = tok / p.M, j = tok - i * p.M;
       const double den = p.M > 1 ? static_cast<double>(p.M - 1) : 1.0;
@@ -77,35 +84,43 @@ __device__ __forceinline__ float gelu_erf_grad(float a) {
   return cdf + a * pdf;
 }
 
+__host__ __device__ constexpr size_t pos_fwd_smem_floats(int F, int hid) {
+  return static_cast<size_t>(kPosTok) * (pad1(4 * F) + pad1(hid));
+}
+
+__host__ __device__ constexpr size_t mlp_bwd_smem_floats(int F, int hid, int dout) {
+  return static_cast<size_t>(kPosTok) * (pad1(4 * F) + 2 * pad1(hid) + pad1(dout));
+}
+
 // grid (ceil(N / kPosTok), 2): blockIdx.y selects the q (0) or k (1) MLP.
 __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   extern __shared__ float sm_pos[];
   const int side = blockIdx.y;
   const int t0 = blockIdx.x * kPosTok;
-  const int din = 4 * p.F;
-  float* g = sm_pos;                   // [kPosTok][din]
-  float* h = g + kPosTok * din;        // [kPosTok][hid]
-  fourier_tile(p, t0, kPosTok, g);
+  const int din = 4 * p.F, ldg = pad1(din), ldh = pad1(p.hid);
+  float* g = sm_pos;                   // [kPosTok][din+1]
+  float* h = g + kPosTok * ldg;        // [kPosTok][hid+1]
+  fourier_tile(p, t0, g);
   __syncthreads();
+  const int t = threadIdx.x % kPosTok, q = threadIdx.x / kPosTok;  // 4 threads per token
+  const int nq = blockDim.x / kPosTok;
   const float* w1 = p.w1[side];
   const float* b1 = p.b1[side];
-  for (int idx = threadIdx.x; idx < kPosTok * p.hid; idx += blockDim.x) {
-    const int t = idx / p.hid, jh = idx - t * p.hid;
+  const float* gr = g + t * ldg;
+  for (int jh = q; jh < p.hid; jh += nq) {
     const float* wr = w1 + static_cast<size_t>(jh) * din;
-    const float* gr = g + t * din;
     float acc = __ldg(b1 + jh);
     for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
-    h[t * p.hid + jh] = gelu_erf(acc);
+    h[t * ldh + jh] = gelu_erf(acc);
   }
   __syncthreads();
+  const int tok = t0 + t;
+  if (tok >= p.N) return;
   const float* w2 = p.w2[side];
   const float* b2 = p.b2[side];
-  for (int idx = threadIdx.x; idx < kPosTok * p.dout; idx += blockDim.x) {
-    const int t = idx / p.dout, o = idx - t * p.dout;
-    const int tok = t0 + t;
-    if (tok >= p.N) continue;
+  const float* hr = h + t * ldh;
+  for (int o = q; o < p.dout; o += nq) {
     const float* wr = w2 + static_cast<size_t>(o) * p.hid;
-    const float* hr = h + t * p.hid;
     float acc = __ldg(b2 + o);
     for (int k = 0; k < p.hid; ++k) acc = fmaf(__ldg(wr + k), hr[k], acc);
     const int head = o / p.rank, r = o - head * p.rank;
@@ -115,68 +130,71 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   }
 }
 
-// Partial sums over kMlpBwdTok tokens of the position-MLP weight gradients.
+// Partial sums over kPosTok tokens of the position-MLP weight gradients.
 // grid (n_chunks, 2).  partial[side][chunk][:] = [dw1 | db1 | dw2 | db2].
 __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams p) {
   extern __shared__ float sm_pos[];
   const int side = blockIdx.y;
   const int chunk = blockIdx.x;
-  const int t0 = chunk * kMlpBwdTok;
+  const int t0 = chunk * kPosTok;
   const int din = 4 * p.F, hid = p.hid, dout = p.dout;
-  constexpr int T = kMlpBwdTok;
-  float* g = sm_pos;             // [T][din]  Fourier features
-  float* a = g + T * din;        // [T][hid]  pre-activation, then dL/da
-  float* h = a + T * hid;        // [T][hid]  GELU(a)
-  float* go = h + T * hid;       // [T][dout] dL/d(out)
-  fourier_tile(p, t0, T, g);
+  const int ldg = pad1(din), ldh = pad1(hid), ldo = pad1(dout);
+  constexpr int T = kPosTok;
+  float* g = sm_pos;             // [T][din+1]  Fourier features
+  float* h = g + T * ldg;        // [T][hid+1]  GELU(a)
+  float* da = h + T * ldh;       // [T][hid+1]  dL/da
+  float* go = da + T * ldh;      // [T][dout+1] dL/d(out)
+  fourier_tile(p, t0, g);
   for (int idx = threadIdx.x; idx < T * dout; idx += blockDim.x) {
-    const int t = idx / dout, o = idx - t * dout;
+    const int o = idx / T, t = idx - o * T;
     const int tok = t0 + t;
     const int head = o / p.rank, r = o - head * p.rank;
-    go[idx] = tok < p.N ? p.dtok[side][(static_cast<size_t>(head) * p.N + tok) * p.rank + r]
-                        : 0.f;
+    go[t * ldo + o] =
+        tok < p.N ? p.dtok[side][(static_cast<size_t>(head) * p.N + tok) * p.rank + r] : 0.f;
   }
   __syncthreads();
   const float* w1 = p.w1[side];
   const float* b1 = p.b1[side];
   const float* w2 = p.w2[side];
-  for (int idx = threadIdx.x; idx < T * hid; idx += blockDim.x) {
-    const int t = idx / hid, jh = idx - t * hid;
-    const float* wr = w1 + static_cast<size_t>(jh) * din;
-    const float* gr = g + t * din;
-    float acc = __ldg(b1 + jh);
-    for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
-    float dh = 0.f;
-    for (int o = 0; o < dout; ++o) dh = fmaf(__ldg(w2 + static_cast<size_t>(o) * hid + jh),
-                                             go[t * dout + o], dh);
-    h[idx] = gelu_erf(acc);
-    a[idx] = dh * gelu_erf_grad(acc);  // tokens past N have go == 0, so dL/da == 0
+  {
+    const int t = threadIdx.x % T, q = threadIdx.x / T, nq = blockDim.x / T;
+    const float* gr = g + t * ldg;
+    const float* gor = go + t * ldo;
+    for (int jh = q; jh < hid; jh += nq) {
+      const float* wr = w1 + static_cast<size_t>(jh) * din;
+      float acc = __ldg(b1 + jh);
+      for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
+      float dh = 0.f;
+      for (int o = 0; o < dout; ++o) dh = fmaf(__ldg(w2 + static_cast<size_t>(o) * hid + jh), gor[o], dh);
+      h[t * ldh + jh] = gelu_erf(acc);
+      da[t * ldh + jh] = dh * gelu_erf_grad(acc);  // tokens past N have go == 0
+    }
   }
   __syncthreads();
   float* out = p.partial + (static_cast<size_t>(side) * p.n_chunks + chunk) * p.n_params;
-  // dw1[jh][k] = sum_t da[t][jh] g[t][k]
+  // dw1[jh][k] = sum_t da[t][jh] g[t][k]  (warp: one jh, consecutive k)
   for (int idx = threadIdx.x; idx < hid * din; idx += blockDim.x) {
     const int jh = idx / din, k = idx - jh * din;
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc = fmaf(a[t * hid + jh], g[t * din + k], acc);
+    for (int t = 0; t < T; ++t) acc = fmaf(da[t * ldh + jh], g[t * ldg + k], acc);
     out[idx] = acc;
   }
   for (int jh = threadIdx.x; jh < hid; jh += blockDim.x) {
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc += a[t * hid + jh];
+    for (int t = 0; t < T; ++t) acc += da[t * ldh + jh];
     out[hid * din + jh] = acc;
   }
   float* o2 = out + hid * din + hid;
-  // dw2[o][jh] = sum_t go[t][o] h[t][jh]
+  // dw2[o][jh] = sum_t go[t][o] h[t][jh]  (warp: one o, consecutive jh)
   for (int idx = threadIdx.x; idx < dout * hid; idx += blockDim.x) {
     const int o = idx / hid, jh = idx - o * hid;
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc = fmaf(go[t * dout + o], h[t * hid + jh], acc);
+    for (int t = 0; t < T; ++t) acc = fmaf(go[t * ldo + o], h[t * ldh + jh], acc);
     o2[idx] = acc;
   }
   for (int o = threadIdx.x; o < dout; o += blockDim.x) {
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc += go[t * dout + o];
+    for (int t = 0; t < T; ++t) acc += go[t * ldo + o];
     o2[dout * hid + o] = acc;
   }
 }

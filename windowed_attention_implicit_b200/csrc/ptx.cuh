@@ -75,17 +75,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // when `abort` (a shared flag of the CTA) is set by another thread, or when
 // `limit_ns` elapses; in the latter case it records RIB_ERR_TIMEOUT with the
 // site code and raises the CTA's abort flag.  Returns true on success.
+// The retry loop polls only the barrier: the abort flag and the (slow to
+// read) global timer are checked once every 64 tries, so a waiter resumes
+// within a few cycles of the phase completing.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      record_error(kErrTimeout, site);
-      *abort = 1;
-      return false;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        record_error(kErrTimeout, site);
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
@@ -313,6 +318,65 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
   asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a),
                "f"(b), "f"(c), "f"(d)
                : "memory");
+}
+
+
+// ---------------------------------------------------------------- packed fp32
+// Two fp32 values in one 64-bit register pair (low = first).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) |
+         (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi2(uint64_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two packed x <= 8 on the FMA pipe (no MUFU).
+// Cody-Waite reduction: n = round(x) via the 1.5*2^23 rounding constant,
+// f = x - n in [-1/2, 1/2] (exact); 2^f from the degree-3 polynomial that
+// minimises the maximum relative error on [-1/2, 1/2] (Remez exchange,
+// csrc/fit_exp2_poly.py: 7.5e-5); 2^n is added to the exponent field.
+// x is clamped at -125 so the exponent stays normal (2^-125 is negligible
+// wherever this feeds a bf16 softmax numerator).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  const float xl = fmaxf(lo2(x2), -125.f), xh = fmaxf(hi2(x2), -125.f);
+  const uint64_t xc = pk2(xl, xh);
+  const uint64_t t = fadd2(xc, pk2(kRoundMagic, kRoundMagic));
+  const uint64_t nf = fadd2(t, pk2(-kRoundMagic, -kRoundMagic));
+  const uint64_t f = ffma2(nf, pk2(-1.f, -1.f), xc);
+  uint64_t p = ffma2(pk2(kExp2C3, kExp2C3), f, pk2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, pk2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, pk2(kExp2C0, kExp2C0));
+  const uint32_t rl = static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23);
+  const uint32_t rh = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+  return static_cast<uint64_t>(rl) | (static_cast<uint64_t>(rh) << 32);
 }
 
 template <typename T>

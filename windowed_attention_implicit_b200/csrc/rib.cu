@@ -90,6 +90,17 @@ int map_pos(CUtensorMap* m, const void* base, int heads, int M) {
                   CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
+// The same tensor fetched as 64-byte rows: the box is 32 channels wide, so
+// TMA zero-fills channels 16..31 (out of bounds), giving a 64B-swizzle tile
+// that sits beside a content tile as a second atom of one MMA operand.
+int map_pos_padded(CUtensorMap* m, const void* base, int heads, int M) {
+  const uint64_t dims[4] = {16, (uint64_t)M, (uint64_t)M, (uint64_t)heads};
+  const uint64_t strides[3] = {32, 32ull * M, 32ull * M * M};
+  const uint32_t box[4] = {32, 8, 8, 1};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 // per-pixel fp32 [B][heads][H][W], 8x8-pixel boxes.
 int map_pixel_f32(CUtensorMap* m, const void* base, int B, int heads, int H, int W) {
   const uint64_t dims[4] = {(uint64_t)W, (uint64_t)H, (uint64_t)heads, (uint64_t)B};
@@ -258,7 +269,8 @@ int launch_mlp_bwd(const rib_mlp_t* mlp, int window, const float* dqp, const flo
   pp.grads[0][2] = dmlp->q_dw2; pp.grads[0][3] = dmlp->q_db2;
   pp.grads[1][0] = dmlp->k_dw1; pp.grads[1][1] = dmlp->k_db1;
   pp.grads[1][2] = dmlp->k_dw2; pp.grads[1][3] = dmlp->k_db2;
-  const size_t smem = (size_t)kMlpBwdTok * (4 * pp.F + 2 * pp.hid + pp.dout) * sizeof(float);
+  const size_t smem = mlp_bwd_smem_floats(pp.F, pp.hid, pp.dout) * sizeof(float);
+  if (smem > 200 * 1024) return RIB_ERR_UNSUPPORTED;
   int rc;
   if ((rc = set_smem(mlp_bwd_partial_kernel, smem))) return rc;
   {
@@ -289,6 +301,14 @@ __global__ void debug_wait_kernel(unsigned long long limit_ns) {
   __syncthreads();
   // Nothing ever arrives on `bar`: the wait must run out and record a timeout.
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns, SITE_DEBUG);
+}
+
+__global__ void debug_exp2_kernel(const float* x, float* y, int n_pairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pairs) return;
+  const uint64_t r = exp2_fma2(pk2(x[2 * i], x[2 * i + 1]));
+  y[2 * i] = lo2(r);
+  y[2 * i + 1] = hi2(r);
 }
 
 }  // namespace
@@ -367,6 +387,14 @@ int rib_trace_collect(rib_trace_entry_t* entries, int max_entries, int* n_entrie
   return rc;
 }
 
+int rib_debug_exp2(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 0 || (n & 1)) return RIB_ERR_ARG;
+  if (n == 0) return RIB_OK;
+  const int pairs = n / 2;
+  debug_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, pairs);
+  return launch_status();
+}
+
 int rib_debug_wait_timeout(unsigned long long limit_ns, void* stream) {
   debug_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
   return launch_status();
@@ -384,7 +412,8 @@ int rib_pos_tokens(const rib_mlp_t* mlp, int window, float* qp, float* kp, void*
   p.out32[1] = kp;
   p.out16[0] = static_cast<__nv_bfloat16*>(qp_bf16);
   p.out16[1] = static_cast<__nv_bfloat16*>(kp_bf16);
-  const size_t smem = (size_t)kPosTok * (4 * p.F + p.hid) * sizeof(float);
+  const size_t smem = pos_fwd_smem_floats(p.F, p.hid) * sizeof(float);
+  if (smem > 200 * 1024) return RIB_ERR_UNSUPPORTED;
   if ((rc = set_smem(pos_tokens_kernel, smem))) return rc;
   dim3 grid((p.N + kPosTok - 1) / kPosTok, 2);
   TraceScope ts(K_POS, static_cast<cudaStream_t>(stream));
@@ -517,8 +546,8 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
   if ((rc = map_pixel_f32(&tl, a.lse2, B, heads, H, W))) return rc;
   if ((rc = map_pixel_f32(&td, a.dd, B, heads, H, W))) return rc;
   if (rank > 0) {
-    if ((rc = map_pos(&tqp, qp_bf16, heads, window))) return rc;
-    if ((rc = map_pos(&tkp, kp_bf16, heads, window))) return rc;
+    if ((rc = map_pos_padded(&tqp, qp_bf16, heads, window))) return rc;
+    if ((rc = map_pos_padded(&tkp, kp_bf16, heads, window))) return rc;
   } else {
     tqp = tq;
     tkp = tq;
