@@ -118,6 +118,35 @@ int rib_pos_tokens_bwd(const rib_mlp_t* mlp, int window, const float* dqp,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * rib_pos_tokens_bwd_noalloc -- rib_pos_tokens_bwd without a workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory when they need the gradients: code that
+ * runs while a CUDA graph is being captured (cudaMalloc is not allowed
+ * there), hosts and plugins whose allocator owns every device byte, and
+ * latency-bound loops that cannot afford the device-wide synchronisation a
+ * cudaMalloc/cudaFree pair implies.  It computes exactly what
+ * rib_pos_tokens_bwd computes, using a scratch area that is part of the
+ * library itself: a statically allocated device array of
+ * RIB_NOALLOC_SCRATCH_BYTES (24 MiB), which every GPU that loads the library
+ * keeps until the process exits.  Sizes whose scratch need
+ * (rib_pos_tokens_bwd_workspace) exceeds that return RIB_ERR_WORKSPACE.
+ *
+ *   The first call on each device looks up the device address of the array
+ *   (a host-side step, done once per device with that device current); make
+ *   that first call before any stream capture begins.
+ *   All calls share the one array: calls whose kernels may overlap on the
+ *   GPU (different streams without ordering between them) race on it and
+ *   give undefined results.  Every scratch byte a call reads is written by
+ *   the same call first, so no clearing is needed between calls.
+ *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * ------------------------------------------------------------------------ */
+#define RIB_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
+int rib_pos_tokens_bwd_noalloc(const rib_mlp_t* mlp, int window, const float* dqp,
+                               const float* dkp, const rib_mlp_grad_t* dmlp,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
  * rib_window_attn_fwd -- RIB window attention forward.
  *
  * English summary §2.A steps 3-4 and the score equation; the paper's

@@ -24,7 +24,7 @@ from . import _abi
 
 __all__ = [
     "RibError", "PositionMLP", "PositionMLPGrad", "PosTokenCache", "rib_pos_tokens",
-    "rib_pos_tokens_bwd", "rib_pos_tokens_bwd_workspace",
+    "rib_pos_tokens_bwd", "rib_pos_tokens_bwd_workspace", "rib_pos_tokens_bwd_noalloc",
     "rib_window_attn_fwd", "rib_window_attn_bwd", "rib_window_attn_bwd_workspace",
     "rib_window_gather", "rib_window_scatter", "rib_last_status", "rib_status_string",
     "rib_set_wait_limit_ns", "rib_debug_wait_timeout", "rib_version", "library",
@@ -180,6 +180,23 @@ def rib_pos_tokens_bwd(mlp: PositionMLP, window: int, dqp: torch.Tensor, dkp: to
         ctypes.byref(c), int(window), _ptr(dqp, torch.float32, "dqp"),
         _ptr(dkp, torch.float32, "dkp"), ctypes.byref(cg), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "rib_pos_tokens_bwd")
+    return dmlp
+
+
+def rib_pos_tokens_bwd_noalloc(mlp: PositionMLP, window: int, dqp: torch.Tensor,
+                               dkp: torch.Tensor, dmlp: "PositionMLPGrad", stream=None):
+    """rib_pos_tokens_bwd for callers that cannot allocate device memory at
+    the point of the call (inside CUDA graph capture, under an allocator that
+    owns all device memory, or where cudaMalloc's synchronisation is too
+    costly).  The library's own static 24 MiB device scratch is used instead
+    of a workspace; `dmlp` must be given (preallocated).  Calls that overlap
+    on the GPU share that scratch and race; the first call on a device should
+    precede any stream capture."""
+    c, cg = mlp.c_struct(), dmlp.c_struct()
+    _check(library().rib_pos_tokens_bwd_noalloc(
+        ctypes.byref(c), int(window), _ptr(dqp, torch.float32, "dqp"),
+        _ptr(dkp, torch.float32, "dkp"), ctypes.byref(cg), _stream(stream)),
+        "rib_pos_tokens_bwd_noalloc")
     return dmlp
 
 

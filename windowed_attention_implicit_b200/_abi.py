@@ -15,6 +15,7 @@ RIB_ERR_WORKSPACE = -4
 RIB_ERR_CUDA = -5
 RIB_ERR_TIMEOUT = -6
 RIB_ERR_ALIGN = -7
+RIB_NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
 
 _p = ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
@@ -45,6 +46,8 @@ _SIGS = {
     "rib_pos_tokens_bwd_workspace": (ctypes.c_size_t, [ctypes.POINTER(rib_mlp_t), _i]),
     "rib_pos_tokens_bwd": (_i, [ctypes.POINTER(rib_mlp_t), _i, _p, _p,
                                 ctypes.POINTER(rib_mlp_grad_t), _p, ctypes.c_size_t, _p]),
+    "rib_pos_tokens_bwd_noalloc": (_i, [ctypes.POINTER(rib_mlp_t), _i, _p, _p,
+                                        ctypes.POINTER(rib_mlp_grad_t), _p]),
     "rib_window_attn_fwd": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
                                  ctypes.c_float, _p, _p, _p]),
     "rib_window_attn_bwd_workspace": (ctypes.c_size_t,

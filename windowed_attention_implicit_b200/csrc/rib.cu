@@ -290,6 +290,30 @@ bool mlp_grad_complete(const rib_mlp_grad_t* d) {
          d->k_dw2 && d->k_db2;
 }
 
+// Scratch of rib_pos_tokens_bwd_noalloc: part of the library image, one copy
+// per device.  Host code cannot take its address directly (the name is a
+// host-side stand-in), so each device's address is looked up once with
+// cudaGetSymbolAddress and cached here.
+__device__ __align__(256) unsigned char g_noalloc_scratch[RIB_NOALLOC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (set up on first use).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RIB_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return RIB_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RIB_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return RIB_OK;
+}
+
 __global__ void debug_wait_kernel(unsigned long long limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -446,6 +470,24 @@ int rib_pos_tokens_bwd(const rib_mlp_t* mlp, int window, const float* dqp, const
   const int n_params = mlp->d_hidden * 4 * mlp->n_freq + mlp->d_hidden +
                        mlp->heads * mlp->rank * mlp->d_hidden + mlp->heads * mlp->rank;
   return launch_mlp_bwd(mlp, window, dqp, dkp, dmlp, workspace, n_chunks, n_params,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int rib_pos_tokens_bwd_noalloc(const rib_mlp_t* mlp, int window, const float* dqp,
+                               const float* dkp, const rib_mlp_grad_t* dmlp, void* stream) {
+  int rc = check_mlp(mlp);
+  if (rc) return rc;
+  if (window <= 0 || !dqp || !dkp || !mlp_grad_complete(dmlp)) return RIB_ERR_ARG;
+  if (window > 256) return RIB_ERR_UNSUPPORTED;
+  if (rib_pos_tokens_bwd_workspace(mlp, window) > RIB_NOALLOC_SCRATCH_BYTES)
+    return RIB_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  const int N = window * window;
+  const int n_chunks = (N + kMlpBwdTok - 1) / kMlpBwdTok;
+  const int n_params = mlp->d_hidden * 4 * mlp->n_freq + mlp->d_hidden +
+                       mlp->heads * mlp->rank * mlp->d_hidden + mlp->heads * mlp->rank;
+  return launch_mlp_bwd(mlp, window, dqp, dkp, dmlp, scratch, n_chunks, n_params,
                         static_cast<cudaStream_t>(stream));
 }
 
