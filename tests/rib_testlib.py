@@ -28,8 +28,9 @@ def stats(got, ref):
 def check_close(got, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS, normalize=False):
     """Returns an error message ('' if within bounds).  normalize=True divides
     the errors by max(1, max|ref|) first, and a number divides them by
-    max(1, that number) (used for fp32 sums whose magnitude grows with the
-    number of tokens summed)."""
+    max(1, that number): used for fp32 sums whose magnitude grows with the
+    number of windows or tokens summed (dQp, dKp, MLP weight gradients),
+    whose bf16-level errors grow in proportion."""
     mx, mn = stats(got, ref)
     if normalize is True:
         scale = max(1.0, float(np.abs(np.asarray(ref, dtype=np.float64)).max()))

@@ -118,8 +118,8 @@ def test_bwd_parity(case):
     checks = [check_close(got[:, :, :, k], dq[:, :, :, k], name)
               for k, name in enumerate(("dQc", "dKc", "dV"))]
     if rank:
-        checks.append(check_close(to_np(g["dqp"]), dqp, "dQp"))
-        checks.append(check_close(to_np(g["dkp"]), dkp, "dKp"))
+        checks.append(check_close(to_np(g["dqp"]), dqp, "dQp", normalize=True))
+        checks.append(check_close(to_np(g["dkp"]), dkp, "dKp", normalize=True))
     assert_all(checks)
 
 
@@ -137,7 +137,7 @@ def test_bwd_mlp_grads_parity():
     _, dqp, dkp = c.oracle_bwd()
     (gq, gk) = O.pos_tokens_backward(c.freqs, c.mlp_q, c.mlp_k, M, dqp, dkp)
     dm = g["dmlp"]
-    checks = [check_close(to_np(g["dqp"]), dqp, "dQp"), check_close(to_np(g["dkp"]), dkp, "dKp")]
+    checks = [check_close(to_np(g["dqp"]), dqp, "dQp", normalize=True), check_close(to_np(g["dkp"]), dkp, "dKp", normalize=True)]
     checks += mlp_grad_checks(dm, gq, gk)
     assert_all(checks)
 

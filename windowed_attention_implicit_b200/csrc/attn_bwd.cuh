@@ -17,22 +17,29 @@
 //   dq_finalize      dQ content channels -> bf16 dqkv at the rolled pixels
 //   posgrad_reduce   fixed-order sums over (batch, window) of dQp, dKp
 //
-// attn_bwd_kernel, 320 threads:
-//   warps 0-7  compute: thread = key row (TMEM lane), warps 0-3 take query
-//              columns 0-63 and warps 4-7 columns 64-127 of each tile
-//   warp  8    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 4 stages: the
-//              prefetch distance must cover the TMA latency of a tile)
-//   warp  9    TMEM allocator; issues the S^T / dP^T MMAs
-//   warp 10    issues the gradient MMAs (dV, dK_aug, dQ_aug)
-// Two issuing threads: a tcgen05.mma blocks its issuing thread for ~45
-// cycles, so with one issuer the scores of tile i+1 could only be issued
-// after the 24 gradient MMAs of tile i-1, serialising MMAs and
-// exponentials.
+// attn_bwd_kernel, 512 threads (4 warpgroups):
+//   warps 0-7   compute: thread = key row (TMEM lane), warps 0-3 take query
+//               columns 0-63 and warps 4-7 columns 64-127 of each tile
+//               (168 registers each after setmaxnreg)
+//   warps 8-11  dQ drain: TMEM -> shared-memory staging tile -> one bulk
+//               TMA reduce-add into the fp32 accumulator per query tile
+//   warp  12    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 4 stages)
+//   warp  13    issues the S^T / dP^T MMAs
+//   warp  14    TMEM allocator; issues the gradient MMAs (dV, dK_aug, dQ_aug)
+//   warp  15    idle
+// The tensor pipe runs all of these back to back only if no single thread's
+// waits stall it: a tcgen05.mma blocks its issuing thread for ~45 cycles and
+// a tcgen05.commit for ~270, so scores and gradients have separate issuers;
+// and the compute warps neither drain dQ (dedicated warps do) nor wait for
+// the previous tile's gradient MMAs before their exponentials (they form the
+// whole tile in registers first, then wait for the P^T/dS^T buffers).
 // Per query tile i:  S^T = K_aug Q_aug^T and dP^T = V dO^T (MMA, TMEM) ->
 // compute warps form P^T and dS^T (to TMEM) and dS (to shared memory,
 // core-matrix layout, double-buffered) -> MMA: dV += P^T dO and
 // dK_aug += dS^T [Qc|Qp] (A from TMEM), dQ_aug = dS [Kc|Kp] (A from shared
-// memory) -> compute warps drain dQ with red.global.add.v4.f32.
+// memory) -> drain warps fold dQ into the fp32 accumulator with one bulk
+// reduce-add per tile (per-thread vector atomics cost more L2 time than the
+// whole rest of the kernel).
 // At d = 32 the MMAs are narrow: a tcgen05.mma of M=128, K=16 costs ~40-50
 // cycles however small N is, and with both operands in shared memory an
 // N <= 64 MMA moves more bytes than its flops cover.  So the A operand comes
@@ -53,7 +60,13 @@
 namespace rib {
 
 constexpr int kBwdStages = 4;
-constexpr int kBwdThreads = 352;
+constexpr int kBwdThreads = 512;
+constexpr int kBwdLaunchRegs = 128;     // 65536 / 512: what the host checks ptxas gave
+constexpr int kBwdComputeRegs = 168;    // warpgroups 0-1
+constexpr int kBwdServiceRegs = 80;     // warpgroups 2-3
+static_assert(2 * 128 * kBwdComputeRegs + 2 * 128 * kBwdServiceRegs <=
+                  kBwdThreads * kBwdLaunchRegs,
+              "register split exceeds the launch budget");
 constexpr uint32_t kBwdTmemCols = 512;
 // TMEM columns (512): S^T, dP^T fp32; P^T, dS^T bf16; dV; dK = [dKc | dKp];
 // dQ = [dQc | dQp]
@@ -73,7 +86,7 @@ struct BwdParams {
   float scale;       // tau
   float scale_log2;  // tau * log2(e)
   __nv_bfloat16* dqkv;
-  float* dq_acc;     // [units][n_tiles][128][48]
+  float* dq_acc;     // [units][n_tiles][48][128]  (channel-major per tile)
   float* dkp_part;   // [units][n_tiles][128][16]
   uint64_t wait_limit_ns;
 };
@@ -86,12 +99,14 @@ struct __align__(1024) BwdSmem {
   uint8_t qc[kBwdStages][8192];
   uint8_t qp[kBwdStages][8192];    // positional, zero-padded (qc + kBwdStages * 8 KB)
   uint8_t dO[kBwdStages][8192];
+  float dq_stage[48 * 128];        // dQ of one query tile, [channel][row], for the bulk reduce
   float lse2[kBwdStages][128];     // -lse * log2(e), tile row order
   float dd[kBwdStages][128];       // -D = -rowsum(dO * O), tile row order
   uint64_t k_full;
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
   uint64_t s_full, s_free, ds_full, pt_free /* P^T and dS^T in TMEM */, ds_free[2];
-  uint64_t dq_full, dq_free;
+  uint64_t dq_full, dq_free, mma_done;
+  int drain_ok[4];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -241,59 +256,63 @@ __device__ __forceinline__ void bwd_mma_grads(BwdSmem& sm, uint32_t tmem, const 
     umma_commit(&sm.dq_full);
     umma_commit(&sm.q_empty[st]);
   }
+  umma_commit(&sm.mma_done);   // every gradient MMA of the kernel has completed
   umma_commit(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
 }
 
-// Drains dQ of query tile `it` from TMEM into the fp32 accumulator.
-// Group 0 takes columns 0-23, group 1 columns 24-47 (32-47 = dQp).
-__device__ __forceinline__ bool bwd_drain_dq(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
-                                             int unit, int it, int g, int wq, bool pos) {
+// Warps 8-11: drain dQ of every query tile from TMEM into the staging tile
+// (lane quarter wq = warp & 3, all 48 channels), then one thread folds the
+// tile into the fp32 accumulator with a bulk reduce-add.
+constexpr int kDrainBar = 1;   // named barrier of the 4 drain warps
+__device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
+                                          int unit, int wq) {
   volatile int* ab = &sm.abort_flag;
   const int lane = threadIdx.x & 31;
-  if (!warp_wait(&sm.dq_full, it & 1, ab, p.wait_limit_ns, SITE_BWD_COMPUTE)) return false;
-  tc_fence_after();
+  const bool pos = p.rank > 0;
+  const bool leader = wq == 0 && lane == 0;
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-  uint32_t r16[16] = {0}, r8[8];
-  if (g == 0) {
-    tmem_ld_x16(tmem + lane_off + kBColDQ, r16);
-    tmem_ld_x8(tmem + lane_off + kBColDQ + 16, r8);
-  } else {
-    tmem_ld_x8(tmem + lane_off + kBColDQ + 24, r8);
-    if (pos) tmem_ld_x16(tmem + lane_off + kBColDQ + 32, r16);
-  }
-  tmem_wait_ld();
-  reg_fence_x16(r16);
-  reg_fence_x8(r8);
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&sm.dq_free);
   const int row = wq * 32 + lane;
-  float* dst = p.dq_acc + ((static_cast<size_t>(unit) * p.n_tiles + it) * 128 + row) * 48;
-  auto f = [](uint32_t x) { return __uint_as_float(x); };
-  if (g == 0) {
+  const uint32_t tile_bytes = 48u * 128u * 4u;
+  volatile int* drain_ok = sm.drain_ok;
+  for (int it = 0; it < p.n_tiles; ++it) {
+    const bool ok = warp_wait(&sm.dq_full, it & 1, ab, p.wait_limit_ns, SITE_BWD_COMPUTE);
+    tc_fence_after();
+    uint32_t r32[32], r16[16] = {0};
+    if (ok) {
+      tmem_ld_x32(tmem + lane_off + kBColDQ, r32);
+      if (pos) tmem_ld_x16(tmem + lane_off + kBColDQ + 32, r16);
+      tmem_wait_ld();
+      reg_fence_x32(r32);
+      reg_fence_x16(r16);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.dq_free);
+    }
+    if (lane == 0) drain_ok[wq] = ok ? 1 : 0;
+    // the staging tile is free once the previous bulk reduce has read it
+    if (leader) tma_store_wait_read_all();
+    named_bar_sync(kDrainBar, 128);
+    // every drain thread reads the same four flags: one decision for all
+    const bool all_ok = drain_ok[0] && drain_ok[1] && drain_ok[2] && drain_ok[3];
+    if (all_ok) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      red_add_v4(dst + 4 * q, f(r16[4 * q]), f(r16[4 * q + 1]), f(r16[4 * q + 2]),
-                 f(r16[4 * q + 3]));
+      for (int c = 0; c < 32; ++c) sm.dq_stage[c * 128 + row] = __uint_as_float(r32[c]);
 #pragma unroll
-    for (int q = 0; q < 2; ++q)
-      red_add_v4(dst + 16 + 4 * q, f(r8[4 * q]), f(r8[4 * q + 1]), f(r8[4 * q + 2]),
-                 f(r8[4 * q + 3]));
-  } else {
-#pragma unroll
-    for (int q = 0; q < 2; ++q)
-      red_add_v4(dst + 24 + 4 * q, f(r8[4 * q]), f(r8[4 * q + 1]), f(r8[4 * q + 2]),
-                 f(r8[4 * q + 3]));
-    if (pos) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        red_add_v4(dst + 32 + 4 * q, f(r16[4 * q]), f(r16[4 * q + 1]), f(r16[4 * q + 2]),
-                   f(r16[4 * q + 3]));
+      for (int c = 0; c < 16; ++c) sm.dq_stage[(32 + c) * 128 + row] = __uint_as_float(r16[c]);
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(kDrainBar, 128);
+    if (!all_ok) break;
+    if (leader) {
+      bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(unit) * p.n_tiles + it) * 48 * 128,
+                          sm.dq_stage, tile_bytes);
+      tma_store_commit();
     }
   }
-  return true;
+  // the reductions must be complete before the kernel's work is considered done
+  if (leader) tma_store_wait_all();
 }
 
 __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
@@ -329,6 +348,34 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     // lse*log2e and D of this query tile (written by TMA)
     if (!(ok = warp_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_COMPUTE)))
       break;
+    const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[st] + 64 * g);
+    const float4* dd4 = reinterpret_cast<const float4*>(sm.dd[st] + 64 * g);
+    // the whole 64-column slice in registers: P and dS, packed bf16 pairs
+    uint32_t pk[32], dk[32];
+#pragma unroll
+    for (int v4 = 0; v4 < 16; ++v4) {
+      const float4 l = lse4[v4];    // -lse*log2e
+      const float4 dv = dd4[v4];    // -D
+      const uint32_t* sc = &s[v4 >> 3][(v4 & 7) * 4];
+      const uint32_t* dc = &dp[v4 >> 3][(v4 & 7) * 4];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const uint64_t nl = h2 ? pk2(l.z, l.w) : pk2(l.x, l.y);
+        const uint64_t nd = h2 ? pk2(dv.z, dv.w) : pk2(dv.x, dv.y);
+        const uint64_t x2 = ffma2(pk2(__uint_as_float(sc[2 * h2]), __uint_as_float(sc[2 * h2 + 1])),
+                                  sl2, nl);
+        uint64_t p2;
+        if (((2 * v4 + h2) & 7) < kBwdPolyPairs) {
+          p2 = exp2_fma2(x2);
+        } else {
+          p2 = pk2(ex2_approx(lo2(x2)), ex2_approx(hi2(x2)));
+        }
+        const uint64_t d2 = fmul2(p2, fadd2(pk2(__uint_as_float(dc[2 * h2]),
+                                                __uint_as_float(dc[2 * h2 + 1])), nd));
+        pk[2 * v4 + h2] = pack_bf16x2(lo2(p2), hi2(p2));
+        dk[2 * v4 + h2] = pack_bf16x2(lo2(d2), hi2(d2));
+      }
+    }
     // P^T and dS^T (TMEM) are free once dV(i-1), dK(i-1) completed; the dS
     // buffer i&1 (shared memory) once tile i-2's dQ MMAs completed.
     if (i > 0 && !(ok = warp_wait(&sm.pt_free, (i - 1) & 1, ab, lim, SITE_BWD_COMPUTE))) break;
@@ -337,54 +384,29 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
       break;
     tc_fence_after();
     uint8_t* ds_row = sm.ds[i & 1];
-    const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[st] + 64 * g);
-    const float4* dd4 = reinterpret_cast<const float4*>(sm.dd[st] + 64 * g);
-    // 16 query columns at a time: P^T and dS^T to TMEM, dS to shared memory.
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
-      const uint32_t* sc = &s[ch >> 1][(ch & 1) * 16];
-      const uint32_t* dc = &dp[ch >> 1][(ch & 1) * 16];
-      uint32_t pk[8], dk[8];
+      uint32_t p8[8], d8[8];
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
-        const float4 l = lse4[ch * 4 + v4];    // -lse*log2e
-        const float4 dv = dd4[ch * 4 + v4];    // -D
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int e = 4 * v4 + 2 * h2;       // element pair (e, e+1) of the chunk
-          const uint64_t nl = h2 ? pk2(l.z, l.w) : pk2(l.x, l.y);
-          const uint64_t nd = h2 ? pk2(dv.z, dv.w) : pk2(dv.x, dv.y);
-          const uint64_t x2 = ffma2(pk2(__uint_as_float(sc[e]), __uint_as_float(sc[e + 1])),
-                                    sl2, nl);
-          uint64_t p2;
-          if (2 * v4 + h2 < kBwdPolyPairs) {
-            p2 = exp2_fma2(x2);
-          } else {
-            p2 = pk2(ex2_approx(lo2(x2)), ex2_approx(hi2(x2)));
-          }
-          const uint64_t d2 = fmul2(p2, fadd2(pk2(__uint_as_float(dc[e]),
-                                                  __uint_as_float(dc[e + 1])), nd));
-          pk[e >> 1] = pack_bf16x2(lo2(p2), hi2(p2));
-          dk[e >> 1] = pack_bf16x2(lo2(d2), hi2(d2));
-        }
+      for (int e = 0; e < 8; ++e) {
+        p8[e] = pk[8 * ch + e];
+        d8[e] = dk[8 * ch + e];
       }
-      tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, pk);
-      tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, dk);
+      tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, p8);
+      tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, d8);
       const int q = 64 * g + 16 * ch;
-      *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+      *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) = make_uint4(d8[0], d8[1], d8[2], d8[3]);
       *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q + 8)) =
-          make_uint4(dk[4], dk[5], dk[6], dk[7]);
+          make_uint4(d8[4], d8[5], d8[6], d8[7]);
     }
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.ds_full);
-    if (i > 0 && !(ok = bwd_drain_dq(sm, tmem, p, unit, i - 1, g, wq, pos))) break;
   }
   if (!ok) return;
-  // dq_full(n-1) is committed after every MMA of the kernel
-  if (!bwd_drain_dq(sm, tmem, p, unit, n - 1, g, wq, pos)) return;
+  if (!warp_wait(&sm.mma_done, 0, ab, lim, SITE_BWD_COMPUTE)) return;
   tc_fence_after();
   int i0, j0, ii, jl;
   tile_origin(kt, p.tiles_x, i0, j0);
@@ -463,18 +485,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.ds_free[0], 1);
     mbar_init(&sm.ds_free[1], 1);
     mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_free, 8);
+    mbar_init(&sm.dq_free, 4);
+    mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_dout);
     tma_prefetch_desc(&tm_lse2);
     tma_prefetch_desc(&tm_dd);
   }
-  if (warp == 9) {
+  if (warp == 14) {
     tmem_alloc(&sm.tmem_base, kBwdTmemCols);
     tmem_relinquish();
   }
@@ -483,17 +506,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   if (warp < 8) {
+    regs_inc<kBwdComputeRegs>();
     bwd_compute(sm, tmem, p, u, unit, kt, warp >> 2, warp & 3);
-  } else if (warp == 8) {
-    if (lane == 0) bwd_producer(sm, &tm_qkv, &tm_dout, &tm_qp, &tm_kp, &tm_lse2, &tm_dd, p, u, kt);
-  } else if (warp == 9) {
-    if (lane == 0) bwd_mma_scores(sm, tmem, p);
   } else {
-    if (lane == 0) bwd_mma_grads(sm, tmem, p);
+    regs_dec<kBwdServiceRegs>();
+    if (warp < 12) {
+      bwd_drain(sm, tmem, p, unit, warp & 3);
+    } else if (warp == 12) {
+      if (lane == 0) bwd_producer(sm, &tm_qkv, &tm_dout, &tm_qp, &tm_kp, &tm_lse2, &tm_dd, p, u, kt);
+    } else if (warp == 13) {
+      if (lane == 0) bwd_mma_scores(sm, tmem, p);
+    } else if (warp == 14) {
+      if (lane == 0) bwd_mma_grads(sm, tmem, p);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 14) {
     tc_fence_after();
     tmem_dealloc(tmem, kBwdTmemCols);
   }
@@ -509,7 +538,7 @@ struct BwdAuxParams {
   const float* lse;
   float* lse2;      // [B][heads][H][W]
   float* dd;        // [B][heads][H][W]
-  float* dq_acc;    // [units][n_tiles][128][48]
+  float* dq_acc;    // [units][n_tiles][48][128]
   const float* dkp_part;
   size_t dq_acc_floats;
   __nv_bfloat16* dqkv;
@@ -572,15 +601,15 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(const BwdAuxParams p) 
   tile_row_local(row, i0, j0, i, j);
   const int y = wrap_once(u.wy * p.M + i + p.s, p.H);
   const int x = wrap_once(u.wx * p.M + j + p.s, p.W);
-  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + idx * 48);
+  const float* src = p.dq_acc + (ut * 48) * 128 + row;     // [tile][channel][row]
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
   uint4* dst = reinterpret_cast<uint4*>(p.dqkv + (pix * 3 * p.heads + u.head) * 32);
   const float t = p.scale;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const float4 a = src[2 * q], b = src[2 * q + 1];
-    dst[q] = make_uint4(pack_bf16x2(a.x * t, a.y * t), pack_bf16x2(a.z * t, a.w * t),
-                        pack_bf16x2(b.x * t, b.y * t), pack_bf16x2(b.z * t, b.w * t));
+    const float* c = src + 8 * q * 128;
+    dst[q] = make_uint4(pack_bf16x2(c[0] * t, c[128] * t), pack_bf16x2(c[256] * t, c[384] * t),
+                        pack_bf16x2(c[512] * t, c[640] * t), pack_bf16x2(c[768] * t, c[896] * t));
   }
 }
 
@@ -601,9 +630,9 @@ __global__ void __launch_bounds__(256) posgrad_reduce_kernel(const BwdAuxParams 
   const int bw_units = p.B * p.nW;
   for (int bw = 0; bw < bw_units; ++bw) {
     const size_t unit = static_cast<size_t>(bw) * p.heads + h;
-    const size_t rr = (unit * p.n_tiles + tile) * 128 + row;
-    aq += p.dq_acc[rr * 48 + 32 + r];
-    ak += p.dkp_part[rr * 16 + r];
+    const size_t ut = unit * p.n_tiles + tile;
+    aq += p.dq_acc[(ut * 48 + 32 + r) * 128 + row];
+    ak += p.dkp_part[(ut * 128 + row) * 16 + r];
   }
   p.dqp[idx] = aq * p.scale;
   p.dkp[idx] = ak;

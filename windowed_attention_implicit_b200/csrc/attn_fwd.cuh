@@ -18,7 +18,11 @@
 //   warps 4-7  softmax group B
 //   warp  8    TMA producer: Q tiles once, then K/V/Kp tiles through a
 //              3-stage shared-memory ring; boxes at rolled map coordinates
-//   warp  9    TMEM allocator and MMA issuer (one thread)
+//   warp  9    TMEM allocator; issues the score MMAs S_X(j) = Q_X K_j^T
+//   warp 10    issues the PV MMAs and releases K/V stages
+// A tcgen05.commit blocks its issuing thread until the thread's MMAs have
+// completed (~270 cycles), so scores and PV are issued by two threads: one
+// thread's commit never leaves the tensor pipe idle.
 // TMEM (512 columns): S_A, S_B fp32 [128 x 128]; P_A, P_B bf16 [128 x 128]
 // (64 packed columns each); [O|L]_A, [O|L]_B fp32 [128 x 48].
 // Per key tile j and group X: S_X(j) = Q_X K_j^T (MMA) -> online softmax in
@@ -42,7 +46,7 @@
 namespace rib {
 
 constexpr int kFwdStages = 3;
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 352;
 constexpr uint32_t kFwdTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // O_X at kColO + 48 X, L at +32
 constexpr int kOCols = 48;
@@ -130,49 +134,52 @@ __device__ __forceinline__ void fwd_producer(FwdSmem& sm, const CUtensorMap* tq,
   }
 }
 
-__device__ __forceinline__ void fwd_mma(FwdSmem& sm, uint32_t tmem, const FwdParams& p) {
+// Warp 9: S_X(j) = Q_X K_j^T for both query tiles of every key tile, each as
+// soon as group X has pulled S_X(j-1) into registers.
+__device__ __forceinline__ void fwd_mma_scores(FwdSmem& sm, uint32_t tmem, const FwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const bool pos = p.rank > 0;
   const int n = p.n_tiles;
-  auto issue_s = [&](int X, int st) {
-    const uint32_t d = tmem + kColS + X * 128;
-    const uint64_t a = make_sdesc(smem_u32(sm.qc[X]), 16, 512, kLayoutSW64);
-    const uint64_t b = make_sdesc(smem_u32(sm.kc[st]), 16, 512, kLayoutSW64);
-    umma_ss(d, a, b, kIdescS, 0u);
-    umma_ss(d, a + 2, b + 2, kIdescS, 1u);  // channels 16..31: start address + 32 B
-    if (pos)
-      umma_ss(d, make_sdesc(smem_u32(sm.qp[X]), 16, 256, kLayoutSW32),
-              make_sdesc(smem_u32(sm.kp[st]), 16, 256, kLayoutSW32), kIdescS, 1u);
-    umma_commit(&sm.s_full[X]);
-  };
-  bool ok = mbar_wait(&sm.q_full, 0, ab, lim, SITE_FWD_MMA) &&
-            mbar_wait(&sm.kv_full[0], 0, ab, lim, SITE_FWD_MMA);
-  if (ok) {
-    tc_fence_after();
-    issue_s(0, 0);
-    issue_s(1, 0);
-  }
+  bool ok = mbar_wait(&sm.q_full, 0, ab, lim, SITE_FWD_MMA);
   for (int j = 0; ok && j < n; ++j) {
     const int st = j % kFwdStages;
-    if (j + 1 < n) {
-      const int st1 = (j + 1) % kFwdStages;
-      ok = mbar_wait(&sm.kv_full[st1], ((j + 1) / kFwdStages) & 1, ab, lim, SITE_FWD_MMA);
-      for (int X = 0; ok && X < 2; ++X) {
-        ok = mbar_wait(&sm.s_free[X], j & 1, ab, lim, SITE_FWD_MMA);
-        if (ok) {
-          tc_fence_after();
-          issue_s(X, st1);
-        }
-      }
-      if (!ok) break;
+    ok = mbar_wait(&sm.kv_full[st], (j / kFwdStages) & 1, ab, lim, SITE_FWD_MMA);
+    for (int X = 0; ok && X < 2; ++X) {
+      if (j > 0 && !(ok = mbar_wait(&sm.s_free[X], (j - 1) & 1, ab, lim, SITE_FWD_MMA))) break;
+      tc_fence_after();
+      const uint32_t d = tmem + kColS + X * 128;
+      const uint64_t a = make_sdesc(smem_u32(sm.qc[X]), 16, 512, kLayoutSW64);
+      const uint64_t b = make_sdesc(smem_u32(sm.kc[st]), 16, 512, kLayoutSW64);
+      umma_ss(d, a, b, kIdescS, 0u);
+      umma_ss(d, a + 2, b + 2, kIdescS, 1u);  // channels 16..31: start address + 32 B
+      if (pos)
+        umma_ss(d, make_sdesc(smem_u32(sm.qp[X]), 16, 256, kLayoutSW32),
+                make_sdesc(smem_u32(sm.kp[st]), 16, 256, kLayoutSW32), kIdescS, 1u);
+      umma_commit(&sm.s_full[X]);
     }
+  }
+  // Every MMA issued above must finish before the tensor memory is freed.
+  umma_commit(&sm.drain);
+  volatile int no_abort = 0;
+  mbar_wait(&sm.drain, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
+}
+
+// Warp 10: [O|L]_X += P_X(j) [V_j | 1] once group X has written P_X(j), then
+// releases the K/V stage of tile j.
+__device__ __forceinline__ void fwd_mma_pv(FwdSmem& sm, uint32_t tmem, const FwdParams& p) {
+  volatile int* ab = &sm.abort_flag;
+  const uint64_t lim = p.wait_limit_ns;
+  const int n = p.n_tiles;
+  bool ok = true;
+  for (int j = 0; ok && j < n; ++j) {
+    const int st = j % kFwdStages;
     const uint32_t vaddr = smem_u32(sm.v[st]);
     // B = [V | ones]: two MN-major 64B-swizzle atoms, the second LBO bytes on
     const uint32_t lbo = smem_u32(sm.ones) - vaddr;
     for (int X = 0; ok && X < 2; ++X) {
-      ok = mbar_wait(&sm.p_full[X], j & 1, ab, lim, SITE_FWD_MMA);
-      if (!ok) break;
+      // p_full_X(j) implies K/V stage st has landed: S_X(j) was computed from it
+      if (!(ok = mbar_wait(&sm.p_full[X], j & 1, ab, lim, SITE_FWD_MMA))) break;
       tc_fence_after();
       const uint32_t d = tmem + kColO + X * kOCols;
       const uint32_t a = tmem + kColP + X * 64;
@@ -184,7 +191,6 @@ __device__ __forceinline__ void fwd_mma(FwdSmem& sm, uint32_t tmem, const FwdPar
     }
     if (ok) umma_commit(&sm.kv_empty[st]);
   }
-  // Every MMA issued above must finish before the tensor memory is freed.
   umma_commit(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&sm.p_full[X], 4);
       mbar_init(&sm.pv_done[X], 1);
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -364,8 +370,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_softmax(sm, tmem, p, u, tile0, warp >> 2, warp & 3);
   } else if (warp == 8) {
     if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p, u, tile0);
+  } else if (warp == 9) {
+    if (lane == 0) fwd_mma_scores(sm, tmem, p);
   } else {
-    if (lane == 0) fwd_mma(sm, tmem, p);
+    if (lane == 0) fwd_mma_pv(sm, tmem, p);
   }
   tc_fence_before();
   __syncthreads();

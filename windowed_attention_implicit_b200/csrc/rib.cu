@@ -614,6 +614,17 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
   p.wait_limit_ns = g_wait_limit_ns;
   if ((rc = set_smem(attn_bwd_kernel, kBwdSmemBytes))) return rc;
   {
+    // The kernel moves registers between warpgroups with setmaxnreg; that is
+    // only safe if the compiled launch budget is the one the split assumes.
+    static int launch_regs = -1;
+    if (launch_regs < 0) {
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, attn_bwd_kernel) != cudaSuccess) return RIB_ERR_CUDA;
+      launch_regs = fa.numRegs;
+    }
+    if (launch_regs != kBwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
+  }
+  {
     TraceScope ts(K_BWD, st);
     attn_bwd_kernel<<<dim3(g.n_tiles, g.units), kBwdThreads, kBwdSmemBytes, st>>>(
         tq, tdo, tqp, tkp, tl, td, p);
