@@ -12,14 +12,21 @@
 // content tiles and one over the positional tiles, accumulating into the
 // same TMEM score tile.
 //
-// CTA = one unit (batch, window, head) x two 128-query tiles (A, B), 320
-// threads:
-//   warps 0-3  softmax group A (thread = query row = TMEM lane)
-//   warps 4-7  softmax group B
-//   warp  8    TMA producer: Q tiles once, then K/V/Kp tiles through a
-//              3-stage shared-memory ring; boxes at rolled map coordinates
-//   warp  9    TMEM allocator; issues the score MMAs S_X(j) = Q_X K_j^T
-//   warp 10    issues the PV MMAs and releases K/V stages
+// CTA = one unit (batch, window, head) x two 128-query tiles (A, B), 640
+// threads (5 warpgroups):
+//   warps 0-7    softmax group A: warp w owns TMEM lanes 32(w%4).. (query
+//                rows) and key columns 64((w/4)%2).. of each score tile; the
+//                two warps sharing a row exchange partial row maxima
+//   warps 8-15   softmax group B, the same for the second query tile
+//   warp  16     TMA producer: Q tiles once, then K/V/Kp tiles through a
+//                3-stage shared-memory ring; boxes at rolled map coordinates
+//   warp  17     TMEM allocator; issues the score MMAs S_X(j) = Q_X K_j^T
+//   warp  18     issues the PV MMAs and releases K/V stages
+//   warp  19     idle
+// Four softmax warps per SM sub-partition hide the latency of the
+// exponential chains (with one row per thread there were only two); the
+// softmax warpgroups take 104 registers and the service warpgroup 64
+// (setmaxnreg).
 // A tcgen05.commit blocks its issuing thread until the thread's MMAs have
 // completed (~270 cycles), so scores and PV are issued by two threads: one
 // thread's commit never leaves the tensor pipe idle.
@@ -46,7 +53,12 @@
 namespace rib {
 
 constexpr int kFwdStages = 3;
-constexpr int kFwdThreads = 352;
+constexpr int kFwdThreads = 640;
+constexpr int kFwdLaunchRegs = 96;      // what the host checks ptxas gave (65536 / 640)
+constexpr int kFwdSoftmaxRegs = 104;    // warpgroups 0-3
+constexpr int kFwdServiceRegs = 64;     // warpgroup 4
+static_assert(4 * 128 * kFwdSoftmaxRegs + 128 * kFwdServiceRegs <= kFwdThreads * kFwdLaunchRegs,
+              "register split exceeds the launch budget");
 constexpr uint32_t kFwdTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // O_X at kColO + 48 X, L at +32
 constexpr int kOCols = 48;
@@ -77,7 +89,9 @@ struct __align__(1024) FwdSmem {
   uint64_t kv_full[kFwdStages];
   uint64_t kv_empty[kFwdStages];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t pair_bar[2][4];        // the two warps sharing 32 rows of a tile
   uint64_t drain;
+  float red_max[2][2][2][128];    // [tile parity][group][column half][row] partial maxima
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -197,13 +211,14 @@ __device__ __forceinline__ void fwd_mma_pv(FwdSmem& sm, uint32_t tmem, const Fwd
 }
 
 __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
-                                            const UnitCoord& u, int tile0, int X, int wq) {
+                                            const UnitCoord& u, int tile0, int X, int h, int wq) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int lane = threadIdx.x & 31;
+  const int row = wq * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-  const uint32_t tS = tmem + lane_off + kColS + X * 128;
-  const uint32_t tP = tmem + lane_off + kColP + X * 64;
+  const uint32_t tS = tmem + lane_off + kColS + X * 128 + 64 * h;
+  const uint32_t tP = tmem + lane_off + kColP + X * 64 + 32 * h;
   const uint32_t tO = tmem + lane_off + kColO + X * kOCols;
   const float sl = p.scale_log2;
   const uint64_t sl2 = pk2(sl, sl);
@@ -213,27 +228,30 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   for (int j = 0; j < n; ++j) {
     if (!(ok = warp_wait(&sm.s_full[X], j & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
     tc_fence_after();
-    uint32_t s[4][32];
+    uint32_t s[2][32];
     tmem_ld_x32(tS, s[0]);
     tmem_ld_x32(tS + 32, s[1]);
-    tmem_ld_x32(tS + 64, s[2]);
-    tmem_ld_x32(tS + 96, s[3]);
     tmem_wait_ld();
     reg_fence_x32(s[0]);
     reg_fence_x32(s[1]);
-    reg_fence_x32(s[2]);
-    reg_fence_x32(s[3]);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.s_free[X]);
 
+    // row maximum: this warp's 64 columns, then the partner warp's
     float mx = __uint_as_float(s[0][0]);
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
       for (int e = (c == 0 ? 1 : 0); e + 1 < 32; e += 2)
         mx = fmax3(mx, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-    mx = fmaxf(mx, __uint_as_float(s[3][31]));
+    mx = fmaxf(mx, __uint_as_float(s[1][31]));
+    sm.red_max[j & 1][X][h][row] = mx;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.pair_bar[X][wq]);
+    if (!(ok = warp_wait(&sm.pair_bar[X][wq], j & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
+    mx = fmaxf(mx, sm.red_max[j & 1][X][h ^ 1][row]);
+
     const float m_tile = mx * sl;
     float m_new = m_run, alpha = 1.f;
     bool resc = false;
@@ -251,7 +269,7 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     }
     const uint64_t neg2 = pk2(-m_new, -m_new);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -270,7 +288,9 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
       }
       tmem_st_x16(tP + c * 16, pk);
     }
-    if (j > 0 && __any_sync(0xffffffffu, resc)) {
+    // the column-half-0 warp of each row pair rescales [O|L] (both halves
+    // took the same decision from the same row maximum)
+    if (h == 0 && j > 0 && __any_sync(0xffffffffu, resc)) {
       uint32_t o[32], l[16];
       tmem_ld_x32(tO, o);
       tmem_ld_x16(tO + 32, l);
@@ -290,7 +310,7 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     if (lane == 0) mbar_arrive(&sm.p_full[X]);
     m_run = m_new;
   }
-  if (!ok) return;
+  if (!ok || h != 0) return;
   if (!warp_wait(&sm.pv_done[X], (n - 1) & 1, ab, lim, SITE_FWD_SOFTMAX)) return;
   tc_fence_after();
   uint32_t o[32], l[16];
@@ -307,7 +327,7 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
   int i0, j0, i, jl;
   tile_origin(tile0 + X, p.tiles_x, i0, j0);
-  tile_row_local(wq * 32 + lane, i0, j0, i, jl);
+  tile_row_local(row, i0, j0, i, jl);
   const int y = wrap_once(u.wy * p.M + i + p.s, p.H);
   const int x = wrap_once(u.wx * p.M + jl + p.s, p.W);
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
@@ -336,9 +356,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int X = 0; X < 2; ++X) {
       mbar_init(&sm.s_full[X], 1);
-      mbar_init(&sm.s_free[X], 4);
-      mbar_init(&sm.p_full[X], 4);
+      mbar_init(&sm.s_free[X], 8);
+      mbar_init(&sm.p_full[X], 8);
       mbar_init(&sm.pv_done[X], 1);
+      for (int q = 0; q < 4; ++q) mbar_init(&sm.pair_bar[X][q], 2);
     }
     mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
     sm.abort_flag = 0;
@@ -351,14 +372,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_proxy_async_smem();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 16 && lane == 0) {
     tma_prefetch_desc(&tm_qkv);
     if (p.rank > 0) {
       tma_prefetch_desc(&tm_qp);
       tma_prefetch_desc(&tm_kp);
     }
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(&sm.tmem_base, kFwdTmemCols);
     tmem_relinquish();
   }
@@ -366,18 +387,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp < 8) {
-    fwd_softmax(sm, tmem, p, u, tile0, warp >> 2, warp & 3);
-  } else if (warp == 8) {
-    if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p, u, tile0);
-  } else if (warp == 9) {
-    if (lane == 0) fwd_mma_scores(sm, tmem, p);
+  if (warp < 16) {
+    regs_inc<kFwdSoftmaxRegs>();
+    fwd_softmax(sm, tmem, p, u, tile0, warp >> 3, (warp >> 2) & 1, warp & 3);
   } else {
-    if (lane == 0) fwd_mma_pv(sm, tmem, p);
+    regs_dec<kFwdServiceRegs>();
+    if (warp == 16) {
+      if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p, u, tile0);
+    } else if (warp == 17) {
+      if (lane == 0) fwd_mma_scores(sm, tmem, p);
+    } else if (warp == 18) {
+      if (lane == 0) fwd_mma_pv(sm, tmem, p);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, kFwdTmemCols);
   }

@@ -84,6 +84,28 @@ __device__ __forceinline__ float gelu_erf_grad(float a) {
   return cdf + a * pdf;
 }
 
+// sum_k a[k*sa] * b[k*sb] for k < n with four independent accumulators
+// combined in a fixed order (latency of one FMA chain hidden, result
+// deterministic).  `ldg` reads `a` through the read-only cache.
+template <bool kLdgA>
+__device__ __forceinline__ float dot4(const float* a, int sa, const float* b, int sb, int n,
+                                      float init) {
+  float c0 = init, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+  int k = 0;
+  for (; k + 3 < n; k += 4) {
+    const float a0 = kLdgA ? __ldg(a + (k + 0) * sa) : a[(k + 0) * sa];
+    const float a1 = kLdgA ? __ldg(a + (k + 1) * sa) : a[(k + 1) * sa];
+    const float a2 = kLdgA ? __ldg(a + (k + 2) * sa) : a[(k + 2) * sa];
+    const float a3 = kLdgA ? __ldg(a + (k + 3) * sa) : a[(k + 3) * sa];
+    c0 = fmaf(a0, b[(k + 0) * sb], c0);
+    c1 = fmaf(a1, b[(k + 1) * sb], c1);
+    c2 = fmaf(a2, b[(k + 2) * sb], c2);
+    c3 = fmaf(a3, b[(k + 3) * sb], c3);
+  }
+  for (; k < n; ++k) c0 = fmaf(kLdgA ? __ldg(a + k * sa) : a[k * sa], b[k * sb], c0);
+  return (c0 + c1) + (c2 + c3);
+}
+
 __host__ __device__ constexpr size_t pos_fwd_smem_floats(int F, int hid) {
   return static_cast<size_t>(kPosTok) * (pad1(4 * F) + pad1(hid));
 }
@@ -108,9 +130,7 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   const float* b1 = p.b1[side];
   const float* gr = g + t * ldg;
   for (int jh = q; jh < p.hid; jh += nq) {
-    const float* wr = w1 + static_cast<size_t>(jh) * din;
-    float acc = __ldg(b1 + jh);
-    for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
+    const float acc = dot4<true>(w1 + static_cast<size_t>(jh) * din, 1, gr, 1, din, __ldg(b1 + jh));
     h[t * ldh + jh] = gelu_erf(acc);
   }
   __syncthreads();
@@ -120,9 +140,7 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   const float* b2 = p.b2[side];
   const float* hr = h + t * ldh;
   for (int o = q; o < p.dout; o += nq) {
-    const float* wr = w2 + static_cast<size_t>(o) * p.hid;
-    float acc = __ldg(b2 + o);
-    for (int k = 0; k < p.hid; ++k) acc = fmaf(__ldg(wr + k), hr[k], acc);
+    const float acc = dot4<true>(w2 + static_cast<size_t>(o) * p.hid, 1, hr, 1, p.hid, __ldg(b2 + o));
     const int head = o / p.rank, r = o - head * p.rank;
     const size_t off = (static_cast<size_t>(head) * p.N + tok) * p.rank + r;
     p.out32[side][off] = acc;
@@ -161,11 +179,8 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
     const float* gr = g + t * ldg;
     const float* gor = go + t * ldo;
     for (int jh = q; jh < hid; jh += nq) {
-      const float* wr = w1 + static_cast<size_t>(jh) * din;
-      float acc = __ldg(b1 + jh);
-      for (int k = 0; k < din; ++k) acc = fmaf(__ldg(wr + k), gr[k], acc);
-      float dh = 0.f;
-      for (int o = 0; o < dout; ++o) dh = fmaf(__ldg(w2 + static_cast<size_t>(o) * hid + jh), gor[o], dh);
+      const float acc = dot4<true>(w1 + static_cast<size_t>(jh) * din, 1, gr, 1, din, __ldg(b1 + jh));
+      const float dh = dot4<true>(w2 + jh, hid, gor, 1, dout, 0.f);
       h[t * ldh + jh] = gelu_erf(acc);
       da[t * ldh + jh] = dh * gelu_erf_grad(acc);  // tokens past N have go == 0
     }
@@ -175,9 +190,7 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
   // dw1[jh][k] = sum_t da[t][jh] g[t][k]  (warp: one jh, consecutive k)
   for (int idx = threadIdx.x; idx < hid * din; idx += blockDim.x) {
     const int jh = idx / din, k = idx - jh * din;
-    float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc = fmaf(da[t * ldh + jh], g[t * ldg + k], acc);
-    out[idx] = acc;
+    out[idx] = dot4<false>(da + jh, ldh, g + k, ldg, T, 0.f);
   }
   for (int jh = threadIdx.x; jh < hid; jh += blockDim.x) {
     float acc = 0.f;
@@ -188,9 +201,7 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
   // dw2[o][jh] = sum_t go[t][o] h[t][jh]  (warp: one o, consecutive jh)
   for (int idx = threadIdx.x; idx < dout * hid; idx += blockDim.x) {
     const int o = idx / hid, jh = idx - o * hid;
-    float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc = fmaf(go[t * ldo + o], h[t * ldh + jh], acc);
-    o2[idx] = acc;
+    o2[idx] = dot4<false>(go + o, ldo, h + jh, ldh, T, 0.f);
   }
   for (int o = threadIdx.x; o < dout; o += blockDim.x) {
     float acc = 0.f;

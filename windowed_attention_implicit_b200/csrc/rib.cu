@@ -521,6 +521,16 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads, int hea
   p.lse = lse;
   p.wait_limit_ns = g_wait_limit_ns;
   if ((rc = set_smem(attn_fwd_kernel, kFwdSmemBytes))) return rc;
+  {
+    // setmaxnreg split: only safe with the launch budget it was sized for
+    static int launch_regs = -1;
+    if (launch_regs < 0) {
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel) != cudaSuccess) return RIB_ERR_CUDA;
+      launch_regs = fa.numRegs;
+    }
+    if (launch_regs != kFwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
+  }
   dim3 grid(g.n_tiles / 2, g.units);
   TraceScope ts(K_FWD, static_cast<cudaStream_t>(stream));
   attn_fwd_kernel<<<grid, kFwdThreads, kFwdSmemBytes, static_cast<cudaStream_t>(stream)>>>(
