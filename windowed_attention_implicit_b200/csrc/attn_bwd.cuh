@@ -105,6 +105,7 @@ struct __align__(1024) BwdSmem {
   uint64_t k_full;
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
   uint64_t s_full, s_free, ds_full, pt_free /* P^T and dS^T in TMEM */, ds_free[2];
+  uint64_t dsq_full[2];            // dS buffer b written (for the dQ issuer)
   uint64_t dq_full, dq_free, mma_done;
   int drain_ok[4];
   uint64_t drain;
@@ -177,7 +178,8 @@ __device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
   }
 }
 
-// Warp 9: S^T = K_aug Q_aug^T and dP^T = V dO^T of every query tile, each
+// Warp 13 (all lanes; one elected lane issues): S^T = K_aug Q_aug^T and
+// dP^T = V dO^T of every query tile, each
 // issued as soon as the compute warps have pulled the previous one into
 // registers.
 __device__ __forceinline__ void bwd_mma_scores(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
@@ -186,78 +188,87 @@ __device__ __forceinline__ void bwd_mma_scores(BwdSmem& sm, uint32_t tmem, const
   const bool pos = p.rank > 0;
   const int n = p.n_tiles;
   const uint32_t kc = smem_u32(sm.kc), kp = smem_u32(sm.kp), v = smem_u32(sm.v);
-  bool ok = mbar_wait(&sm.k_full, 0, ab, lim, SITE_BWD_MMA);
+  bool ok = warp_wait(&sm.k_full, 0, ab, lim, SITE_BWD_MMA);
   for (int i = 0; ok && i < n; ++i) {
     const int st = i % kBwdStages;
-    ok = mbar_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_MMA) &&
-         (i == 0 || mbar_wait(&sm.s_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA));
+    ok = warp_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_MMA) &&
+         (i == 0 || warp_wait(&sm.s_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA));
     if (!ok) break;
     tc_fence_after();
     // S^T = K_aug Q_aug^T  (M = keys, N = queries, K = 32 + 16)
     const uint64_t a = make_sdesc(kc, 16, 512, kLayoutSW64);
     const uint64_t b = make_sdesc(smem_u32(sm.qc[st]), 16, 512, kLayoutSW64);
-    umma_ss(tmem + kBColS, a, b, kIdescBS, 0u);
-    umma_ss(tmem + kBColS, a + 2, b + 2, kIdescBS, 1u);
+    umma_ss_elect(tmem + kBColS, a, b, kIdescBS, 0u);
+    umma_ss_elect(tmem + kBColS, a + 2, b + 2, kIdescBS, 1u);
     if (pos)
-      umma_ss(tmem + kBColS, make_sdesc(kp, 16, 512, kLayoutSW64),
+      umma_ss_elect(tmem + kBColS, make_sdesc(kp, 16, 512, kLayoutSW64),
               make_sdesc(smem_u32(sm.qp[st]), 16, 512, kLayoutSW64), kIdescBS, 1u);
     // dP^T = V dO^T  (M = keys, N = queries, K = 32)
     const uint64_t av = make_sdesc(v, 16, 512, kLayoutSW64);
     const uint64_t bo = make_sdesc(smem_u32(sm.dO[st]), 16, 512, kLayoutSW64);
-    umma_ss(tmem + kBColDP, av, bo, kIdescBS, 0u);
-    umma_ss(tmem + kBColDP, av + 2, bo + 2, kIdescBS, 1u);
-    umma_commit(&sm.s_full);
+    umma_ss_elect(tmem + kBColDP, av, bo, kIdescBS, 0u);
+    umma_ss_elect(tmem + kBColDP, av + 2, bo + 2, kIdescBS, 1u);
+    umma_commit_elect(&sm.s_full);
   }
-  umma_commit(&sm.drain);
+  umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
 }
 
-// Warp 10: dV += P^T dO, dK_aug += dS^T [Qc|Qp] (A from TMEM) and
-// dQ_aug = dS [Kc|Kp] (A from shared memory) of every query tile.
+// Warp 14 (all lanes; one elected lane issues): dV += P^T dO and
+// dK_aug += dS^T [Qc|Qp] (A from TMEM) of every query tile.
 __device__ __forceinline__ void bwd_mma_grads(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int n = p.n_tiles;
-  const uint32_t kc = smem_u32(sm.kc), kp = smem_u32(sm.kp);
   const uint32_t lbo_q = smem_u32(sm.qp[0]) - smem_u32(sm.qc[0]);   // [Qc|Qp] atoms
-  const uint32_t lbo_k = kp - kc;                                   // [Kc|Kp] atoms
   bool ok = true;
   for (int i = 0; ok && i < n; ++i) {
     const int st = i % kBwdStages;
     // ds_full(i) implies the stage's tiles have landed: the compute warps
     // waited for them (q_full) before forming P^T and dS^T.
-    if (!(ok = mbar_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
+    if (!(ok = warp_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
     tc_fence_after();
     const uint32_t qc = smem_u32(sm.qc[st]), dO = smem_u32(sm.dO[st]);
-    const uint32_t ds = smem_u32(sm.ds[i & 1]);
     // dV += P^T dO   (K = queries, 16 per step; A from TMEM)
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      umma_ts(tmem + kBColDV, tmem + kBColP + k * 8,
-              make_sdesc(dO + k * 1024, 16, 512, kLayoutSW64), kIdescBV,
-              (i > 0 || k > 0) ? 1u : 0u);
+    umma_ts8_elect(tmem + kBColDV, tmem + kBColP, make_sdesc(dO, 16, 512, kLayoutSW64),
+                   1024 >> 4, kIdescBV, i > 0 ? 1u : 0u);
     // dK_aug += dS^T [Qc|Qp]   (A = dS^T from TMEM)
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      umma_ts(tmem + kBColDK, tmem + kBColDST + k * 8,
-              make_sdesc(qc + k * 1024, lbo_q, 512, kLayoutSW64), kIdescBK,
-              (i > 0 || k > 0) ? 1u : 0u);
-    umma_commit(&sm.pt_free);
-    // dQ_aug = dS [Kc|Kp]   (A = dS MN-major core matrices); the single dQ
-    // buffer is free once the compute warps drained tile i-1
-    if (i > 0 && !(ok = mbar_wait(&sm.dq_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA))) break;
-    tc_fence_after();
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      umma_ss(tmem + kBColDQ, make_sdesc(ds + k * 256, 128, 2048, kLayoutNone),
-              make_sdesc(kc + k * 1024, lbo_k, 512, kLayoutSW64), kIdescBQ, k > 0 ? 1u : 0u);
-    umma_commit(&sm.ds_free[i & 1]);
-    umma_commit(&sm.dq_full);
-    umma_commit(&sm.q_empty[st]);
+    umma_ts8_elect(tmem + kBColDK, tmem + kBColDST, make_sdesc(qc, lbo_q, 512, kLayoutSW64),
+                   1024 >> 4, kIdescBK, i > 0 ? 1u : 0u);
+    umma_commit_elect(&sm.pt_free);
+    umma_commit_elect(&sm.q_empty[st]);
   }
-  umma_commit(&sm.mma_done);   // every gradient MMA of the kernel has completed
-  umma_commit(&sm.drain);
+  umma_commit_elect(&sm.mma_done);   // every dV / dK MMA of the kernel has completed
+  umma_commit_elect(&sm.drain);
+  volatile int no_abort = 0;
+  mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
+}
+
+// Warp 15 (all lanes; one elected lane issues): dQ_aug = dS [Kc|Kp] (A = dS
+// MN-major core matrices in shared memory) of every query tile.  dS buffer
+// b has its own barrier, so this issuer's parity waits stay exact even when
+// the compute warps run a tile ahead of it.
+__device__ __forceinline__ void bwd_mma_dq(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
+  volatile int* ab = &sm.abort_flag;
+  const uint64_t lim = p.wait_limit_ns;
+  const int n = p.n_tiles;
+  const uint32_t kc = smem_u32(sm.kc), kp = smem_u32(sm.kp);
+  const uint32_t lbo_k = kp - kc;  // [Kc|Kp] atoms
+  bool ok = true;
+  for (int i = 0; ok && i < n; ++i) {
+    if (!(ok = warp_wait(&sm.dsq_full[i & 1], (i >> 1) & 1, ab, lim, SITE_BWD_MMA))) break;
+    // the single dQ buffer is free once the drain warps pulled tile i-1
+    if (i > 0 && !(ok = warp_wait(&sm.dq_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA))) break;
+    tc_fence_after();
+    const uint32_t ds = smem_u32(sm.ds[i & 1]);
+    // step k: 16 queries further in dS (256 B), 16 keys further in [Kc|Kp] (1 KB)
+    umma_ss8_elect(tmem + kBColDQ, make_sdesc(ds, 128, 2048, kLayoutNone), 256 >> 4,
+                   make_sdesc(kc, lbo_k, 512, kLayoutSW64), 1024 >> 4, kIdescBQ, 0u);
+    umma_commit_elect(&sm.ds_free[i & 1]);
+    umma_commit_elect(&sm.dq_full);
+  }
+  umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
 }
@@ -403,7 +414,10 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.ds_full);
+    if (lane == 0) {
+      mbar_arrive(&sm.ds_full);
+      mbar_arrive(&sm.dsq_full[i & 1]);
+    }
   }
   if (!ok) return;
   if (!warp_wait(&sm.mma_done, 0, ab, lim, SITE_BWD_COMPUTE)) return;
@@ -484,10 +498,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.pt_free, 1);
     mbar_init(&sm.ds_free[0], 1);
     mbar_init(&sm.ds_free[1], 1);
+    mbar_init(&sm.dsq_full[0], 8);
+    mbar_init(&sm.dsq_full[1], 8);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_free, 4);
     mbar_init(&sm.mma_done, 1);
-    mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
+    mbar_init(&sm.drain, 3);   // one commit from each MMA-issuing warp
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -515,9 +531,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     } else if (warp == 12) {
       if (lane == 0) bwd_producer(sm, &tm_qkv, &tm_dout, &tm_qp, &tm_kp, &tm_lse2, &tm_dd, p, u, kt);
     } else if (warp == 13) {
-      if (lane == 0) bwd_mma_scores(sm, tmem, p);
+      bwd_mma_scores(sm, tmem, p);
     } else if (warp == 14) {
-      if (lane == 0) bwd_mma_grads(sm, tmem, p);
+      bwd_mma_grads(sm, tmem, p);
+    } else {
+      bwd_mma_dq(sm, tmem, p);
     }
   }
   tc_fence_before();

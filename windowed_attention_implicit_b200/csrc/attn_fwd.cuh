@@ -20,26 +20,31 @@
 //   warps 8-15   softmax group B, the same for the second query tile
 //   warp  16     TMA producer: Q tiles once, then K/V/Kp tiles through a
 //                3-stage shared-memory ring; boxes at rolled map coordinates
-//   warp  17     TMEM allocator; issues the score MMAs S_X(j) = Q_X K_j^T
-//   warp  18     issues the PV MMAs and releases K/V stages
-//   warp  19     idle
+//   warp  17     TMEM allocator; issues the score MMAs
+//   warp  18     issues the PV MMAs of query tile A
+//   warp  19     issues the PV MMAs of query tile B
 // Four softmax warps per SM sub-partition hide the latency of the
-// exponential chains (with one row per thread there were only two); the
-// softmax warpgroups take 104 registers and the service warpgroup 64
-// (setmaxnreg).
-// A tcgen05.commit blocks its issuing thread until the thread's MMAs have
-// completed (~270 cycles), so scores and PV are issued by two threads: one
-// thread's commit never leaves the tensor pipe idle.
-// TMEM (512 columns): S_A, S_B fp32 [128 x 128]; P_A, P_B bf16 [128 x 128]
-// (64 packed columns each); [O|L]_A, [O|L]_B fp32 [128 x 48].
-// Per key tile j and group X: S_X(j) = Q_X K_j^T (MMA) -> online softmax in
-// registers -> P_X(j) to TMEM -> [O|L]_X += P_X(j) [V_j | 1] (MMA, A from
-// TMEM): the second swizzle atom of the B operand is an all-ones tile, so the
-// tensor core also accumulates the softmax denominators L from the very bf16
-// P it multiplies with V.  S_X(j+1) is issued as soon as group X has pulled
-// S_X(j) into registers, so score MMAs overlap the exponentials.  The
-// running max is updated lazily: O and L are rescaled only when the max
-// grows by more than 2^8.
+// exponential chains; the softmax warpgroups take 104 registers and the
+// service warpgroup 64 (setmaxnreg).
+//
+// One thread issues at most one tcgen05.mma every ~90 cycles, whatever its
+// shape, while the tensor pipe retires an M=128, N=48, K=16 MMA in ~24
+// cycles; so the MMAs of a key tile (3 score MMAs per query tile, 8 PV MMAs
+// per query tile) are spread over three issuing threads.
+//
+// TMEM (512 columns): three score regions R0..R2 of 128 fp32 columns, then
+// [O|L]_A and [O|L]_B (48 columns each).  Score tiles are numbered
+// k = 2j + X (key tile j, query tile X) and S(k) goes to region k % 3.
+// Softmax group X pulls S(k) into registers, writes P(k) as packed bf16 over
+// the first 64 columns of the same region, and signals p_full; the PV thread
+// of X then issues [O|L]_X += P(k) [V_j | 1] with P read from TMEM as the A
+// operand (the second swizzle atom of the B operand is an all-ones tile, so
+// the tensor core also accumulates the softmax denominators L from the very
+// bf16 P it multiplies with V) and frees the region.  The score MMA of
+// k + 3 reuses the region once that PV has completed.  The softmax warps
+// therefore never wait for a PV MMA, except before the rare rescale of O:
+// the running max is updated lazily, O and L being rescaled only when the
+// max grows by more than 2^8.
 //
 // The exponentials are the bottleneck of this kernel (16K per 128x128 tile
 // against 320 tensor-core cycles of MMA at d_qk=48, d_v=32), so a fixed
@@ -60,14 +65,20 @@ constexpr int kFwdServiceRegs = 64;     // warpgroup 4
 static_assert(4 * 128 * kFwdSoftmaxRegs + 128 * kFwdServiceRegs <= kFwdThreads * kFwdLaunchRegs,
               "register split exceeds the launch budget");
 constexpr uint32_t kFwdTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // O_X at kColO + 48 X, L at +32
+constexpr int kRegions = 3;
+constexpr uint32_t kColO = 384;  // [O|L]_X at kColO + 48 X, L at +32
 constexpr int kOCols = 48;
+static_assert(kRegions * 128 + 2 * kOCols <= kFwdTmemCols, "forward TMEM layout exceeds 512 columns");
 // Of every 16 element pairs, how many exponentials run on the FMA pipe.
 #ifndef RIB_FWD_POLY_PAIRS
-#define RIB_FWD_POLY_PAIRS 6
+#define RIB_FWD_POLY_PAIRS 4
 #endif
 constexpr int kPolyPairs = RIB_FWD_POLY_PAIRS;
 constexpr uint64_t kFwdDrainNs = 200ull * 1000ull * 1000ull;
+#ifndef RIB_FWD_SLEEP_NS
+#define RIB_FWD_SLEEP_NS 20000
+#endif
+constexpr uint32_t kFwdSleepNs = RIB_FWD_SLEEP_NS;  // per retry of a waiting warp (0: poll)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct FwdParams {
@@ -87,8 +98,10 @@ struct __align__(1024) FwdSmem {
   uint8_t kp[kFwdStages][4096];
   uint64_t q_full;
   uint64_t kv_full[kFwdStages];
-  uint64_t kv_empty[kFwdStages];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t kv_empty[kFwdStages];  // both PV threads release a stage
+  uint64_t s_full[kRegions], r_free[kRegions];
+  uint64_t p_full[2][2];          // [tile X][key tile parity]
+  int pv_count[2];                // PV steps of tile X known complete
   uint64_t pair_bar[2][4];        // the two warps sharing 32 rows of a tile
   uint64_t drain;
   float red_max[2][2][2][128];    // [tile parity][group][column half][row] partial maxima
@@ -148,66 +161,101 @@ __device__ __forceinline__ void fwd_producer(FwdSmem& sm, const CUtensorMap* tq,
   }
 }
 
-// Warp 9: S_X(j) = Q_X K_j^T for both query tiles of every key tile, each as
-// soon as group X has pulled S_X(j-1) into registers.
+// Warp 17: S(k) = Q_X K_j^T into region k % 3 for k = 2j + X, in order,
+// each once the region has been freed by the PV MMA of score tile k - 3.
+// Phase arithmetic: a region's barriers complete once per use, and use
+// k + 3 cannot start before use k has been consumed, so no barrier is ever
+// more than one phase ahead of the parity a waiter asks for.
 __device__ __forceinline__ void fwd_mma_scores(FwdSmem& sm, uint32_t tmem, const FwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const bool pos = p.rank > 0;
-  const int n = p.n_tiles;
-  bool ok = mbar_wait(&sm.q_full, 0, ab, lim, SITE_FWD_MMA);
-  for (int j = 0; ok && j < n; ++j) {
-    const int st = j % kFwdStages;
-    ok = mbar_wait(&sm.kv_full[st], (j / kFwdStages) & 1, ab, lim, SITE_FWD_MMA);
-    for (int X = 0; ok && X < 2; ++X) {
-      if (j > 0 && !(ok = mbar_wait(&sm.s_free[X], (j - 1) & 1, ab, lim, SITE_FWD_MMA))) break;
-      tc_fence_after();
-      const uint32_t d = tmem + kColS + X * 128;
-      const uint64_t a = make_sdesc(smem_u32(sm.qc[X]), 16, 512, kLayoutSW64);
-      const uint64_t b = make_sdesc(smem_u32(sm.kc[st]), 16, 512, kLayoutSW64);
-      umma_ss(d, a, b, kIdescS, 0u);
-      umma_ss(d, a + 2, b + 2, kIdescS, 1u);  // channels 16..31: start address + 32 B
-      if (pos)
-        umma_ss(d, make_sdesc(smem_u32(sm.qp[X]), 16, 256, kLayoutSW32),
-                make_sdesc(smem_u32(sm.kp[st]), 16, 256, kLayoutSW32), kIdescS, 1u);
-      umma_commit(&sm.s_full[X]);
-    }
+  const int n = 2 * p.n_tiles;
+  bool ok = warp_wait(&sm.q_full, 0, ab, lim, SITE_FWD_MMA);
+  for (int k = 0; ok && k < n; ++k) {
+    const int X = k & 1, j = k >> 1, r = k % kRegions, st = j % kFwdStages;
+    if (X == 0 && !(ok = warp_wait(&sm.kv_full[st], (j / kFwdStages) & 1, ab, lim, SITE_FWD_MMA)))
+      break;
+    if (k >= kRegions &&
+        !(ok = warp_wait(&sm.r_free[r], (k / kRegions - 1) & 1, ab, lim, SITE_FWD_MMA)))
+      break;
+    tc_fence_after();
+    const uint32_t d = tmem + r * 128;
+    const uint64_t a = make_sdesc(smem_u32(sm.qc[X]), 16, 512, kLayoutSW64);
+    const uint64_t b = make_sdesc(smem_u32(sm.kc[st]), 16, 512, kLayoutSW64);
+    umma_ss_elect(d, a, b, kIdescS, 0u);
+    umma_ss_elect(d, a + 2, b + 2, kIdescS, 1u);  // channels 16..31: start address + 32 B
+    if (pos)
+      umma_ss_elect(d, make_sdesc(smem_u32(sm.qp[X]), 16, 256, kLayoutSW32),
+                    make_sdesc(smem_u32(sm.kp[st]), 16, 256, kLayoutSW32), kIdescS, 1u);
+    umma_commit_elect(&sm.s_full[r]);
   }
   // Every MMA issued above must finish before the tensor memory is freed.
-  umma_commit(&sm.drain);
+  umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
 }
 
-// Warp 10: [O|L]_X += P_X(j) [V_j | 1] once group X has written P_X(j), then
-// releases the K/V stage of tile j.
-__device__ __forceinline__ void fwd_mma_pv(FwdSmem& sm, uint32_t tmem, const FwdParams& p) {
+// Warps 18 (X = 0) and 19 (X = 1), all lanes, one elected lane issuing: [O|L]_X += P(k) [V_j | 1] for k = 2j + X
+// once group X has written P(k).  The commits free the region and release
+// K/V stage j (kv_empty counts one arrival per PV thread); the warp then
+// waits for its own MMAs (on the region's barrier) and publishes how many PV steps of tile X are
+// complete in pv_count[X], which the softmax warps read before touching
+// [O|L]_X (the rare rescale, and the epilogue).  The accumulation into
+// [O|L]_X is serial anyway, and the next P arrives much later, so the wait
+// costs this thread nothing.
+__device__ __forceinline__ void fwd_mma_pv(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
+                                           int X) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int n = p.n_tiles;
+  const uint32_t d = tmem + kColO + X * kOCols;
   bool ok = true;
   for (int j = 0; ok && j < n; ++j) {
-    const int st = j % kFwdStages;
+    const int k = 2 * j + X, r = k % kRegions, st = j % kFwdStages;
+    // p_full(k) implies K/V stage st has landed: S(k) was computed from it
+    if (!(ok = warp_wait(&sm.p_full[X][j & 1], (j >> 1) & 1, ab, lim, SITE_FWD_MMA))) break;
+    tc_fence_after();
     const uint32_t vaddr = smem_u32(sm.v[st]);
-    // B = [V | ones]: two MN-major 64B-swizzle atoms, the second LBO bytes on
+    // B = [V | ones]: two MN-major 64B-swizzle atoms, the second LBO bytes
+    // on; step k reads the next 16 keys (1 KB of V further)
     const uint32_t lbo = smem_u32(sm.ones) - vaddr;
-    for (int X = 0; ok && X < 2; ++X) {
-      // p_full_X(j) implies K/V stage st has landed: S_X(j) was computed from it
-      if (!(ok = mbar_wait(&sm.p_full[X], j & 1, ab, lim, SITE_FWD_MMA))) break;
-      tc_fence_after();
-      const uint32_t d = tmem + kColO + X * kOCols;
-      const uint32_t a = tmem + kColP + X * 64;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        umma_ts(d, a + k * 8, make_sdesc(vaddr + k * 1024, lbo, 512, kLayoutSW64), kIdescPV,
-                (j > 0 || k > 0) ? 1u : 0u);
-      umma_commit(&sm.pv_done[X]);
-    }
-    if (ok) umma_commit(&sm.kv_empty[st]);
+    umma_ts8_elect(d, tmem + r * 128, make_sdesc(vaddr, lbo, 512, kLayoutSW64), 1024 >> 4,
+                   kIdescPV, j > 0 ? 1u : 0u);
+    umma_commit_elect(&sm.r_free[r]);
+    umma_commit_elect(&sm.kv_empty[st]);
+    // r_free[r] is exact for this thread: its next phase needs S(k + 3),
+    // which needs this phase
+    if (!(ok = warp_wait(&sm.r_free[r], (k / kRegions) & 1, ab, lim, SITE_FWD_MMA))) break;
+    tc_fence_before();
+    if ((threadIdx.x & 31) == 0) st_release_shared(&sm.pv_count[X], j + 1);
   }
-  umma_commit(&sm.drain);
+  umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
+}
+
+// Waits (bounded) until pv_count[X] >= need, i.e. until the first `need`
+// PV steps of tile X have completed.  Warp-uniform.
+__device__ __forceinline__ bool wait_pv_count(FwdSmem& sm, int X, int need, const FwdParams& p) {
+  volatile int* ab = &sm.abort_flag;
+  bool ok = true;
+  if (ld_acquire_shared(&sm.pv_count[X]) < need) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_shared(&sm.pv_count[X]) < need) {
+      if (*ab) { ok = false; break; }
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        record_error(kErrTimeout, SITE_FWD_SOFTMAX);
+        *ab = 1;
+        ok = false;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) tc_fence_after();
+  return ok;
 }
 
 __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
@@ -216,17 +264,20 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   const uint64_t lim = p.wait_limit_ns;
   const int lane = threadIdx.x & 31;
   const int row = wq * 32 + lane;
-  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-  const uint32_t tS = tmem + lane_off + kColS + X * 128 + 64 * h;
-  const uint32_t tP = tmem + lane_off + kColP + X * 64 + 32 * h;
-  const uint32_t tO = tmem + lane_off + kColO + X * kOCols;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t tO = tl + kColO + X * kOCols;
   const float sl = p.scale_log2;
   const uint64_t sl2 = pk2(sl, sl);
   const int n = p.n_tiles;
   float m_run = 0.f;
   bool ok = true;
   for (int j = 0; j < n; ++j) {
-    if (!(ok = warp_wait(&sm.s_full[X], j & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
+    const int k = 2 * j + X, r = k % kRegions;
+    const uint32_t tS = tl + r * 128 + 64 * h;  // this warp's 64 score columns
+    const uint32_t tP = tl + r * 128 + 32 * h;  // its 64 bf16 P values, packed in pairs
+    if (!(ok = warp_wait(&sm.s_full[r], (k / kRegions) & 1, ab, lim, SITE_FWD_SOFTMAX,
+                         kFwdSleepNs)))
+      break;
     tc_fence_after();
     uint32_t s[2][32];
     tmem_ld_x32(tS, s[0]);
@@ -234,22 +285,29 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     tmem_wait_ld();
     reg_fence_x32(s[0]);
     reg_fence_x32(s[1]);
+
+    // row maximum: this warp's 64 columns, then the partner warp's.  The
+    // exchange also orders both warps' score loads before either overwrites
+    // the region with P.
+    // four independent chains of 16 keep the reduction's latency short
+    float m4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t* v = &s[q >> 1][(q & 1) * 16];
+      float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+      for (int e = 3; e + 1 < 16; e += 2)
+        m = fmax3(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+      m4[q] = fmaxf(m, __uint_as_float(v[15]));
+    }
+    float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+    sm.red_max[j & 1][X][h][row] = mx;
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.s_free[X]);
-
-    // row maximum: this warp's 64 columns, then the partner warp's
-    float mx = __uint_as_float(s[0][0]);
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int e = (c == 0 ? 1 : 0); e + 1 < 32; e += 2)
-        mx = fmax3(mx, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-    mx = fmaxf(mx, __uint_as_float(s[1][31]));
-    sm.red_max[j & 1][X][h][row] = mx;
-    __syncwarp();
     if (lane == 0) mbar_arrive(&sm.pair_bar[X][wq]);
-    if (!(ok = warp_wait(&sm.pair_bar[X][wq], j & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
+    if (!(ok = warp_wait(&sm.pair_bar[X][wq], j & 1, ab, lim, SITE_FWD_SOFTMAX, kFwdSleepNs)))
+      break;
+    tc_fence_after();
     mx = fmaxf(mx, sm.red_max[j & 1][X][h ^ 1][row]);
 
     const float m_tile = mx * sl;
@@ -261,11 +319,6 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
       m_new = m_tile;
       alpha = ex2_approx(m_run - m_tile);
       resc = true;
-    }
-    if (j > 0) {
-      // P_X and [O|L]_X are free once PV_X(j-1) has completed.
-      if (!(ok = warp_wait(&sm.pv_done[X], (j - 1) & 1, ab, lim, SITE_FWD_SOFTMAX))) break;
-      tc_fence_after();
     }
     const uint64_t neg2 = pk2(-m_new, -m_new);
 #pragma unroll
@@ -289,8 +342,10 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
       tmem_st_x16(tP + c * 16, pk);
     }
     // the column-half-0 warp of each row pair rescales [O|L] (both halves
-    // took the same decision from the same row maximum)
-    if (h == 0 && j > 0 && __any_sync(0xffffffffu, resc)) {
+    // took the same decision from the same row maximum), once every PV step
+    // accumulated so far has completed
+    if (h == 0 && __any_sync(0xffffffffu, resc)) {
+      if (!(ok = wait_pv_count(sm, X, j, p))) break;
       uint32_t o[32], l[16];
       tmem_ld_x32(tO, o);
       tmem_ld_x16(tO + 32, l);
@@ -307,12 +362,11 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.p_full[X]);
+    if (lane == 0) mbar_arrive(&sm.p_full[X][j & 1]);
     m_run = m_new;
   }
   if (!ok || h != 0) return;
-  if (!warp_wait(&sm.pv_done[X], (n - 1) & 1, ab, lim, SITE_FWD_SOFTMAX)) return;
-  tc_fence_after();
+  if (!wait_pv_count(sm, X, n, p)) return;
   uint32_t o[32], l[16];
   tmem_ld_x32(tO, o);
   tmem_ld_x16(tO + 32, l);
@@ -352,16 +406,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(&sm.q_full, 1);
     for (int st = 0; st < kFwdStages; ++st) {
       mbar_init(&sm.kv_full[st], 1);
-      mbar_init(&sm.kv_empty[st], 1);
+      mbar_init(&sm.kv_empty[st], 2);  // one commit from each PV thread
+    }
+    for (int r = 0; r < kRegions; ++r) {
+      mbar_init(&sm.s_full[r], 1);
+      mbar_init(&sm.r_free[r], 1);
     }
     for (int X = 0; X < 2; ++X) {
-      mbar_init(&sm.s_full[X], 1);
-      mbar_init(&sm.s_free[X], 8);
-      mbar_init(&sm.p_full[X], 8);
-      mbar_init(&sm.pv_done[X], 1);
+      mbar_init(&sm.p_full[X][0], 8);
+      mbar_init(&sm.p_full[X][1], 8);
+      sm.pv_count[X] = 0;
       for (int q = 0; q < 4; ++q) mbar_init(&sm.pair_bar[X][q], 2);
     }
-    mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
+    mbar_init(&sm.drain, 3);   // one commit from each MMA-issuing thread
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -395,9 +452,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (warp == 16) {
       if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p, u, tile0);
     } else if (warp == 17) {
-      if (lane == 0) fwd_mma_scores(sm, tmem, p);
-    } else if (warp == 18) {
-      if (lane == 0) fwd_mma_pv(sm, tmem, p);
+      fwd_mma_scores(sm, tmem, p);
+    } else {
+      fwd_mma_pv(sm, tmem, p, warp - 18);  // warps 18, 19
     }
   }
   tc_fence_before();

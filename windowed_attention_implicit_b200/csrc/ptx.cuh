@@ -71,6 +71,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but the thread may sleep in it for up to `hint_ns` until
+// the phase completes, instead of returning at once: waiting warps then give
+// their issue slots to the warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // when `abort` (a shared flag of the CTA) is set by another thread, or when
 // `limit_ns` elapses; in the latter case it records RIB_ERR_TIMEOUT with the
@@ -78,12 +94,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // The retry loop polls only the barrier: the abort flag and the (slow to
 // read) global timer are checked once every 64 tries, so a waiter resumes
 // within a few cycles of the phase completing.
+// With `sleep_ns` > 0 each retry may sleep that long (mbar_try_wait_sleep).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns, int site) {
+                                          uint64_t limit_ns, int site, uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity))
+      return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
@@ -93,6 +111,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
+}
+
+// Release store / acquire load of a shared-memory int (a flag or counter
+// that one thread publishes to the rest of the CTA).
+__device__ __forceinline__ void st_release_shared(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
 }
 
 // ---------------------------------------------------------------- TMA
@@ -216,6 +245,106 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same two MMAs issued by one elected lane of a converged warp.  The
+// whole warp executes the call with warp-uniform operands: issued this way a
+// thread sustains one MMA per ~43 cycles (M=128, N=48) against ~90 cycles
+// when a single lane issues from a divergent branch, where the operands are
+// not known to be uniform.
+__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Eight MMAs D (+)= A_k B_k^T, k = 0..7, issued by one elected lane of a
+// converged warp: A_k = tensor memory at a_tmem + 8k (16 bf16 columns per
+// step), B_k = b_desc advanced by k * b_step (descriptor units of 16 bytes).
+// `first_acc` = 0 makes the first MMA overwrite D.  One election and no
+// per-MMA descriptor arithmetic keep the issuing warp's instruction count
+// low while it shares its scheduler with busy warps.
+__device__ __forceinline__ void umma_ts8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t b_step, uint32_t idesc,
+                                               uint32_t first_acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
+      "add.s32 a, %1, 8;\n\t add.s64 b, %2, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "l"(static_cast<uint64_t>(b_step)), "r"(idesc), "r"(first_acc)
+      : "memory");
+}
+
+// The same with A from shared memory: A_k = a_desc + k * a_step.
+__device__ __forceinline__ void umma_ss8_elect(uint32_t d_tmem, uint64_t a_desc, uint32_t a_step,
+                                               uint64_t b_desc, uint32_t b_step, uint32_t idesc,
+                                               uint32_t first_acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b64 a, b, sa, sb;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "setp.eq.b32 t, %5, %5;\n\t"
+      "cvt.u64.u32 sa, %2;\n\t cvt.u64.u32 sb, %4;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %5, p;\n\t"
+      "add.s64 a, %1, sa;\n\t add.s64 b, %3, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t"
+      "add.s64 a, a, sa;\n\t add.s64 b, b, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t"
+      "add.s64 a, a, sa;\n\t add.s64 b, b, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t"
+      "add.s64 a, a, sa;\n\t add.s64 b, b, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t"
+      "add.s64 a, a, sa;\n\t add.s64 b, b, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t"
+      "add.s64 a, a, sa;\n\t add.s64 b, b, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t"
+      "add.s64 a, a, sa;\n\t add.s64 b, b, sb;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, t;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "r"(a_step), "l"(b_desc), "r"(b_step), "r"(idesc), "r"(first_acc)
+      : "memory");
+}
+
+// umma_commit from one elected lane of a converged warp (it then tracks the
+// MMAs that lane issued with the *_elect calls above).
+__device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
       : "memory");
 }
 
@@ -415,8 +544,8 @@ __device__ __forceinline__ T* align1024(uint8_t* p) {
 // Warp-uniform bounded wait: the warp proceeds only if every lane saw the
 // phase complete, so no warp-collective tcgen05 op runs on a partial warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit, int site) {
-  const bool ok = mbar_wait(bar, parity, abort, limit, site);
+                                          uint64_t limit, int site, uint32_t sleep_ns = 0) {
+  const bool ok = mbar_wait(bar, parity, abort, limit, site, sleep_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
