@@ -198,16 +198,12 @@ __device__ __forceinline__ void bwd_mma_scores(BwdSmem& sm, uint32_t tmem, const
     // S^T = K_aug Q_aug^T  (M = keys, N = queries, K = 32 + 16)
     const uint64_t a = make_sdesc(kc, 16, 512, kLayoutSW64);
     const uint64_t b = make_sdesc(smem_u32(sm.qc[st]), 16, 512, kLayoutSW64);
-    umma_ss_elect(tmem + kBColS, a, b, kIdescBS, 0u);
-    umma_ss_elect(tmem + kBColS, a + 2, b + 2, kIdescBS, 1u);
-    if (pos)
-      umma_ss_elect(tmem + kBColS, make_sdesc(kp, 16, 512, kLayoutSW64),
-              make_sdesc(smem_u32(sm.qp[st]), 16, 512, kLayoutSW64), kIdescBS, 1u);
+    umma_ss3_elect(tmem + kBColS, a, b, a + 2, b + 2, make_sdesc(kp, 16, 512, kLayoutSW64),
+                   make_sdesc(smem_u32(sm.qp[st]), 16, 512, kLayoutSW64), kIdescBS, pos ? 1u : 0u);
     // dP^T = V dO^T  (M = keys, N = queries, K = 32)
     const uint64_t av = make_sdesc(v, 16, 512, kLayoutSW64);
     const uint64_t bo = make_sdesc(smem_u32(sm.dO[st]), 16, 512, kLayoutSW64);
-    umma_ss_elect(tmem + kBColDP, av, bo, kIdescBS, 0u);
-    umma_ss_elect(tmem + kBColDP, av + 2, bo + 2, kIdescBS, 1u);
+    umma_ss3_elect(tmem + kBColDP, av, bo, av + 2, bo + 2, av, bo, kIdescBS, 0u);
     umma_commit_elect(&sm.s_full);
   }
   umma_commit_elect(&sm.drain);

@@ -337,6 +337,25 @@ __device__ __forceinline__ void umma_ss8_elect(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// The score chain of the augmented product, D = A0 B0^T + A1 B1^T + A2 B2^T
+// (two content K-steps, one positional), issued by one elected lane.  With
+// `three` = 0 only the first two MMAs are issued.
+__device__ __forceinline__ void umma_ss3_elect(uint32_t d_tmem, uint64_t a0, uint64_t b0,
+                                               uint64_t a1, uint64_t b1, uint64_t a2, uint64_t b2,
+                                               uint32_t idesc, uint32_t three) {
+  asm volatile(
+      "{\n\t.reg .pred f, t, e, q;\n\t"
+      "setp.ne.b32 f, %7, %7;\n\t"
+      "setp.eq.b32 t, %7, %7;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.and.b32 q, %8, 0, e;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %7, f;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %7, t;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %7, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "l"(a1), "l"(b1), "l"(a2), "l"(b2), "r"(idesc), "r"(three)
+      : "memory");
+}
+
 // umma_commit from one elected lane of a converged warp (it then tracks the
 // MMAs that lane issued with the *_elect calls above).
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
