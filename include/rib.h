@@ -170,6 +170,49 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads,
                         const void* qp_bf16, const void* kp_bf16, int rank,
                         float scale, void* out, float* lse, void* stream);
 
+/* ------------------------------------------------------------------------
+ * rib_cla_gate -- gating map of the convolutional local attention (CLA).
+ *
+ * English summary, Technical Summary §2.B (a lightweight path of a
+ * depth-wise convolution, a point-wise convolution and a sigmoid produces a
+ * gating map); Chinese summary §2.B (3x3 depth-wise, 1x1 point-wise):
+ *   y[b,i,j,c] = b_dw[c] + sum_{u,v<3} w_dw[c][u][v] x[b,i+u-1,j+v-1,c]
+ *                (zero padding of one pixel; cross-correlation)
+ *   z[b,i,j,o] = b_pw[o] + sum_c w_pw[o][c] y[b,i,j,c]
+ *   G = 1 / (1 + exp(-z))
+ *
+ *   x      : bf16 [B][H][W][C], the layer's input feature map (device)
+ *   w_dw   : fp32 [C][3][3]; b_dw : fp32 [C]            (device)
+ *   w_pw   : fp32 [C][C] ([out][in]); b_pw : fp32 [C]    (device)
+ *   gate   : out, bf16 [B][H][W][C]                      (device)
+ * The point-wise convolution runs on the tensor cores with y and w_pw
+ * rounded to bf16 (fp32 accumulation).  Requires C % 32 == 0, C <= 256,
+ * H % 8 == 0, W % 16 == 0 (else RIB_ERR_UNSUPPORTED / RIB_ERR_SHAPE); x and
+ * gate 16-byte aligned, w_pw 8-byte aligned (RIB_ERR_ALIGN).  Asynchronous
+ * on `stream`; allocates nothing.
+ * ------------------------------------------------------------------------ */
+int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw,
+                 const float* b_dw, const float* w_pw, const float* b_pw,
+                 void* gate, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rib_window_attn_fwd_cla -- rib_window_attn_fwd with the CLA gate applied
+ * in the same kernel's epilogue (German summary, Methodik §B: O' = O * G).
+ *
+ *   gate      : bf16 [B][H][W][heads*head_dim] from rib_cla_gate (channel
+ *               head*head_dim + e gates output channel e of that head)
+ *   out       : out, bf16 O [B][H][W][heads][head_dim] (kept: the backward
+ *               needs the ungated output)
+ *   out_gated : out, bf16 O * G, same layout
+ * Every other argument, requirement and error is as for
+ * rib_window_attn_fwd; gate and out_gated must be 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads,
+                            int head_dim, int window, int shift,
+                            const void* qp_bf16, const void* kp_bf16, int rank,
+                            float scale, const void* gate, void* out,
+                            void* out_gated, float* lse, void* stream);
+
 /* Bytes of device workspace rib_window_attn_bwd needs for these sizes;
  * `mlp` (host pointer, may be NULL) adds the MLP-gradient scratch. */
 size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads,

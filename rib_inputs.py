@@ -35,7 +35,7 @@ import torch
 
 __all__ = [
     "Workload", "WORKLOADS", "get_workload", "default_freqs", "make_qkv",
-    "make_dout", "make_mlp", "make_layer_inputs",
+    "make_dout", "make_mlp", "make_layer_inputs", "make_features", "make_cla", "ClaParams",
 ]
 
 
@@ -95,6 +95,7 @@ def _gen(seed: int, tag: int) -> torch.Generator:
 
 
 _TAG_QKV, _TAG_DOUT, _TAG_MLPQ, _TAG_MLPK, _TAG_MISC = 1, 2, 3, 4, 5
+_TAG_X, _TAG_CLA = 6, 7
 
 
 def default_freqs(n_freq: int = 16) -> torch.Tensor:
@@ -174,6 +175,37 @@ def make_layer_inputs(w: Workload, layer: int = 0, strong: bool = False,
         out["dout"] = make_dout(w.batch, w.height, w.width, w.heads,
                                 w.head_dim, seed)
     return out
+
+
+def make_features(batch, height, width, channels, seed, dtype=torch.bfloat16):
+    """Layer input feature map x [B][H][W][C] ~ N(0, 1), then cast (the
+    input of the convolutional local attention gate)."""
+    g = _gen(seed, _TAG_X)
+    return torch.randn((batch, height, width, channels), generator=g,
+                       dtype=torch.float32).to(dtype)
+
+
+@dataclass
+class ClaParams:
+    """Convolutional local attention gate weights, fp32: depth-wise 3x3
+    (w_dw [C][3][3], b_dw [C]) and point-wise 1x1 (w_pw [C][C], b_pw [C])."""
+    w_dw: torch.Tensor
+    b_dw: torch.Tensor
+    w_pw: torch.Tensor
+    b_pw: torch.Tensor
+
+
+def make_cla(channels, seed):
+    """CLA gate weights: w_dw ~ N(0, (1/3)^2) (a 3x3 tap sum of unit
+    variance), w_pw ~ N(0, 1/C) (unit-variance pre-activation), biases
+    N(0, 0.1^2), so the gate spans the sigmoid's whole range."""
+    g = _gen(seed, _TAG_CLA)
+    C = channels
+    w_dw = torch.randn((C, 3, 3), generator=g) / 3.0
+    b_dw = torch.randn((C,), generator=g) * 0.1
+    w_pw = torch.randn((C, C), generator=g) / math.sqrt(C)
+    b_pw = torch.randn((C,), generator=g) * 0.1
+    return ClaParams(w_dw.contiguous(), b_dw.contiguous(), w_pw.contiguous(), b_pw.contiguous())
 
 
 def randn(shape, seed, tag=_TAG_MISC, std=1.0, dtype=torch.float32):

@@ -1,0 +1,81 @@
+"""GPU parity of the convolutional local attention gate (rib_cla_gate) and of
+the gated forward (rib_window_attn_fwd_cla) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import rib_inputs as I
+import windowed_attention_implicit_b200 as R
+from tests.rib_testlib import Case, assert_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _gate(B, H, W, C, seed):
+    x = I.make_features(B, H, W, C, seed)
+    p = I.make_cla(C, seed)
+    cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    return x, p, cla
+
+
+@pytest.mark.parametrize("B,H,W,C", [
+    (1, 8, 16, 32),       # one tile: every pixel touches the zero padding
+    (1, 24, 48, 96),      # tiny workload's width (3 heads), partial 64-channel group
+    (2, 32, 32, 192),     # six heads, several tiles per image, two images
+    (1, 16, 32, 256),     # largest channel count one MMA covers
+])
+def test_cla_gate_parity(B, H, W, C):
+    x, p, cla = _gate(B, H, W, C, seed=C + H)
+    g = R.rib_cla_gate(x.cuda(), cla)
+    torch.cuda.synchronize()
+    code, site = R.rib_last_status()
+    assert code == 0, (code, site)
+    ref = O.cla_gate(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    assert_close(to_np(g), ref, f"gate B={B} {H}x{W} C={C}")
+
+
+def test_cla_gate_full_size_map():
+    """The 96x96-window training map: B=4, 192x192, C=192 (all 1152 tiles,
+    the persistent grid's every CTA), compared on every pixel."""
+    x, p, cla = _gate(4, 192, 192, 192, seed=3)
+    g = R.rib_cla_gate(x.cuda(), cla)
+    torch.cuda.synchronize()
+    assert R.rib_last_status()[0] == 0
+    ref = O.cla_gate(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    assert_close(to_np(g), ref, "gate 4x192x192x192")
+
+
+@pytest.mark.parametrize("args", [
+    dict(B=1, H=64, W=64, heads=3, M=16, s=0),
+    dict(B=2, H=64, W=96, heads=6, M=32, s=16),
+])
+def test_attn_fwd_cla_parity(args):
+    c = Case(seed=11, **args)
+    C = c.heads * 32
+    x, p, cla = _gate(c.B, c.H, c.W, C, seed=5)
+    d = c.device()
+    gate = R.rib_cla_gate(x.cuda(), cla)
+    out, out_g, lse = R.rib_window_attn_fwd_cla(d["qkv"], c.M, c.s, gate, d["qp16"], d["kp16"])
+    out0, lse0 = R.rib_window_attn_fwd(d["qkv"], c.M, c.s, d["qp16"], d["kp16"])
+    torch.cuda.synchronize()
+    assert R.rib_last_status()[0] == 0
+    # the ungated output and lse are the plain forward's, bit for bit
+    assert torch.equal(out, out0) and torch.equal(lse, lse0)
+    ro, rl = c.oracle_fwd()
+    rg = O.cla_gate(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    assert_close(to_np(out_g), O.cla_apply(ro, rg), "gated output")
+    assert_close(to_np(out), ro, "ungated output")
+
+
+def test_cla_gate_rejects_bad_shapes():
+    x = torch.zeros((1, 8, 16, 48), device="cuda", dtype=torch.bfloat16)
+    p = I.make_cla(48, 1)
+    cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    with pytest.raises(R.RibError):
+        R.rib_cla_gate(x, cla)                      # C % 32 != 0
+    x = torch.zeros((1, 12, 16, 64), device="cuda", dtype=torch.bfloat16)
+    p = I.make_cla(64, 1)
+    cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    with pytest.raises(R.RibError):
+        R.rib_cla_gate(x, cla)                      # H % 8 != 0

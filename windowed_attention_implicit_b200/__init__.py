@@ -28,7 +28,8 @@ __all__ = [
     "rib_window_attn_fwd", "rib_window_attn_bwd", "rib_window_attn_bwd_workspace",
     "rib_window_gather", "rib_window_scatter", "rib_last_status", "rib_status_string",
     "rib_set_wait_limit_ns", "rib_debug_wait_timeout", "rib_version", "library",
-    "rib_trace_enable", "rib_trace_collect", "rib_debug_exp2",
+    "rib_trace_enable", "rib_trace_collect", "rib_debug_exp2", "ClaGate", "rib_cla_gate",
+    "rib_window_attn_fwd_cla",
 ]
 
 
@@ -215,6 +216,61 @@ def rib_window_attn_fwd(qkv: torch.Tensor, window: int, shift: int, qp_bf16=None
         int(rank), float(scale), _ptr(out, torch.bfloat16, "out"),
         _ptr(lse, torch.float32, "lse"), _stream(stream)), "rib_window_attn_fwd")
     return out, lse
+
+
+@dataclass
+class ClaGate:
+    """Device fp32 weights of the convolutional local attention gate:
+    depth-wise 3x3 (w_dw [C][3][3], b_dw [C]) then point-wise 1x1
+    (w_pw [C_out][C_in], b_pw [C]) then a sigmoid."""
+    w_dw: torch.Tensor
+    b_dw: torch.Tensor
+    w_pw: torch.Tensor
+    b_pw: torch.Tensor
+
+    @classmethod
+    def from_params(cls, w_dw, b_dw, w_pw, b_pw, device="cuda"):
+        f = lambda t: torch.as_tensor(t).detach().to(device=device, dtype=torch.float32).contiguous()
+        return cls(f(w_dw), f(b_dw), f(w_pw), f(b_pw))
+
+    @property
+    def channels(self) -> int:
+        return self.b_dw.numel()
+
+
+def rib_cla_gate(x: torch.Tensor, cla: ClaGate, gate=None, stream=None) -> torch.Tensor:
+    """G bf16 [B][H][W][C] = sigmoid(PW1x1(DW3x3(x))) for x bf16 [B][H][W][C]."""
+    B, H, W, C = x.shape
+    gate = torch.empty_like(x) if gate is None else gate
+    f32 = torch.float32
+    _check(library().rib_cla_gate(
+        _ptr(x, torch.bfloat16, "x"), B, H, W, C, _ptr(cla.w_dw, f32, "w_dw"),
+        _ptr(cla.b_dw, f32, "b_dw"), _ptr(cla.w_pw, f32, "w_pw"), _ptr(cla.b_pw, f32, "b_pw"),
+        _ptr(gate, torch.bfloat16, "gate"), _stream(stream)), "rib_cla_gate")
+    return gate
+
+
+def rib_window_attn_fwd_cla(qkv: torch.Tensor, window: int, shift: int, gate: torch.Tensor,
+                            qp_bf16=None, kp_bf16=None, rank: int = 16, scale: float = 0.0,
+                            out=None, out_gated=None, lse=None, stream=None):
+    """(out, out_gated, lse): the attention output O, O * gate (gate bf16
+    [B][H][W][heads*d]) and lse, from one forward launch."""
+    B, H, W, three, heads, d = qkv.shape
+    if three != 3:
+        raise ValueError("qkv must be [B][H][W][3][heads][head_dim]")
+    if tuple(gate.shape) not in ((B, H, W, heads * d), (B, H, W, heads, d)):
+        raise ValueError("gate must be [B][H][W][heads*head_dim]")
+    shape = (B, H, W, heads, d)
+    out = torch.empty(shape, device=qkv.device, dtype=torch.bfloat16) if out is None else out
+    out_gated = torch.empty(shape, device=qkv.device, dtype=torch.bfloat16) if out_gated is None else out_gated
+    lse = torch.empty((B, heads, H, W), device=qkv.device, dtype=torch.float32) if lse is None else lse
+    _check(library().rib_window_attn_fwd_cla(
+        _ptr(qkv, torch.bfloat16, "qkv"), B, H, W, heads, d, int(window), int(shift),
+        _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
+        int(rank), float(scale), _ptr(gate, torch.bfloat16, "gate"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(out_gated, torch.bfloat16, "out_gated"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream)), "rib_window_attn_fwd_cla")
+    return out, out_gated, lse
 
 
 def rib_window_attn_bwd_workspace(B, H, W, heads, head_dim, window, rank,

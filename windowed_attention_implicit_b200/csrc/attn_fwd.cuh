@@ -86,6 +86,8 @@ struct FwdParams {
   float scale_log2;  // softmax scale * log2(e)
   __nv_bfloat16* out;
   float* lse;
+  const __nv_bfloat16* gate;   // CLA gate G [B][H][W][heads*32], or null
+  __nv_bfloat16* out_gated;    // O * G, written when gate is set
   uint64_t wait_limit_ns;
 };
 
@@ -388,6 +390,27 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   uint4* dst = reinterpret_cast<uint4*>(p.out + (pix * p.heads + u.head) * 32);
 #pragma unroll
   for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  if (p.gate != nullptr) {
+    // convolutional local attention: O' = O * G at the same pixel and
+    // channels (German summary, Methodik §B); O itself is kept for the
+    // backward.  The product is formed from the fp32 O, then rounded.
+    const uint4* g4 = reinterpret_cast<const uint4*>(p.gate + (pix * p.heads + u.head) * 32);
+    uint4* dg = reinterpret_cast<uint4*>(p.out_gated + (pix * p.heads + u.head) * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 gv = g4[q];
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+      uint32_t r4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[e]));
+        const int c = 8 * q + 2 * e;
+        r4[e] = pack_bf16x2(__uint_as_float(o[c]) * inv * gf.x,
+                            __uint_as_float(o[c + 1]) * inv * gf.y);
+      }
+      dg[q] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+    }
+  }
   p.lse[(static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x] =
       (m_run + log2f(l_run)) * 0.69314718055994531f;
 }

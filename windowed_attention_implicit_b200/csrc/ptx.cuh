@@ -18,7 +18,7 @@ enum WaitSite : int {
   SITE_DEBUG = 1,
   SITE_FWD_PRODUCER = 10, SITE_FWD_MMA = 11, SITE_FWD_SOFTMAX = 12, SITE_FWD_DRAIN = 13,
   SITE_BWD_PRODUCER = 20, SITE_BWD_MMA = 21, SITE_BWD_COMPUTE = 22, SITE_BWD_DRAIN = 23,
-  SITE_COPY = 30,
+  SITE_COPY = 30, SITE_CLA = 40,
 };
 
 constexpr int kErrTimeout = -6;

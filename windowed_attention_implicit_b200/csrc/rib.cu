@@ -21,6 +21,7 @@
 #include "window_copy.cuh"
 #include "attn_fwd.cuh"
 #include "attn_bwd.cuh"
+#include "cla.cuh"
 
 namespace rib {
 namespace {
@@ -113,13 +114,13 @@ int map_pixel_f32(CUtensorMap* m, const void* base, int B, int heads, int H, int
 // ---------------------------------------------------------------- tracing
 enum KernelId {
   K_POS, K_FWD, K_BWD_PRE, K_BWD, K_DQ_FIN, K_POSGRAD, K_MLP_PART, K_MLP_RED, K_COPY, K_DEBUG,
-  K_COUNT
+  K_CLA, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "pos_tokens_kernel",   "attn_fwd_kernel",        "bwd_preprocess_kernel",
     "attn_bwd_kernel",     "dq_finalize_kernel",     "posgrad_reduce_kernel",
     "mlp_bwd_partial_kernel", "mlp_bwd_reduce_kernel", "window_copy_kernel",
-    "debug_wait_kernel"};
+    "debug_wait_kernel",   "cla_gate_kernel"};
 
 struct TraceRec {
   int id;
@@ -491,10 +492,13 @@ int rib_pos_tokens_bwd_noalloc(const rib_mlp_t* mlp, int window, const float* dq
                         static_cast<cudaStream_t>(stream));
 }
 
-int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads, int head_dim,
-                        int window, int shift, const void* qp_bf16, const void* kp_bf16,
-                        int rank, float scale, void* out, float* lse, void* stream) {
+static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int head_dim,
+                           int window, int shift, const void* qp_bf16, const void* kp_bf16,
+                           int rank, float scale, void* out, float* lse, const void* gate,
+                           void* out_gated, void* stream) {
   if (!qkv || !out || !lse) return RIB_ERR_ARG;
+  if ((gate == nullptr) != (out_gated == nullptr)) return RIB_ERR_ARG;
+  if (gate && (!aligned16(gate) || !aligned16(out_gated))) return RIB_ERR_ALIGN;
   AttnGeom g;
   int rc = check_attn(B, H, W, heads, head_dim, window, shift, rank, &g);
   if (rc) return rc;
@@ -519,6 +523,8 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads, int hea
   p.scale_log2 = tau * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.out_gated = static_cast<__nv_bfloat16*>(out_gated);
   p.wait_limit_ns = g_wait_limit_ns;
   if ((rc = set_smem(attn_fwd_kernel, kFwdSmemBytes))) return rc;
   {
@@ -535,6 +541,57 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads, int hea
   TraceScope ts(K_FWD, static_cast<cudaStream_t>(stream));
   attn_fwd_kernel<<<grid, kFwdThreads, kFwdSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       tq, tqp, tkp, p);
+  return launch_status();
+}
+
+int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads, int head_dim,
+                        int window, int shift, const void* qp_bf16, const void* kp_bf16,
+                        int rank, float scale, void* out, float* lse, void* stream) {
+  return attn_fwd_launch(qkv, B, H, W, heads, head_dim, window, shift, qp_bf16, kp_bf16, rank,
+                         scale, out, lse, nullptr, nullptr, stream);
+}
+
+int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads, int head_dim,
+                            int window, int shift, const void* qp_bf16, const void* kp_bf16,
+                            int rank, float scale, const void* gate, void* out, void* out_gated,
+                            float* lse, void* stream) {
+  if (!gate || !out_gated) return RIB_ERR_ARG;
+  return attn_fwd_launch(qkv, B, H, W, heads, head_dim, window, shift, qp_bf16, kp_bf16, rank,
+                         scale, out, lse, gate, out_gated, stream);
+}
+
+int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, const float* b_dw,
+                 const float* w_pw, const float* b_pw, void* gate, void* stream) {
+  if (!x || !w_dw || !b_dw || !w_pw || !b_pw || !gate) return RIB_ERR_ARG;
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
+  if (C % 32 != 0 || C > kClaMaxC) return RIB_ERR_UNSUPPORTED;
+  if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
+  if ((long long)B * H * W * C > (1ll << 40)) return RIB_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(gate) || (reinterpret_cast<uintptr_t>(w_pw) & 7u) ||
+      (reinterpret_cast<uintptr_t>(w_dw) & 3u) || (reinterpret_cast<uintptr_t>(b_dw) & 3u) ||
+      (reinterpret_cast<uintptr_t>(b_pw) & 3u))
+    return RIB_ERR_ALIGN;
+  ClaParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.w_dw = w_dw; p.b_dw = b_dw; p.w_pw = w_pw; p.b_pw = b_pw;
+  p.gate = static_cast<__nv_bfloat16*>(gate);
+  p.B = B; p.H = H; p.W = W; p.C = C;
+  p.tiles_x = W / 16;
+  p.tiles_per_img = (H / 8) * (W / 16);
+  const long long n_tiles = (long long)B * p.tiles_per_img;
+  if (n_tiles > (1ll << 30)) return RIB_ERR_UNSUPPORTED;
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.wait_limit_ns = g_wait_limit_ns;
+  const size_t smem = cla_smem_bytes(C);
+  int rc;
+  if ((rc = set_smem(cla_gate_kernel, smem))) return rc;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return RIB_ERR_CUDA;
+  const int grid = static_cast<int>(n_tiles < sms ? n_tiles : sms);
+  TraceScope ts(K_CLA, static_cast<cudaStream_t>(stream));
+  cla_gate_kernel<<<grid, kClaThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
   return launch_status();
 }
 
