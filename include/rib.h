@@ -186,7 +186,7 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads,
  *   w_pw   : fp32 [C][C] ([out][in]); b_pw : fp32 [C]    (device)
  *   gate   : out, bf16 [B][H][W][C]                      (device)
  * The point-wise convolution runs on the tensor cores with y and w_pw
- * rounded to bf16 (fp32 accumulation).  Requires C % 32 == 0, C <= 256,
+ * rounded to bf16 (fp32 accumulation).  Requires C % 32 == 0, C <= 192,
  * H % 8 == 0, W % 16 == 0 (else RIB_ERR_UNSUPPORTED / RIB_ERR_SHAPE); x and
  * gate 16-byte aligned, w_pw 8-byte aligned (RIB_ERR_ALIGN).  Asynchronous
  * on `stream`; allocates nothing.

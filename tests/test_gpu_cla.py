@@ -23,7 +23,7 @@ def _gate(B, H, W, C, seed):
     (1, 8, 16, 32),       # one tile: every pixel touches the zero padding
     (1, 24, 48, 96),      # tiny workload's width (3 heads), partial 64-channel group
     (2, 32, 32, 192),     # six heads, several tiles per image, two images
-    (1, 16, 32, 256),     # largest channel count one MMA covers
+    (1, 16, 32, 160),     # five heads: a partial 64-channel halo box
 ])
 def test_cla_gate_parity(B, H, W, C):
     x, p, cla = _gate(B, H, W, C, seed=C + H)
@@ -79,3 +79,8 @@ def test_cla_gate_rejects_bad_shapes():
     cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
     with pytest.raises(R.RibError):
         R.rib_cla_gate(x, cla)                      # H % 8 != 0
+    x = torch.zeros((1, 8, 16, 256), device="cuda", dtype=torch.bfloat16)
+    p = I.make_cla(256, 1)
+    cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    with pytest.raises(R.RibError):
+        R.rib_cla_gate(x, cla)                      # C > 192: no room for the buffers

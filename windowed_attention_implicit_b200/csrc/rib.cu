@@ -564,15 +564,22 @@ int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, c
                  const float* w_pw, const float* b_pw, void* gate, void* stream) {
   if (!x || !w_dw || !b_dw || !w_pw || !b_pw || !gate) return RIB_ERR_ARG;
   if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
-  if (C % 32 != 0 || C > kClaMaxC) return RIB_ERR_UNSUPPORTED;
+  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u) return RIB_ERR_UNSUPPORTED;
   if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
-  if ((long long)B * H * W * C > (1ll << 40)) return RIB_ERR_UNSUPPORTED;
+  if ((long long)B * H * W * C > (1ll << 40) || B > (1 << 20)) return RIB_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(gate) || (reinterpret_cast<uintptr_t>(w_pw) & 7u) ||
       (reinterpret_cast<uintptr_t>(w_dw) & 3u) || (reinterpret_cast<uintptr_t>(b_dw) & 3u) ||
       (reinterpret_cast<uintptr_t>(b_pw) & 3u))
     return RIB_ERR_ALIGN;
+  // x [B][H][W][C] bf16 as a 4D map; box = one tile's 10 x 18 halo, 64 channels
+  CUtensorMap tm;
+  const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)H, (uint64_t)B};
+  const uint64_t strides[3] = {2ull * C, 2ull * C * W, 2ull * C * W * H};
+  const uint32_t box[4] = {64, 18, 10, 1};
+  int rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, dims, strides, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
   ClaParams p{};
-  p.x = static_cast<const __nv_bfloat16*>(x);
   p.w_dw = w_dw; p.b_dw = b_dw; p.w_pw = w_pw; p.b_pw = b_pw;
   p.gate = static_cast<__nv_bfloat16*>(gate);
   p.B = B; p.H = H; p.W = W; p.C = C;
@@ -583,7 +590,6 @@ int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, c
   p.n_tiles = static_cast<int>(n_tiles);
   p.wait_limit_ns = g_wait_limit_ns;
   const size_t smem = cla_smem_bytes(C);
-  int rc;
   if ((rc = set_smem(cla_gate_kernel, smem))) return rc;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -591,7 +597,7 @@ int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, c
     return RIB_ERR_CUDA;
   const int grid = static_cast<int>(n_tiles < sms ? n_tiles : sms);
   TraceScope ts(K_CLA, static_cast<cudaStream_t>(stream));
-  cla_gate_kernel<<<grid, kClaThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  cla_gate_kernel<<<grid, kClaThreads, smem, static_cast<cudaStream_t>(stream)>>>(tm, p);
   return launch_status();
 }
 
