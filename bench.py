@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--step-only", action="store_true",
                     help="run only warm-up + timed training steps (for profiler launch lists)")
+    ap.add_argument("--cla-only", action="store_true",
+                    help="run only the convolutional local attention gate and the gated "
+                         "forward, warm-up + timed (for profiler captures)")
     return ap.parse_args()
 
 
@@ -151,6 +154,23 @@ def stored_traffic(kernel, workload):
     if d.get("source_hash") != kernel_source_hash():
         return None
     return d.get("dram_bytes_per_launch")
+
+
+def cla_line(w, kern_g, ms_gate_total, ms_fwd_cla_total, ms_fwd, pk):
+    """Convolutional local attention (measured beside the hot path, not part
+    of its step): the gate kernel against the HBM roofline (x read + G
+    written, 2 bytes each per pixel and channel) and the extra cost of
+    applying the gate in the forward epilogue."""
+    steps = kern_g["cla_gate_kernel"][0]
+    ms_g = kern_g["cla_gate_kernel"][1] / steps
+    C = w.heads * w.head_dim
+    byt = 2 * w.batch * w.height * w.width * C * 2
+    gbs = byt / (ms_g * 1e-3) / 1e9
+    fwd_cla = ms_fwd_cla_total / steps
+    return {"gate_kernel_ms": ms_g, "gate_bytes": byt, "gate_gbs": gbs,
+            "gate_frac_hbm": gbs / pk["hbm_gbs"], "fwd_cla_ms": fwd_cla,
+            "fwd_cla_extra_ms": fwd_cla - ms_fwd, "bound": "hbm",
+            "workload": f"x, G bf16 [{w.batch}][{w.height}][{w.width}][{C}]"}
 
 
 # ---------------------------------------------------------------- oracle leg
@@ -285,6 +305,20 @@ def run_rib(args, w):
     def fwd_only():
         R.rib_window_attn_fwd(qkv, M, s, q16, k16, out=out, lse=lse)
 
+    # convolutional local attention gate on this workload's feature map
+    # (C = heads * d channels) and the forward with the gate applied
+    cla_p = I.make_cla(heads * d, w.seed)
+    cla = R.ClaGate.from_params(cla_p.w_dw, cla_p.b_dw, cla_p.w_pw, cla_p.b_pw, device=dev)
+    feat = I.make_features(B, H, W, heads * d, w.seed).to(dev)
+    gate = torch.empty_like(feat)
+    out_g = torch.empty_like(out)
+
+    def cla_gate_only():
+        R.rib_cla_gate(feat, cla, gate=gate)
+
+    def fwd_cla():
+        R.rib_window_attn_fwd_cla(qkv, M, s, gate, q16, k16, out=out, out_gated=out_g, lse=lse)
+
     def timed(fn, steps, trace=False):
         stream = torch.cuda.current_stream()
         if world > 1:
@@ -313,6 +347,20 @@ def run_rib(args, w):
     sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
     if sampler:
         sampler.start()       # samples cover warm-up and every timed loop below
+    if args.cla_only:
+        for _ in range(args.warmup):
+            cla_gate_only()
+            fwd_cla()
+        ms_g, _, _ = timed(cla_gate_only, args.steps)
+        ms_c, _, _ = timed(fwd_cla, args.steps)
+        if sampler:
+            sampler.stop()
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"cla_only": True, "cla_gate_ms": ms_g / args.steps,
+                              "fwd_cla_ms": ms_c / args.steps}))
+        return 0
     for _ in range(args.warmup):
         step()
     code, site = R.rib_last_status()
@@ -336,6 +384,15 @@ def run_rib(args, w):
         fwd_only()
     ms_f, kern_f, _ = timed(fwd_only, args.steps, trace=True)
     ms_fwd = ms_f / args.steps
+    code, site = R.rib_last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
+
+    for _ in range(args.warmup):
+        cla_gate_only()
+        fwd_cla()
+    ms_g, kern_g, _ = timed(cla_gate_only, args.steps, trace=True)
+    ms_c, _, _ = timed(fwd_cla, args.steps)
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
@@ -414,6 +471,7 @@ def run_rib(args, w):
                 "tokens_per_s": world * w.tokens() / (ms_fwd * 1e-3),
                 "kernel_tflops": fwd_ach, "kernel_frac": fwd_ach / peak},
         "roofline": roof,
+        "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk),
         "kernels": per_kernel,
         "gpu_launches": launches,
         "cpu_baseline": cpu,

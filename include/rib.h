@@ -239,8 +239,9 @@ size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads,
  *   dmlp     : host pointer to device gradient buffers (may be NULL)
  *   workspace: device scratch of at least rib_window_attn_bwd_workspace()
  *              bytes, 256-byte aligned; contents need not be initialised
- * dQ is accumulated with fp32 atomics across key tiles, so dqkv's query
- * part and dqp may differ in the last bits between runs.
+ * dQ partials of the key tiles are summed with fp32 reduce-adds in no fixed
+ * order, so dqkv's query part and dqp may differ in the last bits between
+ * runs.
  * ------------------------------------------------------------------------ */
 int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout,
                         const float* lse, int B, int H, int W, int heads,

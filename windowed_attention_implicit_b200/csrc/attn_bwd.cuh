@@ -25,14 +25,15 @@
 //               TMA reduce-add into the fp32 accumulator per query tile
 //   warp  12    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 4 stages)
 //   warp  13    issues the S^T / dP^T MMAs
-//   warp  14    TMEM allocator; issues the gradient MMAs (dV, dK_aug, dQ_aug)
-//   warp  15    idle
-// The tensor pipe runs all of these back to back only if no single thread's
-// waits stall it: a tcgen05.mma blocks its issuing thread for ~45 cycles and
-// a tcgen05.commit for ~270, so scores and gradients have separate issuers;
-// and the compute warps neither drain dQ (dedicated warps do) nor wait for
-// the previous tile's gradient MMAs before their exponentials (they form the
-// whole tile in registers first, then wait for the P^T/dS^T buffers).
+//   warp  14    TMEM allocator; issues the dV and dK_aug MMAs
+//   warp  15    issues the dQ_aug MMAs
+// Each MMA-issuing warp runs converged and issues through one elected lane
+// (a thread issues one tcgen05.mma per ~43 cycles that way, against ~90 from
+// a divergent branch), and the three MMA groups have separate issuers so
+// that no group's waits hold back another's.  The compute warps neither
+// drain dQ (dedicated warps do) nor wait for the previous tile's gradient
+// MMAs before their exponentials (they form the whole tile in registers
+// first, then wait for the P^T/dS^T buffers).
 // Per query tile i:  S^T = K_aug Q_aug^T and dP^T = V dO^T (MMA, TMEM) ->
 // compute warps form P^T and dS^T (to TMEM) and dS (to shared memory,
 // core-matrix layout, double-buffered) -> MMA: dV += P^T dO and
