@@ -25,8 +25,8 @@
 //               TMA reduce-add into the fp32 accumulator per query tile
 //   warp  12    TMA producer (K tile once; Q/dO/Qp/lse/D tiles, 4 stages)
 //   warp  13    issues the S^T / dP^T MMAs
-//   warp  14    TMEM allocator; issues the dV and dK_aug MMAs
-//   warp  15    issues the dQ_aug MMAs
+//   warp  14    TMEM allocator; issues the dV MMAs
+//   warp  15    issues the dK_aug, then the dQ_aug MMAs
 // Each MMA-issuing warp runs converged and issues through one elected lane
 // (a thread issues one tcgen05.mma per ~43 cycles that way, against ~90 from
 // a divergent branch), and the three MMA groups have separate issuers so
@@ -106,7 +106,6 @@ struct __align__(1024) BwdSmem {
   uint64_t k_full;
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
   uint64_t s_full, s_free, ds_full, pt_free /* P^T and dS^T in TMEM */, ds_free[2];
-  uint64_t dsq_full[2];            // dS buffer b written (for the dQ issuer)
   uint64_t dq_full, dq_free, mma_done;
   int drain_ok[4];
   uint64_t drain;
@@ -212,13 +211,13 @@ __device__ __forceinline__ void bwd_mma_scores(BwdSmem& sm, uint32_t tmem, const
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
 }
 
-// Warp 14 (all lanes; one elected lane issues): dV += P^T dO and
-// dK_aug += dS^T [Qc|Qp] (A from TMEM) of every query tile.
+// Warp 14 (all lanes; one elected lane issues): dV += P^T dO (A = P^T from
+// TMEM) of every query tile.  P^T/dS^T (pt_free) and the query stage
+// (q_empty) are released by this warp and warp 15 together (two arrivals).
 __device__ __forceinline__ void bwd_mma_grads(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int n = p.n_tiles;
-  const uint32_t lbo_q = smem_u32(sm.qp[0]) - smem_u32(sm.qc[0]);   // [Qc|Qp] atoms
   bool ok = true;
   for (int i = 0; ok && i < n; ++i) {
     const int st = i % kBwdStages;
@@ -226,35 +225,41 @@ __device__ __forceinline__ void bwd_mma_grads(BwdSmem& sm, uint32_t tmem, const 
     // waited for them (q_full) before forming P^T and dS^T.
     if (!(ok = warp_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
     tc_fence_after();
-    const uint32_t qc = smem_u32(sm.qc[st]), dO = smem_u32(sm.dO[st]);
+    const uint32_t dO = smem_u32(sm.dO[st]);
     // dV += P^T dO   (K = queries, 16 per step; A from TMEM)
     umma_ts8_elect(tmem + kBColDV, tmem + kBColP, make_sdesc(dO, 16, 512, kLayoutSW64),
                    1024 >> 4, kIdescBV, i > 0 ? 1u : 0u);
-    // dK_aug += dS^T [Qc|Qp]   (A = dS^T from TMEM)
-    umma_ts8_elect(tmem + kBColDK, tmem + kBColDST, make_sdesc(qc, lbo_q, 512, kLayoutSW64),
-                   1024 >> 4, kIdescBK, i > 0 ? 1u : 0u);
     umma_commit_elect(&sm.pt_free);
     umma_commit_elect(&sm.q_empty[st]);
   }
-  umma_commit_elect(&sm.mma_done);   // every dV / dK MMA of the kernel has completed
+  umma_commit_elect(&sm.mma_done);   // every dV MMA of the kernel has completed
   umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
 }
 
-// Warp 15 (all lanes; one elected lane issues): dQ_aug = dS [Kc|Kp] (A = dS
-// MN-major core matrices in shared memory) of every query tile.  dS buffer
-// b has its own barrier, so this issuer's parity waits stay exact even when
-// the compute warps run a tile ahead of it.
+// Warp 15 (all lanes; one elected lane issues): dK_aug += dS^T [Qc|Qp] (A =
+// dS^T from TMEM), then dQ_aug = dS [Kc|Kp] (A = dS MN-major core matrices
+// in shared memory) of every query tile.  Its dK commit releases P^T/dS^T
+// together with warp 14's dV commit, so the compute warps cannot form tile
+// i+1 before this warp has taken tile i: ds_full never runs ahead of it.
 __device__ __forceinline__ void bwd_mma_dq(BwdSmem& sm, uint32_t tmem, const BwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int n = p.n_tiles;
   const uint32_t kc = smem_u32(sm.kc), kp = smem_u32(sm.kp);
-  const uint32_t lbo_k = kp - kc;  // [Kc|Kp] atoms
+  const uint32_t lbo_k = kp - kc;                                   // [Kc|Kp] atoms
+  const uint32_t lbo_q = smem_u32(sm.qp[0]) - smem_u32(sm.qc[0]);  // [Qc|Qp] atoms
   bool ok = true;
   for (int i = 0; ok && i < n; ++i) {
-    if (!(ok = warp_wait(&sm.dsq_full[i & 1], (i >> 1) & 1, ab, lim, SITE_BWD_MMA))) break;
+    const int st = i % kBwdStages;
+    if (!(ok = warp_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
+    tc_fence_after();
+    umma_ts8_elect(tmem + kBColDK, tmem + kBColDST,
+                   make_sdesc(smem_u32(sm.qc[st]), lbo_q, 512, kLayoutSW64), 1024 >> 4, kIdescBK,
+                   i > 0 ? 1u : 0u);
+    umma_commit_elect(&sm.pt_free);
+    umma_commit_elect(&sm.q_empty[st]);
     // the single dQ buffer is free once the drain warps pulled tile i-1
     if (i > 0 && !(ok = warp_wait(&sm.dq_free, (i - 1) & 1, ab, lim, SITE_BWD_MMA))) break;
     tc_fence_after();
@@ -265,6 +270,7 @@ __device__ __forceinline__ void bwd_mma_dq(BwdSmem& sm, uint32_t tmem, const Bwd
     umma_commit_elect(&sm.ds_free[i & 1]);
     umma_commit_elect(&sm.dq_full);
   }
+  umma_commit_elect(&sm.mma_done);   // every dK MMA of the kernel has completed
   umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
   mbar_wait(&sm.drain, 0, &no_abort, kBwdDrainNs, SITE_BWD_DRAIN);
@@ -411,10 +417,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&sm.ds_full);
-      mbar_arrive(&sm.dsq_full[i & 1]);
-    }
+    if (lane == 0) mbar_arrive(&sm.ds_full);
   }
   if (!ok) return;
   if (!warp_wait(&sm.mma_done, 0, ab, lim, SITE_BWD_COMPUTE)) return;
@@ -487,19 +490,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.k_full, 1);
     for (int st = 0; st < kBwdStages; ++st) {
       mbar_init(&sm.q_full[st], 1);
-      mbar_init(&sm.q_empty[st], 1);
+      mbar_init(&sm.q_empty[st], 2);   // warps 14 and 15
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.s_free, 8);
     mbar_init(&sm.ds_full, 8);
-    mbar_init(&sm.pt_free, 1);
+    mbar_init(&sm.pt_free, 2);       // dV (warp 14) and dK (warp 15)
     mbar_init(&sm.ds_free[0], 1);
     mbar_init(&sm.ds_free[1], 1);
-    mbar_init(&sm.dsq_full[0], 8);
-    mbar_init(&sm.dsq_full[1], 8);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_free, 4);
-    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.mma_done, 2);
     mbar_init(&sm.drain, 3);   // one commit from each MMA-issuing warp
     sm.abort_flag = 0;
     fence_mbarrier_init();
