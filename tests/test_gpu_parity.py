@@ -71,6 +71,10 @@ FWD_CASES = [
     (1, 96, 96, 1, 48, 24, 16, True),     # 3 tiles per tile row, 18 tiles
     (1, 64, 64, 2, 32, 0, 0, True),       # rank 0: plain windowed attention
     (1, 128, 128, 1, 64, 56, 16, True),   # largest shift < M
+    (1, 96, 96, 2, 96, 0, 16, True),      # 96x96 window, no shift
+    (1, 96, 192, 1, 96, 72, 16, True),    # H != W, shift 72: boxes wrap at the map edge
+    (1, 96, 96, 1, 48, 0, 0, True),       # rank 0, 18 tiles per unit
+    (1, 96, 96, 1, 48, 8, 16, True),      # shift of one box
 ]
 
 

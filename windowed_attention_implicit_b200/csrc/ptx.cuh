@@ -275,37 +275,53 @@ __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
       : "memory");
 }
 
-// Eight MMAs D (+)= A_k B_k^T, k = 0..7, issued by one elected lane of a
-// converged warp: A_k = tensor memory at a_tmem + 8k (16 bf16 columns per
-// step), B_k = b_desc advanced by k * b_step (descriptor units of 16 bytes).
-// `first_acc` = 0 makes the first MMA overwrite D.  One election and no
-// per-MMA descriptor arithmetic keep the issuing warp's instruction count
-// low while it shares its scheduler with busy warps.
+// STEPS MMAs D (+)= A_k B_k^T, k = 0..STEPS-1 (STEPS = 6 or 8), issued by
+// one elected lane of a converged warp: A_k = tensor memory at a_tmem + 8k
+// (16 bf16 columns per step), B_k = b_desc advanced by k * b_step
+// (descriptor units of 16 bytes).  `first_acc` = 0 makes the first MMA
+// overwrite D.  One election and no per-step descriptor arithmetic keep the
+// issuing warp's instruction count low while it shares its scheduler with
+// busy warps.
+#define RIB_TS_STEP                                                   \
+  "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"                    \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+template <int STEPS>
+__device__ __forceinline__ void umma_ts_chain_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                    uint64_t b_desc, uint32_t b_step,
+                                                    uint32_t idesc, uint32_t first_acc) {
+  static_assert(STEPS == 6 || STEPS == 8, "chains of 6 or 8 K-steps");
+  if constexpr (STEPS == 8) {
+    asm volatile(
+        "{\n\t.reg .pred p, e, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "mov.b32 a, %1;\n\t mov.b64 b, %2;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, p;\n\t"
+        RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP
+        "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "l"(static_cast<uint64_t>(b_step)),
+        "r"(idesc), "r"(first_acc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p, e, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "mov.b32 a, %1;\n\t mov.b64 b, %2;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, p;\n\t"
+        RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP RIB_TS_STEP
+        "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "l"(static_cast<uint64_t>(b_step)),
+        "r"(idesc), "r"(first_acc)
+        : "memory");
+  }
+}
+#undef RIB_TS_STEP
+
 __device__ __forceinline__ void umma_ts8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                uint32_t b_step, uint32_t idesc,
                                                uint32_t first_acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, e, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "setp.eq.b32 t, %4, %4;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
-      "add.s32 a, %1, 8;\n\t add.s64 b, %2, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
-      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
-      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
-      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
-      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
-      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
-      "add.s32 a, a, 8;\n\t add.s64 b, b, %3;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "l"(static_cast<uint64_t>(b_step)), "r"(idesc), "r"(first_acc)
-      : "memory");
+  umma_ts_chain_elect<8>(d_tmem, a_tmem, b_desc, b_step, idesc, first_acc);
 }
 
 // The same with A from shared memory: A_k = a_desc + k * a_step.
