@@ -213,6 +213,37 @@ int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads,
                             float scale, const void* gate, void* out,
                             void* out_gated, float* lse, void* stream);
 
+/* ------------------------------------------------------------------------
+ * rib_cla_bwd -- backward of the CLA gate (the gradients of O' = O * G for
+ * the gate of rib_cla_gate; English summary §2.B, German summary §B).
+ * With dO' the gradient of the gated output:
+ *   dO = dO' * G,   dz = dO' * O * G * (1 - G),
+ *   db_pw = sum_pixels dz,   dW_pw = sum_pixels dz^T y   (y recomputed),
+ *   dy = dz W_pw,   db_dw = sum_pixels dy,
+ *   dW_dw[c][u][v] = sum_pixels dy[p][c] x[p + (u-1, v-1)][c],
+ *   dx[p][c] = sum_{u,v} W_dw[c][u][v] dy[p - (u-1, v-1)][c]  (zero outside).
+ *
+ *   x, w_dw, b_dw, w_pw : as given to rib_cla_gate (device)
+ *   gate       : bf16 [B][H][W][C], G from rib_cla_gate
+ *   out        : bf16 [B][H][W][C], the ungated attention output O
+ *   dout_gated : bf16 [B][H][W][C], dO'
+ *   dout       : out, bf16 dO (pass it to rib_window_attn_bwd as its dout)
+ *   dx         : out, bf16 [B][H][W][C], the CLA path's share of dL/dx
+ *   dw_dw, db_dw, dw_pw, db_pw : out, fp32, shapes of the weights
+ *   workspace  : device, >= rib_cla_bwd_workspace() bytes, 256-byte aligned
+ * The point-wise GEMMs run on the tensor cores with bf16 operands (dz, y,
+ * W_pw rounded) and fp32 accumulation; sums over pixels go through per-CTA
+ * partials added in a fixed order, so results are deterministic.  Same
+ * shape requirements and errors as rib_cla_gate; RIB_ERR_WORKSPACE for a
+ * missing or short workspace.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+size_t rib_cla_bwd_workspace(int B, int H, int W, int C);
+int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw,
+                const float* b_dw, const float* w_pw, const void* gate,
+                const void* out, const void* dout_gated, void* dout, void* dx,
+                float* dw_dw, float* db_dw, float* dw_pw, float* db_pw,
+                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace rib_window_attn_bwd needs for these sizes;
  * `mlp` (host pointer, may be NULL) adds the MLP-gradient scratch. */
 size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads,

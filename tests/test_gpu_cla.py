@@ -7,7 +7,7 @@ import torch
 import oracle as O
 import rib_inputs as I
 import windowed_attention_implicit_b200 as R
-from tests.rib_testlib import Case, assert_close, to_np
+from tests.rib_testlib import Case, assert_all, assert_close, check_close, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -84,3 +84,48 @@ def test_cla_gate_rejects_bad_shapes():
     cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
     with pytest.raises(R.RibError):
         R.rib_cla_gate(x, cla)                      # C > 192: no room for the buffers
+
+
+def _cla_bwd_case(B, H, W, C, seed):
+    x, p, cla = _gate(B, H, W, C, seed)
+    o = I.make_features(B, H, W, C, seed + 100)          # an ungated output O
+    dout_g = I.make_features(B, H, W, C, seed + 200)     # dO'
+    xd = x.cuda()
+    gate = R.rib_cla_gate(xd, cla)
+    g = R.rib_cla_bwd(xd, cla, gate, o.cuda(), dout_g.cuda())
+    torch.cuda.synchronize()
+    assert R.rib_last_status()[0] == 0
+    ref = O.cla_backward(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw, o, dout_g)
+    # dO = dO' * G has the magnitude of the upstream gradient (up to ~5 for
+    # N(0,1) draws over 28 M elements), where one bf16 half-ulp is 0.016:
+    # judged, like the sums below, on max(1, max|ref|)
+    checks = [check_close(to_np(g["dout"]), ref["d_o"], "dO", normalize=True),
+              check_close(to_np(g["dx"]), ref["dx"], "dx")]
+    # sums over every pixel: judged on their magnitude (bf16 operands)
+    for k in ("dw_pw", "db_pw", "dw_dw", "db_dw"):
+        checks.append(check_close(to_np(g[k]), ref[k], k, normalize=True))
+    assert_all(checks)
+    return g
+
+
+@pytest.mark.parametrize("B,H,W,C", [
+    (1, 8, 16, 32),       # one tile, every pixel at the border
+    (1, 16, 32, 96),      # three heads, a partial 64-channel group
+    (2, 32, 48, 192),     # six heads (two point-wise accumulators), several tiles
+])
+def test_cla_bwd_parity(B, H, W, C):
+    _cla_bwd_case(B, H, W, C, seed=C + 7)
+
+
+def test_cla_bwd_full_size_and_deterministic():
+    """The w96train map (1152 tiles, every CTA of the persistent grids), and
+    bit-identical weight gradients on a second call (fixed-order sums)."""
+    g1 = _cla_bwd_case(4, 192, 192, 192, seed=3)
+    x, p, cla = _gate(4, 192, 192, 192, 3)
+    o = I.make_features(4, 192, 192, 192, 103).cuda()
+    dout_g = I.make_features(4, 192, 192, 192, 203).cuda()
+    xd = x.cuda()
+    g2 = R.rib_cla_bwd(xd, cla, R.rib_cla_gate(xd, cla), o, dout_g)
+    torch.cuda.synchronize()
+    for k in ("dw_pw", "db_pw", "dw_dw", "db_dw", "dx", "dout"):
+        assert torch.equal(g1[k], g2[k]), k

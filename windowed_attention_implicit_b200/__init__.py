@@ -29,7 +29,7 @@ __all__ = [
     "rib_window_gather", "rib_window_scatter", "rib_last_status", "rib_status_string",
     "rib_set_wait_limit_ns", "rib_debug_wait_timeout", "rib_version", "library",
     "rib_trace_enable", "rib_trace_collect", "rib_debug_exp2", "ClaGate", "rib_cla_gate",
-    "rib_window_attn_fwd_cla",
+    "rib_window_attn_fwd_cla", "rib_cla_bwd", "rib_cla_bwd_workspace",
 ]
 
 
@@ -271,6 +271,36 @@ def rib_window_attn_fwd_cla(qkv: torch.Tensor, window: int, shift: int, gate: to
         _ptr(out, torch.bfloat16, "out"), _ptr(out_gated, torch.bfloat16, "out_gated"),
         _ptr(lse, torch.float32, "lse"), _stream(stream)), "rib_window_attn_fwd_cla")
     return out, out_gated, lse
+
+
+def rib_cla_bwd_workspace(B: int, H: int, W: int, C: int) -> int:
+    return int(library().rib_cla_bwd_workspace(B, H, W, C))
+
+
+def rib_cla_bwd(x: torch.Tensor, cla: ClaGate, gate: torch.Tensor, out: torch.Tensor,
+                dout_gated: torch.Tensor, dout=None, dx=None, workspace=None, stream=None):
+    """Backward of O' = O * gate: returns dict(dout = dO' * G (the attention
+    backward's input), dx, dw_dw, db_dw, dw_pw, db_pw).  out / dout_gated may be
+    [B][H][W][heads][d] or [B][H][W][C]."""
+    B, H, W, C = x.shape
+    dev = x.device
+    dout = torch.empty(out.shape, device=dev, dtype=torch.bfloat16) if dout is None else dout
+    dx = torch.empty_like(x) if dx is None else dx
+    g = {k: torch.empty_like(getattr(cla, k.replace("d", "", 1)))
+         for k in ("dw_dw", "db_dw", "dw_pw", "db_pw")}
+    need = rib_cla_bwd_workspace(B, H, W, C)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
+    bf, f32 = torch.bfloat16, torch.float32
+    _check(library().rib_cla_bwd(
+        _ptr(x, bf, "x"), B, H, W, C, _ptr(cla.w_dw, f32, "w_dw"), _ptr(cla.b_dw, f32, "b_dw"),
+        _ptr(cla.w_pw, f32, "w_pw"), _ptr(gate, bf, "gate"), _ptr(out, bf, "out"),
+        _ptr(dout_gated, bf, "dout_gated"), _ptr(dout, bf, "dout"), _ptr(dx, bf, "dx"),
+        _ptr(g["dw_dw"], f32, "dw_dw"), _ptr(g["db_dw"], f32, "db_dw"),
+        _ptr(g["dw_pw"], f32, "dw_pw"), _ptr(g["db_pw"], f32, "db_pw"),
+        _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "rib_cla_bwd")
+    return dict(dout=dout, dx=dx, **g)
 
 
 def rib_window_attn_bwd_workspace(B, H, W, heads, head_dim, window, rank,

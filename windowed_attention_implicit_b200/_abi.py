@@ -53,6 +53,9 @@ _SIGS = {
     "rib_window_attn_fwd_cla": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
                                      ctypes.c_float, _p, _p, _p, _p, _p]),
     "rib_cla_gate": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]),
+    "rib_cla_bwd_workspace": (ctypes.c_size_t, [_i, _i, _i, _i]),
+    "rib_cla_bwd": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                         _p, ctypes.c_size_t, _p]),
     "rib_window_attn_bwd_workspace": (ctypes.c_size_t,
                                       [_i, _i, _i, _i, _i, _i, _i,
                                        ctypes.POINTER(rib_mlp_t)]),

@@ -22,6 +22,7 @@
 #include "attn_fwd.cuh"
 #include "attn_bwd.cuh"
 #include "cla.cuh"
+#include "cla_bwd.cuh"
 
 namespace rib {
 namespace {
@@ -114,13 +115,14 @@ int map_pixel_f32(CUtensorMap* m, const void* base, int B, int heads, int H, int
 // ---------------------------------------------------------------- tracing
 enum KernelId {
   K_POS, K_FWD, K_BWD_PRE, K_BWD, K_DQ_FIN, K_POSGRAD, K_MLP_PART, K_MLP_RED, K_COPY, K_DEBUG,
-  K_CLA, K_COUNT
+  K_CLA, K_CLA_DZ, K_CLA_DWPW, K_CLA_DX, K_CLA_RED, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "pos_tokens_kernel",   "attn_fwd_kernel",        "bwd_preprocess_kernel",
     "attn_bwd_kernel",     "dq_finalize_kernel",     "posgrad_reduce_kernel",
     "mlp_bwd_partial_kernel", "mlp_bwd_reduce_kernel", "window_copy_kernel",
-    "debug_wait_kernel",   "cla_gate_kernel"};
+    "debug_wait_kernel",   "cla_gate_kernel",        "cla_bwd_dz_kernel",
+    "cla_bwd_dwpw_kernel", "cla_bwd_dx_kernel",      "cla_bwd_reduce_kernel"};
 
 struct TraceRec {
   int id;
@@ -334,6 +336,44 @@ __global__ void debug_exp2_kernel(const float* x, float* y, int n_pairs) {
   const uint64_t r = exp2_fma2(pk2(x[2 * i], x[2 * i + 1]));
   y[2 * i] = lo2(r);
   y[2 * i + 1] = hi2(r);
+}
+
+struct ClaBwdLayout {
+  size_t dz, dy, part_dbpw, part_dwpw, part_dw, total;
+  int grid, n_tiles;
+};
+
+int cla_check(int B, int H, int W, int C) {
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
+  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u) return RIB_ERR_UNSUPPORTED;
+  if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
+  if ((long long)B * H * W * C > (1ll << 40) || B > (1 << 20)) return RIB_ERR_UNSUPPORTED;
+  if ((long long)B * (H / 8) * (W / 16) > (1ll << 30)) return RIB_ERR_UNSUPPORTED;
+  return RIB_OK;
+}
+
+// At most 1024 CTAs (the partial sums are sized for the launch grid).
+ClaBwdLayout cla_bwd_layout(int B, int H, int W, int C, int sms) {
+  ClaBwdLayout L;
+  L.n_tiles = B * (H / 8) * (W / 16);
+  L.grid = std::min(std::min(L.n_tiles, sms), 1024);
+  const size_t P = (size_t)B * H * W;
+  size_t off = 0;
+  L.dz = off; off = align256(off + P * C * 2);
+  L.dy = off; off = align256(off + P * C * 2);
+  L.part_dbpw = off; off = align256(off + (size_t)L.grid * C * 4);
+  L.part_dwpw = off; off = align256(off + (size_t)L.grid * C * C * 4);
+  L.part_dw = off; off = align256(off + (size_t)L.grid * 10 * C * 4);
+  L.total = off;
+  return L;
+}
+
+int device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return RIB_ERR_CUDA;
+  return RIB_OK;
 }
 
 }  // namespace
@@ -598,6 +638,78 @@ int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, c
   const int grid = static_cast<int>(n_tiles < sms ? n_tiles : sms);
   TraceScope ts(K_CLA, static_cast<cudaStream_t>(stream));
   cla_gate_kernel<<<grid, kClaThreads, smem, static_cast<cudaStream_t>(stream)>>>(tm, p);
+  return launch_status();
+}
+
+size_t rib_cla_bwd_workspace(int B, int H, int W, int C) {
+  int sms = 0;
+  if (cla_check(B, H, W, C) != RIB_OK || device_sms(&sms) != RIB_OK) return 0;
+  return cla_bwd_layout(B, H, W, C, sms).total;
+}
+
+int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, const float* b_dw,
+                const float* w_pw, const void* gate, const void* out, const void* dout_gated,
+                void* dout, void* dx, float* dw_dw, float* db_dw, float* dw_pw, float* db_pw,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !w_dw || !b_dw || !w_pw || !gate || !out || !dout_gated || !dout || !dx || !dw_dw ||
+      !db_dw || !dw_pw || !db_pw)
+    return RIB_ERR_ARG;
+  int rc = cla_check(B, H, W, C);
+  if (rc) return rc;
+  const void* a16[] = {x, gate, out, dout_gated, dout, dx, dw_pw};
+  for (const void* q : a16)
+    if (!aligned16(q)) return RIB_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(w_pw) & 7u) || (reinterpret_cast<uintptr_t>(w_dw) & 3u) ||
+      (reinterpret_cast<uintptr_t>(b_dw) & 3u) || (reinterpret_cast<uintptr_t>(dw_dw) & 3u) ||
+      (reinterpret_cast<uintptr_t>(db_dw) & 3u) || (reinterpret_cast<uintptr_t>(db_pw) & 3u))
+    return RIB_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = device_sms(&sms))) return rc;
+  const ClaBwdLayout L = cla_bwd_layout(B, H, W, C, sms);
+  if (!workspace || workspace_bytes < L.total) return RIB_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RIB_ERR_ALIGN;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  ClaBwdParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.w_dw = w_dw; p.b_dw = b_dw; p.w_pw = w_pw;
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.out = static_cast<const __nv_bfloat16*>(out);
+  p.dout_g = static_cast<const __nv_bfloat16*>(dout_gated);
+  p.dout = static_cast<__nv_bfloat16*>(dout);
+  p.dx = static_cast<__nv_bfloat16*>(dx);
+  p.dw_dw = dw_dw; p.db_dw = db_dw; p.dw_pw = dw_pw; p.db_pw = db_pw;
+  p.dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz);
+  p.dy = reinterpret_cast<__nv_bfloat16*>(ws + L.dy);
+  p.part_dbpw = reinterpret_cast<float*>(ws + L.part_dbpw);
+  p.part_dwpw = reinterpret_cast<float*>(ws + L.part_dwpw);
+  p.part_dw = reinterpret_cast<float*>(ws + L.part_dw);
+  p.B = B; p.H = H; p.W = W; p.C = C;
+  p.tiles_x = W / 16;
+  p.tiles_per_img = (H / 8) * (W / 16);
+  p.n_tiles = L.n_tiles;
+  p.grid = L.grid;
+  p.wait_limit_ns = g_wait_limit_ns;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem_dz = cla_dz_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
+  if ((rc = set_smem(cla_bwd_dz_kernel, smem_dz))) return rc;
+  if ((rc = set_smem(cla_bwd_dwpw_kernel, smem_dw))) return rc;
+  {
+    TraceScope ts(K_CLA_DZ, st);
+    cla_bwd_dz_kernel<<<L.grid, kClaBwdThreads, smem_dz, st>>>(p);
+    if ((rc = launch_status())) return rc;
+  }
+  {
+    TraceScope ts(K_CLA_DWPW, st);
+    cla_bwd_dwpw_kernel<<<L.grid, kClaBwdThreads, smem_dw, st>>>(p);
+    if ((rc = launch_status())) return rc;
+  }
+  {
+    TraceScope ts(K_CLA_DX, st);
+    cla_bwd_dx_kernel<<<L.grid, kClaBwdThreads, 0, st>>>(p);
+    if ((rc = launch_status())) return rc;
+  }
+  TraceScope ts(K_CLA_RED, st);
+  cla_bwd_reduce_kernel<<<(C * C + 11 * C + 255) / 256, 256, 0, st>>>(p);
   return launch_status();
 }
 
