@@ -156,7 +156,8 @@ def stored_traffic(kernel, workload):
     return d.get("dram_bytes_per_launch")
 
 
-def cla_line(w, kern_g, ms_gate_total, ms_fwd_cla_total, ms_fwd, pk):
+def cla_line(w, kern_g, ms_gate_total, ms_fwd_cla_total, ms_fwd, pk, ms_cla_step_total,
+             kern_cs, ms_step):
     """Convolutional local attention (measured beside the hot path, not part
     of its step): the gate kernel against the HBM roofline (x read + G
     written, 2 bytes each per pixel and channel) and the extra cost of
@@ -167,9 +168,13 @@ def cla_line(w, kern_g, ms_gate_total, ms_fwd_cla_total, ms_fwd, pk):
     byt = 2 * w.batch * w.height * w.width * C * 2
     gbs = byt / (ms_g * 1e-3) / 1e9
     fwd_cla = ms_fwd_cla_total / steps
+    step = ms_cla_step_total / steps
+    bwd_k = {k: v[1] / v[0] for k, v in kern_cs.items() if k.startswith("cla_bwd")}
     return {"gate_kernel_ms": ms_g, "gate_bytes": byt, "gate_gbs": gbs,
             "gate_frac_hbm": gbs / pk["hbm_gbs"], "fwd_cla_ms": fwd_cla,
             "fwd_cla_extra_ms": fwd_cla - ms_fwd, "bound": "hbm",
+            "training_step_with_cla_ms": step, "cla_extra_ms_per_step": step - ms_step,
+            "cla_bwd_kernels_ms": bwd_k,
             "workload": f"x, G bf16 [{w.batch}][{w.height}][{w.width}][{C}]"}
 
 
@@ -316,6 +321,20 @@ def run_rib(args, w):
     def cla_gate_only():
         R.rib_cla_gate(feat, cla, gate=gate)
 
+    # a training step with the gate: the upstream gradient is that of O' = O * G
+    d_att = torch.empty_like(dout)
+    dfeat = torch.empty_like(feat)
+    cla_ws = torch.empty(R.rib_cla_bwd_workspace(B, H, W, heads * d), device=dev,
+                         dtype=torch.uint8)
+
+    def cla_step():
+        R.rib_pos_tokens(mlp, M, qp, kp, q16, k16)
+        R.rib_cla_gate(feat, cla, gate=gate)
+        R.rib_window_attn_fwd_cla(qkv, M, s, gate, q16, k16, out=out, out_gated=out_g, lse=lse)
+        R.rib_cla_bwd(feat, cla, gate, out, dout, dout=d_att, dx=dfeat, workspace=cla_ws)
+        R.rib_window_attn_bwd(qkv, out, d_att, lse, M, s, q16, k16, mlp=mlp, dqkv=dqkv,
+                              dqp=dqp, dkp=dkp, dmlp=dmlp, workspace=ws)
+
     def fwd_cla():
         R.rib_window_attn_fwd_cla(qkv, M, s, gate, q16, k16, out=out, out_gated=out_g, lse=lse)
 
@@ -348,18 +367,24 @@ def run_rib(args, w):
     if sampler:
         sampler.start()       # samples cover warm-up and every timed loop below
     if args.cla_only:
+        def cla_bwd_only():
+            R.rib_cla_bwd(feat, cla, gate, out, dout, dout=d_att, dx=dfeat, workspace=cla_ws)
+
         for _ in range(args.warmup):
             cla_gate_only()
             fwd_cla()
+            cla_bwd_only()
         ms_g, _, _ = timed(cla_gate_only, args.steps)
         ms_c, _, _ = timed(fwd_cla, args.steps)
+        ms_b, _, _ = timed(cla_bwd_only, args.steps)
         if sampler:
             sampler.stop()
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
             print(json.dumps({"cla_only": True, "cla_gate_ms": ms_g / args.steps,
-                              "fwd_cla_ms": ms_c / args.steps}))
+                              "fwd_cla_ms": ms_c / args.steps,
+                              "cla_bwd_ms": ms_b / args.steps}))
         return 0
     for _ in range(args.warmup):
         step()
@@ -393,6 +418,9 @@ def run_rib(args, w):
         fwd_cla()
     ms_g, kern_g, _ = timed(cla_gate_only, args.steps, trace=True)
     ms_c, _, _ = timed(fwd_cla, args.steps)
+    for _ in range(args.warmup):
+        cla_step()
+    ms_cs, kern_cs, _ = timed(cla_step, args.steps, trace=True)
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
@@ -471,7 +499,7 @@ def run_rib(args, w):
                 "tokens_per_s": world * w.tokens() / (ms_fwd * 1e-3),
                 "kernel_tflops": fwd_ach, "kernel_frac": fwd_ach / peak},
         "roofline": roof,
-        "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk),
+        "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk, ms_cs, kern_cs, ms_step),
         "kernels": per_kernel,
         "gpu_launches": launches,
         "cpu_baseline": cpu,

@@ -27,7 +27,8 @@
 
 namespace rib {
 
-constexpr int kClaBwdThreads = 256;
+constexpr int kClaBwdThreads = 512;   // dz and dW_pw kernels
+constexpr int kClaDxThreads = 256;
 
 struct ClaBwdParams {
   const __nv_bfloat16* x;
@@ -44,8 +45,8 @@ struct ClaBwdParams {
   __nv_bfloat16* dy;               // workspace [P][C]
   float* part_dbpw;                // [grid][C]
   float* part_dwpw;                // [grid][C][C]
-  float* part_dw;                  // [grid][10][C]  (9 taps, then the bias)
-  int B, H, W, C, tiles_x, tiles_per_img, n_tiles, grid;
+  float* part_dw;                  // [grid_dx][10][C]  (9 taps, then the bias)
+  int B, H, W, C, tiles_x, tiles_per_img, n_tiles, grid, grid_dx;
   uint64_t wait_limit_ns;
 };
 
@@ -61,7 +62,7 @@ __device__ __forceinline__ size_t cla_pix(const ClaBwdParams& p, int b, int i, i
 }
 
 __host__ __device__ __forceinline__ size_t cla_dz_smem_bytes(int C) {
-  return 2ull * C * C + 256ull * C + 32ull * C + 64 + 1024;
+  return 2ull * C * C + 256ull * C + 4ull * (kClaBwdThreads / 32) * C + 64 + 1024;
 }
 
 // -------------------------------------------------------------- dz and dy
@@ -72,8 +73,8 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   const int C = p.C;
   uint8_t* sB = base;                                   // W_pw^T bf16 [N = c][K = o]
   uint8_t* sA = base + 2ull * C * C;                    // dz bf16 [M = 128 pixels][K = o]
-  float* red = reinterpret_cast<float*>(sA + 256ull * C);   // [8 warps][C]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 8 * C);
+  float* red = reinterpret_cast<float*>(sA + 256ull * C);   // [warps][C]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + (kClaBwdThreads / 32) * C);
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -144,11 +145,12 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
     ok = __syncthreads_and(ok);
     tc_fence_after();
     if (ok) {
-      const int q = warp & 3, half = warp >> 2;
+      // warp w reads TMEM lanes 32 (w % 4).. (pixels), columns 32 (w / 4) + 32 k (warps / 4)
+      const int q = warp & 3, slot = warp >> 2;
       const int r = q * 32 + lane;
       __nv_bfloat16* dst = p.dy + cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 32 * half; c0 < C; c0 += 64) {
+      for (int c0 = 32 * slot; c0 < C; c0 += 32 * (kClaBwdThreads / 128)) {
         uint32_t v[32];
         tmem_ld_x32(taddr + c0, v);
         tmem_wait_ld();
@@ -314,7 +316,7 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
     mbar_wait(bar, phase ^ 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
   }
   // the CTA's partial dW_pw: rows o from TMEM lanes, C columns each
-  if (ok) {
+  if (ok && warp < 8) {
     const int q = warp & 3, half = warp >> 2;
     const int o = half * 128 + q * 32 + lane;
     const uint32_t taddr = tmem + half * 256 + (static_cast<uint32_t>(q * 32) << 16);
@@ -346,11 +348,11 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
 }
 
 // -------------------------------------------------------------- dx, dW_dw, db_dw
-// grid p.grid, block kClaBwdThreads, static smem.  Lanes along channel
+// grid p.grid_dx, block kClaDxThreads, static smem.  Lanes along channel
 // pairs, warps over the tile's pixels; one 64-channel group at a time over
 // all of the CTA's tiles, so each thread keeps 20 partial sums.
-__global__ void __launch_bounds__(kClaBwdThreads) cla_bwd_dx_kernel(const ClaBwdParams p) {
-  __shared__ float red[kClaBwdThreads / 32][10][64];
+__global__ void __launch_bounds__(kClaDxThreads) cla_bwd_dx_kernel(const ClaBwdParams p) {
+  __shared__ float red[kClaDxThreads / 32][10][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.C;
   for (int g = 0; g * 64 < C; ++g) {
@@ -366,7 +368,7 @@ __global__ void __launch_bounds__(kClaBwdThreads) cla_bwd_dx_kernel(const ClaBwd
     for (int t = blockIdx.x; act && t < p.n_tiles; t += gridDim.x) {
       int b, i0, j0;
       cla_tile(p, t, b, i0, j0);
-      for (int r = warp; r < 128; r += kClaBwdThreads / 32) {
+      for (int r = warp; r < 128; r += kClaDxThreads / 32) {
         const int i = i0 + (r >> 4), j = j0 + (r & 15);
         const float2 d = __bfloat1622float2(
             *reinterpret_cast<const __nv_bfloat162*>(p.dy + cla_pix(p, b, i, j) * C + c));
@@ -411,7 +413,7 @@ __global__ void __launch_bounds__(kClaBwdThreads) cla_bwd_dx_kernel(const ClaBwd
       const int tp = e / 64, cc = e % 64;
       if (g * 64 + cc >= C) continue;
       float s = 0.f;
-      for (int w = 0; w < kClaBwdThreads / 32; ++w) s += red[w][tp][cc];
+      for (int w = 0; w < kClaDxThreads / 32; ++w) s += red[w][tp][cc];
       p.part_dw[(static_cast<size_t>(blockIdx.x) * 10 + tp) * C + g * 64 + cc] = s;
     }
     __syncthreads();
@@ -437,7 +439,7 @@ __global__ void __launch_bounds__(256) cla_bwd_reduce_kernel(const ClaBwdParams 
   } else {
     const int e = idx - n_pw - C;           // 0 .. 10C-1: tap-major [10][C]
     const int tp = e / C, c = e % C;
-    for (int k = 0; k < p.grid; ++k) s += p.part_dw[(static_cast<size_t>(k) * 10 + tp) * C + c];
+    for (int k = 0; k < p.grid_dx; ++k) s += p.part_dw[(static_cast<size_t>(k) * 10 + tp) * C + c];
     if (tp < 9) p.dw_dw[c * 9 + tp] = s;
     else p.db_dw[c] = s;
   }

@@ -340,7 +340,7 @@ __global__ void debug_exp2_kernel(const float* x, float* y, int n_pairs) {
 
 struct ClaBwdLayout {
   size_t dz, dy, part_dbpw, part_dwpw, part_dw, total;
-  int grid, n_tiles;
+  int grid, grid_dx, n_tiles;
 };
 
 int cla_check(int B, int H, int W, int C) {
@@ -352,18 +352,20 @@ int cla_check(int B, int H, int W, int C) {
   return RIB_OK;
 }
 
-// At most 1024 CTAs (the partial sums are sized for the launch grid).
+// The partial sums are sized for the launch grids: one CTA per SM for the
+// two tensor-core kernels, up to eight per SM for the dx kernel.
 ClaBwdLayout cla_bwd_layout(int B, int H, int W, int C, int sms) {
   ClaBwdLayout L;
   L.n_tiles = B * (H / 8) * (W / 16);
   L.grid = std::min(std::min(L.n_tiles, sms), 1024);
+  L.grid_dx = std::min(std::min(L.n_tiles, 8 * sms), 8192);
   const size_t P = (size_t)B * H * W;
   size_t off = 0;
   L.dz = off; off = align256(off + P * C * 2);
   L.dy = off; off = align256(off + P * C * 2);
   L.part_dbpw = off; off = align256(off + (size_t)L.grid * C * 4);
   L.part_dwpw = off; off = align256(off + (size_t)L.grid * C * C * 4);
-  L.part_dw = off; off = align256(off + (size_t)L.grid * 10 * C * 4);
+  L.part_dw = off; off = align256(off + (size_t)L.grid_dx * 10 * C * 4);
   L.total = off;
   return L;
 }
@@ -688,6 +690,7 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   p.tiles_per_img = (H / 8) * (W / 16);
   p.n_tiles = L.n_tiles;
   p.grid = L.grid;
+  p.grid_dx = L.grid_dx;
   p.wait_limit_ns = g_wait_limit_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t smem_dz = cla_dz_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
@@ -705,7 +708,7 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   }
   {
     TraceScope ts(K_CLA_DX, st);
-    cla_bwd_dx_kernel<<<L.grid, kClaBwdThreads, 0, st>>>(p);
+    cla_bwd_dx_kernel<<<L.grid_dx, kClaDxThreads, 0, st>>>(p);
     if ((rc = launch_status())) return rc;
   }
   TraceScope ts(K_CLA_RED, st);
