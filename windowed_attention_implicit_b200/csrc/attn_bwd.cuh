@@ -74,10 +74,11 @@ constexpr uint32_t kBwdTmemCols = 512;
 constexpr uint32_t kBColS = 0, kBColDP = 128, kBColP = 256, kBColDST = 320, kBColDV = 384,
                    kBColDK = 416, kBColDQ = 464;
 // Of every 8 element pairs, how many exponentials run on the FMA pipe.  The
-// backward is issue-bound rather than MUFU-bound (its MMA work per score is
-// 2.6x the forward's), so by default every exponential stays on MUFU.
+// backward's exponential phase runs at about the MUFU rate with two compute
+// warps per scheduler; moving one pair in eight to the FMA pipe measured
+// ~1 % faster on the 96x96 training workload, two or three pairs slower.
 #ifndef RIB_BWD_POLY_PAIRS
-#define RIB_BWD_POLY_PAIRS 0
+#define RIB_BWD_POLY_PAIRS 1
 #endif
 constexpr int kBwdPolyPairs = RIB_BWD_POLY_PAIRS;
 constexpr uint64_t kBwdDrainNs = 200ull * 1000ull * 1000ull;
