@@ -129,3 +129,34 @@ def test_cla_bwd_full_size_and_deterministic():
     torch.cuda.synchronize()
     for k in ("dw_pw", "db_pw", "dw_dw", "db_dw", "dx", "dout"):
         assert torch.equal(g1[k], g2[k]), k
+
+
+def test_training_layer_with_cla_matches_oracle_composition():
+    """One training layer through the library's composed path, gate ->
+    gated forward -> CLA backward -> attention backward (fed the CLA
+    backward's dO), against the same composition of fp64 oracle functions."""
+    c = Case(1, 64, 64, 2, 32, 16, seed=21)
+    C = c.heads * 32
+    x, p, cla = _gate(c.B, c.H, c.W, C, seed=9)
+    dout_g = I.make_features(c.B, c.H, c.W, C, 909)          # dO' of the gated output
+    d = c.device()
+    xd = x.cuda()
+    gate = R.rib_cla_gate(xd, cla)
+    out, out_g, lse = R.rib_window_attn_fwd_cla(d["qkv"], c.M, c.s, gate, d["qp16"], d["kp16"])
+    g = R.rib_cla_bwd(xd, cla, gate, out, dout_g.cuda())
+    ga = R.rib_window_attn_bwd(d["qkv"], out, g["dout"], lse, c.M, c.s, d["qp16"], d["kp16"])
+    torch.cuda.synchronize()
+    assert R.rib_last_status()[0] == 0
+    ro, _ = c.oracle_fwd()
+    rg = O.cla_gate(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    rc = O.cla_backward(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw, ro, dout_g)
+    d_o = rc["d_o"].reshape(c.B, c.H, c.W, c.heads, 32)
+    rdq, rdqp, rdkp = O.attn_bwd(c.qkv, d_o, c.M, c.s, c.qp16, c.kp16, c.scale)
+    checks = [check_close(to_np(out_g), O.cla_apply(ro, rg), "gated output"),
+              check_close(to_np(g["dx"]), rc["dx"], "dx"),
+              check_close(to_np(ga["dqkv"]), rdq, "dqkv"),
+              check_close(to_np(ga["dqp"]), rdqp, "dqp", normalize=True),
+              check_close(to_np(ga["dkp"]), rdkp, "dkp", normalize=True)]
+    for k in ("dw_pw", "db_pw", "dw_dw", "db_dw"):
+        checks.append(check_close(to_np(g[k]), rc[k], k, normalize=True))
+    assert_all(checks)

@@ -10,7 +10,7 @@
 //   db_dw = sum_pixels dy,            dW_dw[c][u][v] = sum_pixels dy[p][c] x[p + (u-1, v-1)][c]
 //   dx[p][c] = sum_{u,v} W_dw[c][u][v] dy[p - (u-1, v-1)][c]   (zero outside the map)
 //
-// Kernels, in launch order (all persistent, one CTA per SM at most, tiles of
+// Kernels, in launch order (persistent grids, tiles of
 // 8 x 16 pixels; sums over pixels go through per-CTA partials and a
 // fixed-order reduction, so the weight gradients are deterministic):
 //   cla_bwd_dz_kernel    dO, dz (to the workspace), db_pw partials, and
@@ -19,7 +19,7 @@
 //   cla_bwd_dwpw_kernel  dW_pw partials = sum over the CTA's tiles of
 //                        dz^T y, y recomputed from x; both operands MN-major
 //                        in shared memory, the C x C partial in TMEM
-//   cla_bwd_dx_kernel    dx, and dW_dw / db_dw partials (FMA pipe)
+//   cla_bwd_dx_kernel    dx, and dW_dw / db_dw partials (FMA pipe, two CTAs per SM)
 //   cla_bwd_reduce_kernel fixed-order sums of the partials
 #pragma once
 

@@ -353,12 +353,13 @@ int cla_check(int B, int H, int W, int C) {
 }
 
 // The partial sums are sized for the launch grids: one CTA per SM for the
-// two tensor-core kernels, up to eight per SM for the dx kernel.
+// two tensor-core kernels, two per SM for the dx kernel (its registers allow
+// two or three; more CTAs would only lengthen the reduction's sums).
 ClaBwdLayout cla_bwd_layout(int B, int H, int W, int C, int sms) {
   ClaBwdLayout L;
   L.n_tiles = B * (H / 8) * (W / 16);
   L.grid = std::min(std::min(L.n_tiles, sms), 1024);
-  L.grid_dx = std::min(std::min(L.n_tiles, 8 * sms), 8192);
+  L.grid_dx = std::min(std::min(L.n_tiles, 2 * sms), 2048);
   const size_t P = (size_t)B * H * W;
   size_t off = 0;
   L.dz = off; off = align256(off + P * C * 2);
