@@ -92,7 +92,7 @@ typedef struct {
  * layer with this M and these weights.
  *
  *   mlp      : host pointer to the weight struct (device weight pointers)
- *   window   : M, 1 <= M <= 128
+ *   window   : M, 1 <= M <= 256
  *   qp, kp   : out, fp32 [heads][M][M][rank]
  *   qp_bf16, kp_bf16 : out, bf16 copies of the same shape (may be NULL)
  * Computes in fp32 (coordinate Fourier features in fp64, rounded to fp32).
@@ -163,7 +163,9 @@ int rib_pos_tokens_bwd_noalloc(const rib_mlp_t* mlp, int window, const float* dq
  *   scale    : softmax scale; <= 0 selects 1/sqrt(head_dim + rank)
  *   out      : bf16 [B][H][W][heads][head_dim]
  *   lse      : fp32 [B][heads][H][W] (natural log), needed by the backward
- * Supported: head_dim == 32, M % 16 == 0, 16 <= M <= 128, s % 8 == 0.
+ * Supported: head_dim == 32, M % 16 == 0, 16 <= M <= 256, s % 8 == 0.
+ * B == 0 (an empty batch) is valid: nothing is read, written or launched,
+ * and the pointers are not looked at.
  * ------------------------------------------------------------------------ */
 int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads,
                         int head_dim, int window, int shift,
@@ -187,7 +189,8 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads,
  *   gate   : out, bf16 [B][H][W][C]                      (device)
  * The point-wise convolution runs on the tensor cores with y and w_pw
  * rounded to bf16 (fp32 accumulation).  Requires C % 32 == 0, C <= 192,
- * H % 8 == 0, W % 16 == 0 (else RIB_ERR_UNSUPPORTED / RIB_ERR_SHAPE); x and
+ * H % 8 == 0, W % 16 == 0 (else RIB_ERR_UNSUPPORTED / RIB_ERR_SHAPE); B == 0
+ * is a valid no-op (pointers not looked at); x and
  * gate 16-byte aligned, w_pw 8-byte aligned (RIB_ERR_ALIGN).  Asynchronous
  * on `stream`; allocates nothing.
  * ------------------------------------------------------------------------ */
@@ -235,7 +238,8 @@ int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads,
  * W_pw rounded) and fp32 accumulation; sums over pixels go through per-CTA
  * partials added in a fixed order, so results are deterministic.  Same
  * shape requirements and errors as rib_cla_gate; RIB_ERR_WORKSPACE for a
- * missing or short workspace.  Asynchronous on `stream`.
+ * missing or short workspace.  B == 0 zeroes the four weight gradients and
+ * touches nothing else.  Asynchronous on `stream`.
  * ------------------------------------------------------------------------ */
 size_t rib_cla_bwd_workspace(int B, int H, int W, int C);
 int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw,
@@ -270,6 +274,8 @@ size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads,
  *   dmlp     : host pointer to device gradient buffers (may be NULL)
  *   workspace: device scratch of at least rib_window_attn_bwd_workspace()
  *              bytes, 256-byte aligned; contents need not be initialised
+ * B == 0 is valid: dqp, dkp and the MLP gradients (when requested) are
+ * zeroed, being sums over no windows, and nothing else is touched.
  * dQ partials of the key tiles are summed with fp32 reduce-adds in no fixed
  * order, so dqkv's query part and dqp may differ in the last bits between
  * runs.

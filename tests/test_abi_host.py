@@ -56,8 +56,9 @@ def fwd(**kw):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(qkv=None), _abi.RIB_ERR_ARG),
-    (dict(B=0), _abi.RIB_ERR_ARG),
+    (dict(B=-1), _abi.RIB_ERR_ARG),
     (dict(H=0), _abi.RIB_ERR_ARG),
+    (dict(B=0, H=72), _abi.RIB_ERR_SHAPE),           # an empty batch is still shape-checked
     (dict(H=72), _abi.RIB_ERR_SHAPE),
     (dict(W=40), _abi.RIB_ERR_SHAPE),
     (dict(s=16), _abi.RIB_ERR_SHAPE),
@@ -72,6 +73,17 @@ def fwd(**kw):
 ])
 def test_fwd_validation(kw, code):
     assert fwd(**kw) == code
+
+
+def test_empty_batch_is_a_no_op():
+    # B = 0: valid shapes return RIB_OK before any pointer is looked at or
+    # anything is launched (empty tensors may have null data pointers)
+    assert fwd(B=0, qkv=None, out=None, lse=None, qp=None, kp=None) == _abi.RIB_OK
+    lib = R.library()
+    assert lib.rib_window_gather(None, 0, 64, 64, 96, 2, 16, 8, None, None) == _abi.RIB_OK
+    assert lib.rib_window_scatter(None, 0, 64, 64, 96, 2, 16, 8, None, None) == _abi.RIB_OK
+    assert lib.rib_cla_gate(None, 0, 16, 32, 96, FAKE, FAKE, FAKE, FAKE, None, None) == _abi.RIB_OK
+    assert lib.rib_cla_gate(None, -1, 16, 32, 96, FAKE, FAKE, FAKE, FAKE, None, None) == _abi.RIB_ERR_ARG
 
 
 def test_fwd_rank0_needs_no_position_tokens():

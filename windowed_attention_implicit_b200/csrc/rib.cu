@@ -186,7 +186,7 @@ struct AttnGeom {
 // Shape checks shared by forward and backward.
 int check_attn(int B, int H, int W, int heads, int head_dim, int M, int shift, int rank,
                AttnGeom* g) {
-  if (B <= 0 || H <= 0 || W <= 0 || heads <= 0 || M <= 0) return RIB_ERR_ARG;
+  if (B < 0 || H <= 0 || W <= 0 || heads <= 0 || M <= 0) return RIB_ERR_ARG;
   if (H % M != 0 || W % M != 0 || shift < 0 || shift >= M) return RIB_ERR_SHAPE;
   if (head_dim != 32 || (rank != 0 && rank != 16)) return RIB_ERR_UNSUPPORTED;
   if (M % 16 != 0 || M > 256 || shift % 8 != 0) return RIB_ERR_UNSUPPORTED;
@@ -344,7 +344,7 @@ struct ClaBwdLayout {
 };
 
 int cla_check(int B, int H, int W, int C) {
-  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
+  if (B < 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
   if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u) return RIB_ERR_UNSUPPORTED;
   if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
   if ((long long)B * H * W * C > (1ll << 40) || B > (1 << 20)) return RIB_ERR_UNSUPPORTED;
@@ -539,12 +539,14 @@ static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int 
                            int window, int shift, const void* qp_bf16, const void* kp_bf16,
                            int rank, float scale, void* out, float* lse, const void* gate,
                            void* out_gated, void* stream) {
-  if (!qkv || !out || !lse) return RIB_ERR_ARG;
-  if ((gate == nullptr) != (out_gated == nullptr)) return RIB_ERR_ARG;
-  if (gate && (!aligned16(gate) || !aligned16(out_gated))) return RIB_ERR_ALIGN;
   AttnGeom g;
   int rc = check_attn(B, H, W, heads, head_dim, window, shift, rank, &g);
   if (rc) return rc;
+  if (!std::isfinite(scale)) return RIB_ERR_ARG;
+  if (B == 0) return RIB_OK;   // an empty batch: nothing to compute or write
+  if (!qkv || !out || !lse) return RIB_ERR_ARG;
+  if ((gate == nullptr) != (out_gated == nullptr)) return RIB_ERR_ARG;
+  if (gate && (!aligned16(gate) || !aligned16(out_gated))) return RIB_ERR_ALIGN;
   if (rank > 0 && (!qp_bf16 || !kp_bf16)) return RIB_ERR_ARG;
   if (!aligned16(qkv) || !aligned16(out) || !aligned16(lse) ||
       (rank > 0 && (!aligned16(qp_bf16) || !aligned16(kp_bf16))))
@@ -605,11 +607,10 @@ int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads, int
 
 int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, const float* b_dw,
                  const float* w_pw, const float* b_pw, void* gate, void* stream) {
+  int rc = cla_check(B, H, W, C);
+  if (rc) return rc;
+  if (B == 0) return RIB_OK;   // an empty batch: nothing to compute or write
   if (!x || !w_dw || !b_dw || !w_pw || !b_pw || !gate) return RIB_ERR_ARG;
-  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
-  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u) return RIB_ERR_UNSUPPORTED;
-  if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
-  if ((long long)B * H * W * C > (1ll << 40) || B > (1 << 20)) return RIB_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(gate) || (reinterpret_cast<uintptr_t>(w_pw) & 7u) ||
       (reinterpret_cast<uintptr_t>(w_dw) & 3u) || (reinterpret_cast<uintptr_t>(b_dw) & 3u) ||
       (reinterpret_cast<uintptr_t>(b_pw) & 3u))
@@ -619,7 +620,7 @@ int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, c
   const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)H, (uint64_t)B};
   const uint64_t strides[3] = {2ull * C, 2ull * C * W, 2ull * C * W * H};
   const uint32_t box[4] = {64, 18, 10, 1};
-  int rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, dims, strides, box,
+  rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, dims, strides, box,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
   ClaParams p{};
@@ -654,11 +655,21 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
                 const float* w_pw, const void* gate, const void* out, const void* dout_gated,
                 void* dout, void* dx, float* dw_dw, float* db_dw, float* dw_pw, float* db_pw,
                 void* workspace, size_t workspace_bytes, void* stream) {
-  if (!x || !w_dw || !b_dw || !w_pw || !gate || !out || !dout_gated || !dout || !dx || !dw_dw ||
-      !db_dw || !dw_pw || !db_pw)
-    return RIB_ERR_ARG;
   int rc = cla_check(B, H, W, C);
   if (rc) return rc;
+  if (!dw_dw || !db_dw || !dw_pw || !db_pw) return RIB_ERR_ARG;
+  if (B == 0) {
+    // an empty batch: the weight gradients are empty sums, zero
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(dw_dw, 0, 9ull * C * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(db_dw, 0, (size_t)C * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(dw_pw, 0, (size_t)C * C * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(db_pw, 0, (size_t)C * sizeof(float), st) != cudaSuccess)
+      return RIB_ERR_CUDA;
+    return RIB_OK;
+  }
+  if (!x || !w_dw || !b_dw || !w_pw || !gate || !out || !dout_gated || !dout || !dx)
+    return RIB_ERR_ARG;
   const void* a16[] = {x, gate, out, dout_gated, dout, dx, dw_pw};
   for (const void* q : a16)
     if (!aligned16(q)) return RIB_ERR_ALIGN;
@@ -731,12 +742,34 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
                         void* dqkv, float* dqp, float* dkp, const rib_mlp_t* mlp,
                         const rib_mlp_grad_t* dmlp, void* workspace, size_t workspace_bytes,
                         void* stream) {
-  if (!qkv || !out || !dout || !lse || !dqkv) return RIB_ERR_ARG;
   AttnGeom g;
   int rc = check_attn(B, H, W, heads, head_dim, window, shift, rank, &g);
   if (rc) return rc;
-  if (rank > 0 && (!qp_bf16 || !kp_bf16 || !dqp || !dkp)) return RIB_ERR_ARG;
   const bool do_mlp = mlp != nullptr && dmlp != nullptr && rank > 0;
+  if (B == 0) {
+    // an empty batch: the position-token gradients are empty sums, zero
+    if (rank > 0 && (!dqp || !dkp)) return RIB_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t pbytes = sizeof(float) * heads * g.N * rank;
+    if (rank > 0 && (cudaMemsetAsync(dqp, 0, pbytes, st) != cudaSuccess ||
+                     cudaMemsetAsync(dkp, 0, pbytes, st) != cudaSuccess))
+      return RIB_ERR_CUDA;
+    if (do_mlp) {
+      if ((rc = check_mlp(mlp))) return rc;
+      if (!mlp_grad_complete(dmlp)) return RIB_ERR_ARG;
+      const size_t din = 4ull * mlp->n_freq, hid = mlp->d_hidden,
+                   dout_n = (size_t)mlp->heads * mlp->rank;
+      float* const gp[8] = {dmlp->q_dw1, dmlp->q_db1, dmlp->q_dw2, dmlp->q_db2,
+                            dmlp->k_dw1, dmlp->k_db1, dmlp->k_dw2, dmlp->k_db2};
+      const size_t gn[4] = {hid * din, hid, dout_n * hid, dout_n};
+      for (int i = 0; i < 8; ++i)
+        if (cudaMemsetAsync(gp[i], 0, gn[i % 4] * sizeof(float), st) != cudaSuccess)
+          return RIB_ERR_CUDA;
+    }
+    return RIB_OK;
+  }
+  if (!qkv || !out || !dout || !lse || !dqkv) return RIB_ERR_ARG;
+  if (rank > 0 && (!qp_bf16 || !kp_bf16 || !dqp || !dkp)) return RIB_ERR_ARG;
   if (do_mlp) {
     if ((rc = check_mlp(mlp))) return rc;
     if (mlp->heads != heads || mlp->rank != rank) return RIB_ERR_ARG;
@@ -841,11 +874,12 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
 
 static int window_copy(const void* src, void* dst, int B, int H, int W, int C, int eb, int M,
                        int s, int gather, void* stream) {
-  if (!src || !dst) return RIB_ERR_ARG;
-  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || M <= 0) return RIB_ERR_ARG;
+  if (B < 0 || H <= 0 || W <= 0 || C <= 0 || M <= 0) return RIB_ERR_ARG;
   if (eb != 1 && eb != 2 && eb != 4) return RIB_ERR_ARG;
   if (H % M != 0 || W % M != 0 || s < 0 || s >= M) return RIB_ERR_SHAPE;
   if (M % 8 != 0 || s % 8 != 0 || ((long long)C * eb) % 16 != 0) return RIB_ERR_UNSUPPORTED;
+  if (B == 0) return RIB_OK;   // an empty batch: nothing to copy
+  if (!src || !dst) return RIB_ERR_ARG;
   if (!aligned16(src) || !aligned16(dst)) return RIB_ERR_ALIGN;
   const int nW = (H / M) * (W / M);
   if (nW > 65535 || B > 65535) return RIB_ERR_UNSUPPORTED;
