@@ -81,6 +81,10 @@ constexpr uint32_t kBColS = 0, kBColDP = 128, kBColP = 256, kBColDST = 320, kBCo
 #define RIB_BWD_POLY_PAIRS 1
 #endif
 constexpr int kBwdPolyPairs = RIB_BWD_POLY_PAIRS;
+#ifndef RIB_BWD_DK_SMEM
+#define RIB_BWD_DK_SMEM 1
+#endif
+constexpr bool kBwdDkSmem = RIB_BWD_DK_SMEM != 0;
 constexpr uint64_t kBwdDrainNs = 200ull * 1000ull * 1000ull;
 
 struct BwdParams {
@@ -106,7 +110,8 @@ struct __align__(1024) BwdSmem {
   float dd[kBwdStages][128];       // -D = -rowsum(dO * O), tile row order
   uint64_t k_full;
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
-  uint64_t s_full, s_free, ds_full, pt_free /* P^T and dS^T in TMEM */, ds_free[2];
+  // pt_free: P^T (and dS^T) in TMEM and the dS buffer written next are free
+  uint64_t s_full, s_free, ds_full, pt_free;
   uint64_t dq_full, dq_free, mma_done;
   int drain_ok[4];
   uint64_t drain;
@@ -256,9 +261,17 @@ __device__ __forceinline__ void bwd_mma_dq(BwdSmem& sm, uint32_t tmem, const Bwd
     const int st = i % kBwdStages;
     if (!(ok = warp_wait(&sm.ds_full, i & 1, ab, lim, SITE_BWD_MMA))) break;
     tc_fence_after();
-    umma_ts8_elect(tmem + kBColDK, tmem + kBColDST,
-                   make_sdesc(smem_u32(sm.qc[st]), lbo_q, 512, kLayoutSW64), 1024 >> 4, kIdescBK,
-                   i > 0 ? 1u : 0u);
+    if (kBwdDkSmem) {
+      // A = dS^T read K-major from the dS core matrices in shared memory
+      // (key groups of 8 every 128 B, query groups of 8 every 2048 B)
+      umma_ss8_elect(tmem + kBColDK, make_sdesc(smem_u32(sm.ds[i & 1]), 2048, 128, kLayoutNone),
+                     4096 >> 4, make_sdesc(smem_u32(sm.qc[st]), lbo_q, 512, kLayoutSW64),
+                     1024 >> 4, kIdescBK, i > 0 ? 1u : 0u);
+    } else {
+      umma_ts8_elect(tmem + kBColDK, tmem + kBColDST,
+                     make_sdesc(smem_u32(sm.qc[st]), lbo_q, 512, kLayoutSW64), 1024 >> 4,
+                     kIdescBK, i > 0 ? 1u : 0u);
+    }
     umma_commit_elect(&sm.pt_free);
     umma_commit_elect(&sm.q_empty[st]);
     // the single dQ buffer is free once the drain warps pulled tile i-1
@@ -268,7 +281,6 @@ __device__ __forceinline__ void bwd_mma_dq(BwdSmem& sm, uint32_t tmem, const Bwd
     // step k: 16 queries further in dS (256 B), 16 keys further in [Kc|Kp] (1 KB)
     umma_ss8_elect(tmem + kBColDQ, make_sdesc(ds, 128, 2048, kLayoutNone), 256 >> 4,
                    make_sdesc(kc, lbo_k, 512, kLayoutSW64), 1024 >> 4, kIdescBQ, 0u);
-    umma_commit_elect(&sm.ds_free[i & 1]);
     umma_commit_elect(&sm.dq_full);
   }
   umma_commit_elect(&sm.mma_done);   // every dK MMA of the kernel has completed
@@ -345,7 +357,10 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
   bool ok = true;
   for (int i = 0; i < n; ++i) {
     const int st = i % kBwdStages;
-    if (!(ok = warp_wait(&sm.s_full, i & 1, ab, lim, SITE_BWD_COMPUTE))) break;
+    // S^T/dP^T of tile i, and the stage's lse / D rows (written by TMA)
+    if (!(ok = warp_wait2(&sm.s_full, i & 1, &sm.q_full[st], (i / kBwdStages) & 1, ab, lim,
+                          SITE_BWD_COMPUTE)))
+      break;
     tc_fence_after();
     uint32_t s[2][32], dp[2][32];
     tmem_ld_x32(tmem + lane_off + kBColS + 64 * g, s[0]);
@@ -360,9 +375,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.s_free);
-    // lse*log2e and D of this query tile (written by TMA)
-    if (!(ok = warp_wait(&sm.q_full[st], (i / kBwdStages) & 1, ab, lim, SITE_BWD_COMPUTE)))
-      break;
+    // lse*log2e and D of this query tile
     const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[st] + 64 * g);
     const float4* dd4 = reinterpret_cast<const float4*>(sm.dd[st] + 64 * g);
     // the whole 64-column slice in registers: P and dS, packed bf16 pairs
@@ -391,12 +404,11 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
         dk[2 * v4 + h2] = pack_bf16x2(lo2(d2), hi2(d2));
       }
     }
-    // P^T and dS^T (TMEM) are free once dV(i-1), dK(i-1) completed; the dS
-    // buffer i&1 (shared memory) once tile i-2's dQ MMAs completed.
+    // P^T and dS^T (TMEM) are free once dV(i-1) and dK(i-1) completed.  The
+    // dS buffer i&1 (shared memory) is free once tile i-2's dK and dQ MMAs
+    // completed: warp 15 issued those before dK(i-1), and its pt_free commit
+    // after dK(i-1) tracks every MMA it issued before, so pt_free covers both.
     if (i > 0 && !(ok = warp_wait(&sm.pt_free, (i - 1) & 1, ab, lim, SITE_BWD_COMPUTE))) break;
-    if (i > 1 &&
-        !(ok = warp_wait(&sm.ds_free[i & 1], ((i >> 1) - 1) & 1, ab, lim, SITE_BWD_COMPUTE)))
-      break;
     tc_fence_after();
     uint8_t* ds_row = sm.ds[i & 1];
 #pragma unroll
@@ -408,7 +420,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
         d8[e] = dk[8 * ch + e];
       }
       tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, p8);
-      tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, d8);
+      if (!kBwdDkSmem) tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, d8);
       const int q = 64 * g + 16 * ch;
       *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) = make_uint4(d8[0], d8[1], d8[2], d8[3]);
       *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q + 8)) =
@@ -497,8 +509,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.s_free, 8);
     mbar_init(&sm.ds_full, 8);
     mbar_init(&sm.pt_free, 2);       // dV (warp 14) and dK (warp 15)
-    mbar_init(&sm.ds_free[0], 1);
-    mbar_init(&sm.ds_free[1], 1);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_free, 4);
     mbar_init(&sm.mma_done, 2);

@@ -576,11 +576,39 @@ __device__ __forceinline__ T* align1024(uint8_t* p) {
   return reinterpret_cast<T*>(p + ((1024u - (a & 1023u)) & 1023u));
 }
 
+// Tests two barriers at once (both phases complete?): the two tests are in
+// flight together, so a warp that finds both ready pays one round trip.
+__device__ __forceinline__ bool mbar_try_wait2(uint64_t* bar0, uint32_t parity0, uint64_t* bar1,
+                                               uint32_t parity1) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q, [%3], %4;\n\t"
+      "and.pred p, p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar0)), "r"(parity0), "r"(smem_u32(bar1)), "r"(parity1)
+      : "memory");
+  return ok != 0;
+}
+
 // Warp-uniform bounded wait: the warp proceeds only if every lane saw the
 // phase complete, so no warp-collective tcgen05 op runs on a partial warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit, int site, uint32_t sleep_ns = 0) {
   const bool ok = mbar_wait(bar, parity, abort, limit, site, sleep_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// warp_wait on two barriers; when both phases are already complete (the
+// common case where it is used) the warp pays one test instead of two.
+__device__ __forceinline__ bool warp_wait2(uint64_t* bar0, uint32_t parity0, uint64_t* bar1,
+                                           uint32_t parity1, volatile int* abort, uint64_t limit,
+                                           int site) {
+  const bool ok = mbar_try_wait2(bar0, parity0, bar1, parity1) ||
+                  (mbar_wait(bar0, parity0, abort, limit, site) &&
+                   mbar_wait(bar1, parity1, abort, limit, site));
   return __all_sync(0xffffffffu, ok);
 }
 
