@@ -376,7 +376,7 @@ def run_rib(args, w):
             cla_bwd_only()
         ms_g, _, _ = timed(cla_gate_only, args.steps)
         ms_c, _, _ = timed(fwd_cla, args.steps)
-        ms_b, _, _ = timed(cla_bwd_only, args.steps)
+        ms_b, kern_b, _ = timed(cla_bwd_only, args.steps, trace=True)
         if sampler:
             sampler.stop()
         if world > 1:
@@ -384,7 +384,8 @@ def run_rib(args, w):
         if rank == 0:
             print(json.dumps({"cla_only": True, "cla_gate_ms": ms_g / args.steps,
                               "fwd_cla_ms": ms_c / args.steps,
-                              "cla_bwd_ms": ms_b / args.steps}))
+                              "cla_bwd_ms": ms_b / args.steps,
+                              "cla_bwd_kernels_ms": {k: v[1] / v[0] for k, v in kern_b.items()}}))
         return 0
     for _ in range(args.warmup):
         step()

@@ -61,8 +61,15 @@ __device__ __forceinline__ size_t cla_pix(const ClaBwdParams& p, int b, int i, i
   return (static_cast<size_t>(b) * p.H + i) * p.W + j;
 }
 
+// Element-wise part of the dz kernel: thread = (pixel slot, channel octet),
+// kDzBatch pixels' loads in flight at once.
+constexpr int kDzBatch = 2;
 __host__ __device__ __forceinline__ size_t cla_dz_smem_bytes(int C) {
-  return 2ull * C * C + 256ull * C + 4ull * (kClaBwdThreads / 32) * C + 64 + 1024;
+  return 2ull * C * C + 256ull * C + 4ull * 8 * kClaBwdThreads + 64 + 1024;
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const __nv_bfloat16* ptr) {
+  return __ldg(reinterpret_cast<const uint4*>(ptr));
 }
 
 // -------------------------------------------------------------- dz and dy
@@ -73,8 +80,8 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   const int C = p.C;
   uint8_t* sB = base;                                   // W_pw^T bf16 [N = c][K = o]
   uint8_t* sA = base + 2ull * C * C;                    // dz bf16 [M = 128 pixels][K = o]
-  float* red = reinterpret_cast<float*>(sA + 256ull * C);   // [warps][C]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(red + (kClaBwdThreads / 32) * C);
+  float* red = reinterpret_cast<float*>(sA + 256ull * C);   // [slot][C] db_pw partials
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 8 * kClaBwdThreads);
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,31 +110,54 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   const uint32_t idesc = make_idesc_bf16(128, C, false, false);
   const uint64_t adesc = make_sdesc(smem_u32(sA), 128, 16 * C, kLayoutNone);
   const uint64_t bdesc = make_sdesc(smem_u32(sB), 128, 16 * C, kLayoutNone);
-  const int groups = (C + 63) / 64;
-  float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // db_pw, per group
+  // element-wise part: thread = (pixel slot sl, channel octet k); slots
+  // take pixels sl, sl + slots, ...; consecutive threads read consecutive
+  // 16-byte octets of one pixel
+  const int octets = C / 8, slots = kClaBwdThreads / octets;
+  const int sl = threadIdx.x / octets, k = threadIdx.x % octets;
+  const bool act = sl < slots;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // db_pw, channels 8k..8k+7
   bool ok = true;
   int phase = 0;
   for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x) {
     int b, i0, j0;
     cla_tile(p, t, b, i0, j0);
-    // ---- element-wise: lanes along channel pairs, warps over pixels
+    for (int r0 = sl; act && r0 < 128; r0 += kDzBatch * slots) {
+      uint4 dgv[kDzBatch], ov[kDzBatch], gv[kDzBatch];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      if (g >= groups) break;
-      const int c = g * 64 + 2 * lane;
-      if (c >= C) continue;
-      for (int r = warp; r < 128; r += kClaBwdThreads / 32) {
-        const size_t off = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + c;
-        const float2 dg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p.dout_g + off));
-        const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p.out + off));
-        const float2 gt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p.gate + off));
-        const float z0 = dg.x * o.x * gt.x * (1.f - gt.x), z1 = dg.y * o.y * gt.y * (1.f - gt.y);
-        *reinterpret_cast<uint32_t*>(p.dout + off) = pack_bf16x2(dg.x * gt.x, dg.y * gt.y);
-        const uint32_t zb = pack_bf16x2(z0, z1);
-        *reinterpret_cast<uint32_t*>(p.dz + off) = zb;
-        *reinterpret_cast<uint32_t*>(sA + cla_kmajor_offset(r, c, C)) = zb;
-        acc[g][0] += z0;
-        acc[g][1] += z1;
+      for (int e = 0; e < kDzBatch; ++e) {
+        const int r = r0 + e * slots;
+        if (r < 128) {
+          const size_t off = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
+          dgv[e] = ldg_nc_v4(p.dout_g + off);
+          ov[e] = ldg_nc_v4(p.out + off);
+          gv[e] = ldg_nc_v4(p.gate + off);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < kDzBatch; ++e) {
+        const int r = r0 + e * slots;
+        if (r >= 128) continue;
+        const size_t off = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
+        const uint32_t dw[4] = {dgv[e].x, dgv[e].y, dgv[e].z, dgv[e].w};
+        const uint32_t ow[4] = {ov[e].x, ov[e].y, ov[e].z, ov[e].w};
+        const uint32_t gw[4] = {gv[e].x, gv[e].y, gv[e].z, gv[e].w};
+        uint32_t dov[4], zv[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 dg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw[h]));
+          const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[h]));
+          const float2 gt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[h]));
+          const float z0 = dg.x * o.x * gt.x * (1.f - gt.x), z1 = dg.y * o.y * gt.y * (1.f - gt.y);
+          dov[h] = pack_bf16x2(dg.x * gt.x, dg.y * gt.y);
+          zv[h] = pack_bf16x2(z0, z1);
+          acc[2 * h] += z0;
+          acc[2 * h + 1] += z1;
+        }
+        const uint4 z4 = make_uint4(zv[0], zv[1], zv[2], zv[3]);
+        *reinterpret_cast<uint4*>(p.dout + off) = make_uint4(dov[0], dov[1], dov[2], dov[3]);
+        *reinterpret_cast<uint4*>(p.dz + off) = z4;
+        *reinterpret_cast<uint4*>(sA + cla_kmajor_offset(r, 8 * k, C)) = z4;
       }
     }
     fence_proxy_async_smem();
@@ -172,19 +202,14 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
     volatile int no_abort = 0;
     mbar_wait(bar, phase ^ 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
   }
-  // db_pw partial of this CTA: the warps' sums, added in warp order
+  // db_pw partial of this CTA: the slots' sums, added in slot order
+  // (thread (sl, k) holds channels 8k..8k+7 at red[sl * C + 8k + e] = red[8 tid + e])
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int c = g * 64 + 2 * lane;
-    if (g < groups && c < C) {
-      red[warp * C + c] = acc[g][0];
-      red[warp * C + c + 1] = acc[g][1];
-    }
-  }
+  for (int e = 0; e < 8; ++e) red[8 * threadIdx.x + e] = act ? acc[e] : 0.f;
   __syncthreads();
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     float s = 0.f;
-    for (int w = 0; w < kClaBwdThreads / 32; ++w) s += red[w * C + c];
+    for (int w = 0; w < slots; ++w) s += red[w * C + c];
     p.part_dbpw[static_cast<size_t>(blockIdx.x) * C + c] = s;
   }
   tc_fence_before();
@@ -205,29 +230,47 @@ __device__ __forceinline__ uint32_t cla_mnmajor_offset(int r, int mn) {
 }
 
 // A: dz^T [M = 256 output channels, padded][K = 128 pixels]; B: y^T [N = C][K];
-// weights of the depth-wise convolution [9][C] and its bias [C].
+// the tile's x halo (10 x 18 pixels, one TMA box per 64 channels); weights
+// of the depth-wise convolution [9][C] and its bias [C].
+constexpr uint32_t kDwpwHaloChunk = (kClaHaloBytes + 1023u) & ~1023u;
 __host__ __device__ __forceinline__ size_t cla_dwpw_smem_bytes(int C) {
-  return 256ull * 256 + 256ull * C + 40ull * C + 64 + 1024;
+  return 256ull * 256 + 256ull * C + kDwpwHaloChunk * ((C + 63) / 64) + 40ull * C + 64 + 1024;
 }
 
 // grid p.grid, block kClaBwdThreads, dynamic smem cla_dwpw_smem_bytes(C).
-__global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const ClaBwdParams p) {
+// tm_x: x [B][H][W][C] as a 4D map with boxes of 64 channels x 18 x 10.
+__global__ void __launch_bounds__(kClaBwdThreads, 1)
+    cla_bwd_dwpw_kernel(const __grid_constant__ CUtensorMap tm_x, const ClaBwdParams p) {
   extern __shared__ uint8_t dw_raw[];
   uint8_t* base = dw_raw + ((1024u - (smem_u32(dw_raw) & 1023u)) & 1023u);
   const int C = p.C, octets = C / 8;
   uint8_t* sA = base;                          // dz^T, 64 KB
   uint8_t* sB = base + 256 * 256;              // y^T, 256 C bytes
-  float* sWdw = reinterpret_cast<float*>(sB + 256ull * C);   // [tap][C]
-  float* sBdw = sWdw + 9 * C;
+  const int chunks = (C + 63) / 64;
+  uint8_t* sH = sB + 256ull * C;               // halo [chunk][10 rows][18 cols][64 ch]
+  float* sWdw = reinterpret_cast<float*>(sH + static_cast<size_t>(kDwpwHaloChunk) * chunks);
+  float* sBdw = sWdw + 9 * C;                  // ([tap][C] weights before it)
   uint64_t* bar = reinterpret_cast<uint64_t*>(sBdw + C);
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
+  uint64_t* halo_bar = bar + 1;
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
+    mbar_init(halo_bar, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
+  // thread 0 loads the halo of each of the CTA's tiles; halos issued / waited for
+  int halo_issued = 0, halo_seen = 0;
+  auto load_halo = [&](int t) {
+    int b, i0, j0;
+    cla_tile(p, t, b, i0, j0);
+    mbar_arrive_expect_tx(halo_bar, kClaHaloBytes * chunks);
+    for (int g = 0; g < chunks; ++g)
+      tma_load_4d(sH + g * kDwpwHaloChunk, &tm_x, halo_bar, 64 * g, j0 - 1, i0 - 1, b);
+    ++halo_issued;
+  };
   for (int i = threadIdx.x; i < C; i += blockDim.x) {
     sBdw[i] = p.b_dw[i];
 #pragma unroll
@@ -250,32 +293,50 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
   const uint64_t adesc = make_sdesc(smem_u32(sA), 128, 2048, kLayoutNone);
   const uint64_t bdesc = make_sdesc(smem_u32(sB), 128, 2048, kLayoutNone);
   const bool two = C > 128;
+  // (after the barrier initialisation above is visible to the async proxy)
+  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < p.n_tiles) load_halo(blockIdx.x);
   bool ok = true;
   int phase = 0, n_done = 0;
   for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x, ++n_done) {
     int b, i0, j0;
     cla_tile(p, t, b, i0, j0);
-    // items: (channel octet k, pixel r), consecutive threads on consecutive
-    // pixels, so each 16-byte shared-memory store lands in its own banks
-    for (int it = threadIdx.x; it < octets * 128; it += blockDim.x) {
-      const int k = it >> 7, r = it & 127;
-      const int i = i0 + (r >> 4), j = j0 + (r & 15);
-      // dz^T: 8 output channels of pixel r
-      const uint4 zv = *reinterpret_cast<const uint4*>(p.dz + cla_pix(p, b, i, j) * C + 8 * k);
+    // items: (pixel r, channel octet k = 8 ch + ko); a warp takes 4
+    // neighbouring pixels x 8 octets of one 64-channel chunk, so its global
+    // reads are 128-byte runs and its halo reads 512 contiguous bytes
+    const int n_items = chunks * 1024;
+    // dz^T: 8 output channels of pixel r
+#pragma unroll 2
+    for (int it = threadIdx.x; it < n_items; it += blockDim.x) {
+      const int ko = it & 7, q = it >> 5, ch = q % chunks, k = ch * 8 + ko;
+      const int r = (q / chunks) * 4 + ((it >> 3) & 3);
+      if (k >= octets) continue;
+      const uint4 zv =
+          ldg_nc_v4(p.dz + cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k);
       *reinterpret_cast<uint4*>(sA + cla_mnmajor_offset(r, 8 * k)) = zv;
-      // y^T: the depth-wise convolution of x, 8 input channels of pixel r
+    }
+    ok = mbar_wait(halo_bar, halo_seen & 1, abort_flag, p.wait_limit_ns, SITE_CLA);
+    ++halo_seen;
+    if (!__syncthreads_and(ok)) {
+      ok = false;
+      break;
+    }
+    // y^T: the depth-wise convolution of x from the halo (zero outside the
+    // map: the TMA fills out-of-range pixels with zeros)
+#pragma unroll 2
+    for (int it = threadIdx.x; it < n_items; it += blockDim.x) {
+      const int ko = it & 7, q = it >> 5, ch = q % chunks, k = ch * 8 + ko;
+      const int r = (q / chunks) * 4 + ((it >> 3) & 3);
+      if (k >= octets) continue;
+      const int i = r >> 4, j = r & 15;   // tile-local; halo row i + u, column j + v
+      const uint8_t* h = sH + ch * kDwpwHaloChunk + ko * 16;
       float a[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) a[e] = sBdw[8 * k + e];
 #pragma unroll
-      for (int u = 0; u < 3; ++u) {
-        const int ii = i + u - 1;
-        if (ii < 0 || ii >= p.H) continue;
+      for (int u = 0; u < 3; ++u)
 #pragma unroll
         for (int v = 0; v < 3; ++v) {
-          const int jj = j + v - 1;
-          if (jj < 0 || jj >= p.W) continue;
-          const uint4 xv = *reinterpret_cast<const uint4*>(p.x + cla_pix(p, b, ii, jj) * C + 8 * k);
+          const uint4 xv = *reinterpret_cast<const uint4*>(h + ((i + u) * 18 + (j + v)) * 128);
           const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
           const float* w = sWdw + (u * 3 + v) * C + 8 * k;
 #pragma unroll
@@ -285,7 +346,6 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
             a[2 * e + 1] = fmaf(w[2 * e + 1], xf.y, a[2 * e + 1]);
           }
         }
-      }
       *reinterpret_cast<uint4*>(sB + cla_mnmajor_offset(r, 8 * k)) =
           make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
                      pack_bf16x2(a[6], a[7]));
@@ -294,6 +354,9 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the halo is read: fetch the next tile's while this one's MMAs run
+    if (threadIdx.x == 0 && t + static_cast<int>(gridDim.x) < p.n_tiles)
+      load_halo(t + gridDim.x);
     // D0 (+)= dz^T[o 0..127] y, D1 (+)= dz^T[o 128..255] y: 8 K-steps of 16 pixels
     if (warp == 0) {
       const uint32_t acc = n_done > 0 ? 1u : 0u;
@@ -314,6 +377,9 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
   if (!ok) {
     volatile int no_abort = 0;
     mbar_wait(bar, phase ^ 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
+    // a halo still in flight lands before the CTA exits
+    if (threadIdx.x == 0 && halo_issued > halo_seen)
+      mbar_wait(halo_bar, (halo_issued - 1) & 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
   }
   // the CTA's partial dW_pw: rows o from TMEM lanes, C columns each
   if (ok && warp < 8) {
@@ -349,12 +415,21 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dwpw_kernel(const C
 
 // -------------------------------------------------------------- dx, dW_dw, db_dw
 // grid p.grid_dx, block kClaDxThreads, static smem.  Lanes along channel
-// pairs, warps over the tile's pixels; one 64-channel group at a time over
-// all of the CTA's tiles, so each thread keeps 20 partial sums.
-__global__ void __launch_bounds__(kClaDxThreads) cla_bwd_dx_kernel(const ClaBwdParams p) {
+// pairs (one 64-channel group at a time over all of the CTA's tiles, so each
+// thread keeps 20 partial sums); a warp walks down one column of a tile at a
+// time with the 3 x 3 neighbourhoods of x and dy in registers, loading only
+// the new row of each per pixel.
+__device__ __forceinline__ float2 cla_ld2(const __nv_bfloat16* ptr, bool valid) {
+  if (!valid) return make_float2(0.f, 0.f);
+  const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(ptr));
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+}
+
+__global__ void __launch_bounds__(kClaDxThreads, 2) cla_bwd_dx_kernel(const ClaBwdParams p) {
   __shared__ float red[kClaDxThreads / 32][10][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.C;
+  const size_t row_stride = static_cast<size_t>(p.W) * C;   // elements between map rows
   for (int g = 0; g * 64 < C; ++g) {
     const int c = g * 64 + 2 * lane;
     const bool act = c < C;
@@ -368,36 +443,60 @@ __global__ void __launch_bounds__(kClaDxThreads) cla_bwd_dx_kernel(const ClaBwdP
     for (int t = blockIdx.x; act && t < p.n_tiles; t += gridDim.x) {
       int b, i0, j0;
       cla_tile(p, t, b, i0, j0);
-      for (int r = warp; r < 128; r += kClaDxThreads / 32) {
-        const int i = i0 + (r >> 4), j = j0 + (r & 15);
-        const float2 d = __bfloat1622float2(
-            *reinterpret_cast<const __nv_bfloat162*>(p.dy + cla_pix(p, b, i, j) * C + c));
-        ab0 += d.x;
-        ab1 += d.y;
-        float dx0 = 0.f, dx1 = 0.f;
+      for (int jc = warp; jc < 16; jc += kClaDxThreads / 32) {
+        const int j = j0 + jc;
+        const bool cv[3] = {j > 0, true, j + 1 < p.W};
+        // xw[u][v] = x(i + u - 1, j + v - 1), dw[u][v] = dy(i + u - 1, j + v - 1)
+        float2 xw[3][3], dw[3][3];
+        // element offset of (row i0 - 1, column j - 1), channel c; only
+        // dereferenced where the row and column are inside the map
+        const long long o0 = (static_cast<long long>(b) * p.H + (i0 - 1)) * p.W * C +
+                             static_cast<long long>(j - 1) * C + c;
 #pragma unroll
-        for (int u = 0; u < 3; ++u)
+        for (int u = 0; u < 3; ++u) {
+          const bool rv = i0 - 1 + u >= 0 && i0 - 1 + u < p.H;
 #pragma unroll
           for (int v = 0; v < 3; ++v) {
-            const int tp = u * 3 + v;
-            // dW_dw: dy here times x at (i + u - 1, j + v - 1)
-            const int xi = i + u - 1, xj = j + v - 1;
-            if (xi >= 0 && xi < p.H && xj >= 0 && xj < p.W) {
-              const float2 xf = __bfloat1622float2(
-                  *reinterpret_cast<const __nv_bfloat162*>(p.x + cla_pix(p, b, xi, xj) * C + c));
-              aw0[tp] = fmaf(d.x, xf.x, aw0[tp]);
-              aw1[tp] = fmaf(d.y, xf.y, aw1[tp]);
+            const long long o = o0 + u * static_cast<long long>(row_stride) + v * C;
+            xw[u][v] = cla_ld2(p.x + o, rv && cv[v]);
+            dw[u][v] = cla_ld2(p.dy + o, rv && cv[v]);
+          }
+        }
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii) {
+          const int i = i0 + ii;
+          const float2 d = dw[1][1];
+          ab0 += d.x;
+          ab1 += d.y;
+          float dx0 = 0.f, dx1 = 0.f;
+#pragma unroll
+          for (int u = 0; u < 3; ++u)
+#pragma unroll
+            for (int v = 0; v < 3; ++v) {
+              const int tp = u * 3 + v;
+              // dW_dw: dy here times x at (i + u - 1, j + v - 1)
+              aw0[tp] = fmaf(d.x, xw[u][v].x, aw0[tp]);
+              aw1[tp] = fmaf(d.y, xw[u][v].y, aw1[tp]);
+              // dx: tap (u, v) times dy at (i - u + 1, j - v + 1)
+              dx0 = fmaf(w0[tp], dw[2 - u][2 - v].x, dx0);
+              dx1 = fmaf(w1[tp], dw[2 - u][2 - v].y, dx1);
             }
-            // dx: W_dw tap (u, v) times dy at (i - u + 1, j - v + 1)
-            const int yi = i - u + 1, yj = j - v + 1;
-            if (yi >= 0 && yi < p.H && yj >= 0 && yj < p.W) {
-              const float2 df = __bfloat1622float2(
-                  *reinterpret_cast<const __nv_bfloat162*>(p.dy + cla_pix(p, b, yi, yj) * C + c));
-              dx0 = fmaf(w0[tp], df.x, dx0);
-              dx1 = fmaf(w1[tp], df.y, dx1);
+          *reinterpret_cast<uint32_t*>(p.dx + cla_pix(p, b, i, j) * C + c) = pack_bf16x2(dx0, dx1);
+          if (ii < 7) {
+            // slide down one row: drop row i - 1, load row i + 2
+            const bool rv = i + 2 < p.H;
+#pragma unroll
+            for (int v = 0; v < 3; ++v) {
+              xw[0][v] = xw[1][v];
+              xw[1][v] = xw[2][v];
+              dw[0][v] = dw[1][v];
+              dw[1][v] = dw[2][v];
+              const long long o = o0 + (ii + 3) * static_cast<long long>(row_stride) + v * C;
+              xw[2][v] = cla_ld2(p.x + o, rv && cv[v]);
+              dw[2][v] = cla_ld2(p.dy + o, rv && cv[v]);
             }
           }
-        *reinterpret_cast<uint32_t*>(p.dx + cla_pix(p, b, i, j) * C + c) = pack_bf16x2(dx0, dx1);
+        }
       }
     }
     // this group's partials: the warps' sums, added in warp order

@@ -705,6 +705,16 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   p.grid_dx = L.grid_dx;
   p.wait_limit_ns = g_wait_limit_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // x [B][H][W][C] bf16 as a 4D map; box = one tile's 10 x 18 halo, 64 channels
+  CUtensorMap tm_x;
+  {
+    const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {2ull * C, 2ull * C * W, 2ull * C * W * H};
+    const uint32_t box[4] = {64, 18, 10, 1};
+    rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+  }
   const size_t smem_dz = cla_dz_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
   if ((rc = set_smem(cla_bwd_dz_kernel, smem_dz))) return rc;
   if ((rc = set_smem(cla_bwd_dwpw_kernel, smem_dw))) return rc;
@@ -715,7 +725,7 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   }
   {
     TraceScope ts(K_CLA_DWPW, st);
-    cla_bwd_dwpw_kernel<<<L.grid, kClaBwdThreads, smem_dw, st>>>(p);
+    cla_bwd_dwpw_kernel<<<L.grid, kClaBwdThreads, smem_dw, st>>>(tm_x, p);
     if ((rc = launch_status())) return rc;
   }
   {
