@@ -37,7 +37,11 @@ so a test can vary it):
   4. softmax scale tau applied to the whole augmented product, default
      1/sqrt(d + rank);
   5. the window shift is a pure cyclic roll by -s on both map axes before the
-     partition and +s after it, with no region mask;
+     partition and +s after it, with no region mask.  An optional variant
+     (off by default, `region_mask=True`) adds the usual shifted-window
+     region mask, which the pages do not describe: on the rolled map, rows
+     split into [0, H-M), [H-M, H-s), [H-s, H) and columns likewise, and a
+     query attends only to keys of its own (row band, column band) region;
   6. lse is the natural-log log-sum-exp of the scaled scores.
 
 Memory: rows of the N x N score matrix are processed in row blocks when N is
@@ -59,7 +63,7 @@ __all__ = [
     "mlp_backward", "pos_tokens", "pos_tokens_backward", "window_partition",
     "window_reverse", "unit_scores", "attention_unit", "attention_unit_rows",
     "attention_unit_backward", "attn_fwd", "attn_bwd", "default_scale",
-    "unit_index", "gather_unit",
+    "unit_index", "gather_unit", "region_labels",
 ]
 
 _ROW_BLOCK = 2048
@@ -227,14 +231,32 @@ def unit_index(H, W, M, heads, b, w, h):
 # Attention for one (batch, window, head) unit
 # --------------------------------------------------------------------------
 
-def unit_scores(qc, kc, qp, kp, scale):
+def region_labels(H: int, W: int, M: int, s: int, wy: int, wx: int):
+    """Region label of each token of window (wy, wx), [M*M] ints, t = i*M+j.
+
+    Reading 5's optional mask: on the map rolled by -s, a row y belongs to
+    band 0 if y < H-M, band 1 if y < H-s, else band 2 (columns alike with W);
+    the label is 3*row_band + column_band.  With s = 0 every label is 0."""
+    def band(pos, size):
+        if s == 0:
+            return np.zeros_like(pos)
+        return np.where(pos < size - M, 0, np.where(pos < size - s, 1, 2))
+    i, j = np.divmod(np.arange(M * M), M)
+    return 3 * band(wy * M + i, H) + band(wx * M + j, W)
+
+
+def unit_scores(qc, kc, qp, kp, scale, allowed=None):
     """Scaled scores S = tau * (Qc Kc^T + B) with the explicit bias B = Qp Kp^T.
 
     This is the RPB-style form S = QK^T + B of [EN] §2.A (Mechanism) with the
     bias materialised; the pages' identity says it equals the augmented dot
-    product, which the pins check separately."""
+    product, which the pins check separately.  `allowed` (bool [rows, keys]),
+    if given, sets the scores of the other pairs to -inf."""
     bias = _f64(qp) @ _f64(kp).T
-    return scale * (_f64(qc) @ _f64(kc).T + bias)
+    sc = scale * (_f64(qc) @ _f64(kc).T + bias)
+    if allowed is not None:
+        sc = np.where(allowed, sc, -np.inf)
+    return sc
 
 
 def _softmax_rows(s):
@@ -244,10 +266,20 @@ def _softmax_rows(s):
     return e / l, (m + np.log(l))[:, 0]
 
 
-def attention_unit_rows(qc, kc, v, qp, kp, scale, rows=None):
+def _allowed(labels, r0, r1, rows=None):
+    """Query rows r0..r1 (of `rows`, if given) x all keys: same region label."""
+    if labels is None:
+        return None
+    q = labels[rows][r0:r1] if rows is not None else labels[r0:r1]
+    return q[:, None] == labels[None, :]
+
+
+def attention_unit_rows(qc, kc, v, qp, kp, scale, rows=None, labels=None):
     """Output and lse of the given query rows of one unit (all rows if None).
 
-    softmax over keys of tau*(Qc Kc^T + Qp Kp^T), then P V."""
+    softmax over keys of tau*(Qc Kc^T + Qp Kp^T), then P V.  With `labels`
+    (region label per token, see region_labels) a query only sees keys of its
+    own label."""
     qc, kc, v, qp, kp = map(_f64, (qc, kc, v, qp, kp))
     if rows is not None:
         qc, qp = qc[rows], qp[rows]
@@ -256,24 +288,25 @@ def attention_unit_rows(qc, kc, v, qp, kp, scale, rows=None):
     lse = np.empty(n)
     for r0 in range(0, n, _ROW_BLOCK):
         r1 = min(n, r0 + _ROW_BLOCK)
-        s = unit_scores(qc[r0:r1], kc, qp[r0:r1], kp, scale)
+        s = unit_scores(qc[r0:r1], kc, qp[r0:r1], kp, scale, _allowed(labels, r0, r1, rows))
         p, lse[r0:r1] = _softmax_rows(s)
         out[r0:r1] = p @ v
     return out, lse
 
 
-def attention_unit(qc, kc, v, qp, kp, scale):
+def attention_unit(qc, kc, v, qp, kp, scale, labels=None):
     """Forward of one unit: (O [N, d], lse [N])."""
-    return attention_unit_rows(qc, kc, v, qp, kp, scale)
+    return attention_unit_rows(qc, kc, v, qp, kp, scale, labels=labels)
 
 
-def attention_unit_backward(qc, kc, v, qp, kp, scale, dout):
+def attention_unit_backward(qc, kc, v, qp, kp, scale, dout, labels=None):
     """Textbook softmax-attention backward of one unit, fp64.
 
     With P = softmax(S), O = P V and upstream dO:
       dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(P * dP)),
       dQc = tau dS Kc,  dQp = tau dS Kp,  dKc = tau dS^T Qc,  dKp = tau dS^T Qp
-    (the bias term tau*Qp Kp^T contributes the Qp/Kp gradients)."""
+    (the bias term tau*Qp Kp^T contributes the Qp/Kp gradients).  Masked
+    pairs (`labels`) have P = 0, hence dS = 0."""
     qc, kc, v, qp, kp, do = map(_f64, (qc, kc, v, qp, kp, dout))
     n = qc.shape[0]
     dqc = np.empty_like(qc)
@@ -283,7 +316,7 @@ def attention_unit_backward(qc, kc, v, qp, kp, scale, dout):
     dv = np.zeros_like(v)
     for r0 in range(0, n, _ROW_BLOCK):
         r1 = min(n, r0 + _ROW_BLOCK)
-        s = unit_scores(qc[r0:r1], kc, qp[r0:r1], kp, scale)
+        s = unit_scores(qc[r0:r1], kc, qp[r0:r1], kp, scale, _allowed(labels, r0, r1))
         p, _ = _softmax_rows(s)
         dob = do[r0:r1]
         dv += p.T @ dob
@@ -309,12 +342,13 @@ def gather_unit(qkv, qp, kp, M, s, b, w, h):
 # Whole feature map
 # --------------------------------------------------------------------------
 
-def attn_fwd(qkv, M: int, s: int, qp, kp, scale=None):
+def attn_fwd(qkv, M: int, s: int, qp, kp, scale=None, region_mask=False):
     """Windowed RIB attention over a feature map.
 
     qkv [B][H][W][3][heads][d] (Qc, Kc, V); qp, kp [heads][M][M][r].
     Returns out [B][H][W][heads][d] and lse [B][heads][H][W], both fp64, at
-    the original (un-rolled) pixel positions."""
+    the original (un-rolled) pixel positions.  region_mask: reading 5's
+    optional shifted-window mask."""
     x = _f64(qkv)
     B, H, W, _, heads, d = x.shape
     r = _f64(qp).shape[-1]
@@ -329,8 +363,10 @@ def attn_fwd(qkv, M: int, s: int, qp, kp, scale=None):
         kpf = _f64(kp)[h].reshape(M * M, r)
         for b in range(B):
             for w in range(nW):
+                lab = (region_labels(H, W, M, s, w // (W // M), w % (W // M))
+                       if region_mask else None)
                 o, l = attention_unit(xw[b, w, :, 0, h], xw[b, w, :, 1, h],
-                                      xw[b, w, :, 2, h], qpf, kpf, scale)
+                                      xw[b, w, :, 2, h], qpf, kpf, scale, labels=lab)
                 ow[b, w, :, h] = o
                 lw[b, w, :, h] = l
     out = window_reverse(ow, M, s, H, W)
@@ -338,7 +374,7 @@ def attn_fwd(qkv, M: int, s: int, qp, kp, scale=None):
     return out, lse
 
 
-def attn_bwd(qkv, dout, M: int, s: int, qp, kp, scale=None, units=None):
+def attn_bwd(qkv, dout, M: int, s: int, qp, kp, scale=None, units=None, region_mask=False):
     """Gradients of sum(attn_fwd(...)[0] * dout).
 
     Returns dqkv [B][H][W][3][heads][d] and dqp, dkp [heads][M][M][r] summed
@@ -363,9 +399,11 @@ def attn_bwd(qkv, dout, M: int, s: int, qp, kp, scale=None, units=None):
             for w in range(nW):
                 if units is not None and (b, w, h) not in units:
                     continue
+                lab = (region_labels(H, W, M, s, w // (W // M), w % (W // M))
+                       if region_mask else None)
                 g = attention_unit_backward(
                     xw[b, w, :, 0, h], xw[b, w, :, 1, h], xw[b, w, :, 2, h],
-                    qpf, kpf, scale, dow[b, w, :, h])
+                    qpf, kpf, scale, dow[b, w, :, h], labels=lab)
                 dxw[b, w, :, 0, h] = g[0]
                 dxw[b, w, :, 1, h] = g[1]
                 dxw[b, w, :, 2, h] = g[2]

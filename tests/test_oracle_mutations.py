@@ -12,12 +12,16 @@ from oracle import rib_oracle as R
 import tests.test_oracle_pins as P
 
 
-def _scores_bias_sign(qc, kc, qp, kp, scale):
-    return scale * (R._f64(qc) @ R._f64(kc).T - R._f64(qp) @ R._f64(kp).T)
+def _masked(sc, allowed):
+    return sc if allowed is None else np.where(allowed, sc, -np.inf)
 
 
-def _scores_no_bias(qc, kc, qp, kp, scale):
-    return scale * (R._f64(qc) @ R._f64(kc).T)
+def _scores_bias_sign(qc, kc, qp, kp, scale, allowed=None):
+    return _masked(scale * (R._f64(qc) @ R._f64(kc).T - R._f64(qp) @ R._f64(kp).T), allowed)
+
+
+def _scores_no_bias(qc, kc, qp, kp, scale, allowed=None):
+    return _masked(scale * (R._f64(qc) @ R._f64(kc).T), allowed)
 
 
 def _fourier_swapped(y, x, freqs):
@@ -44,9 +48,9 @@ def _partition_wrong_roll(x, M, s):
 _orig_partition = R.window_partition
 
 
-def _bwd_missing_rowsum(qc, kc, v, qp, kp, scale, dout):
+def _bwd_missing_rowsum(qc, kc, v, qp, kp, scale, dout, labels=None):
     qc, kc, v, qp, kp, do = map(R._f64, (qc, kc, v, qp, kp, dout))
-    s = R.unit_scores(qc, kc, qp, kp, scale)
+    s = R.unit_scores(qc, kc, qp, kp, scale, R._allowed(labels, 0, qc.shape[0]))
     p, _ = R._softmax_rows(s)
     dp = do @ v.T
     ds = p * dp
@@ -54,8 +58,8 @@ def _bwd_missing_rowsum(qc, kc, v, qp, kp, scale, dout):
             scale * ds.T @ qp)
 
 
-def _bwd_dk_transposed(qc, kc, v, qp, kp, scale, dout):
-    g = list(_orig_unit_bwd(qc, kc, v, qp, kp, scale, dout))
+def _bwd_dk_transposed(qc, kc, v, qp, kp, scale, dout, labels=None):
+    g = list(_orig_unit_bwd(qc, kc, v, qp, kp, scale, dout, labels=labels))
     g[4] = scale * 0 + g[3][: g[4].shape[0]]          # dKp taken from dQp
     return tuple(g)
 
