@@ -289,6 +289,31 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * rib_window_attn_fwd_masked / rib_window_attn_bwd_masked -- the same
+ * forward and backward with the shifted-window region mask, an optional
+ * variant the pages do not describe (they use a pure cyclic roll).  On the
+ * map rolled by -shift, rows fall into the bands [0, H-M), [H-M, H-shift),
+ * [H-shift, H) and columns likewise; a query attends only to keys of its own
+ * (row band, column band).  Only windows in the last window row or column
+ * hold more than one region; elsewhere, and with shift == 0, the results
+ * equal the unmasked calls.  Masked pairs get P = 0 exactly (their dS is 0
+ * too).  Arguments, layouts, limits and errors are those of
+ * rib_window_attn_fwd / rib_window_attn_bwd; pass lse from the masked
+ * forward to the masked backward.
+ * ------------------------------------------------------------------------ */
+int rib_window_attn_fwd_masked(const void* qkv, int B, int H, int W, int heads,
+                               int head_dim, int window, int shift,
+                               const void* qp_bf16, const void* kp_bf16, int rank,
+                               float scale, void* out, float* lse, void* stream);
+int rib_window_attn_bwd_masked(const void* qkv, const void* out, const void* dout,
+                               const float* lse, int B, int H, int W, int heads,
+                               int head_dim, int window, int shift,
+                               const void* qp_bf16, const void* kp_bf16, int rank,
+                               float scale, void* dqkv, float* dqp, float* dkp,
+                               const rib_mlp_t* mlp, const rib_mlp_grad_t* dmlp,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * rib_window_gather / rib_window_scatter -- the window partition with cyclic
  * shift as a standalone copy (the same rolled TMA tile addressing the
  * attention kernels use), for bit-exact checks and for callers that want

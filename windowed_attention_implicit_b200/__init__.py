@@ -203,18 +203,22 @@ def rib_pos_tokens_bwd_noalloc(mlp: PositionMLP, window: int, dqp: torch.Tensor,
 
 def rib_window_attn_fwd(qkv: torch.Tensor, window: int, shift: int, qp_bf16=None,
                         kp_bf16=None, rank: int = 16, scale: float = 0.0, out=None, lse=None,
-                        stream=None):
-    """out bf16 [B][H][W][heads][d], lse fp32 [B][heads][H][W]."""
+                        stream=None, region_mask: bool = False):
+    """out bf16 [B][H][W][heads][d], lse fp32 [B][heads][H][W].
+
+    region_mask: the optional shifted-window region mask
+    (rib_window_attn_fwd_masked)."""
     B, H, W, three, heads, d = qkv.shape
     if three != 3:
         raise ValueError("qkv must be [B][H][W][3][heads][head_dim]")
     out = torch.empty((B, H, W, heads, d), device=qkv.device, dtype=torch.bfloat16) if out is None else out
     lse = torch.empty((B, heads, H, W), device=qkv.device, dtype=torch.float32) if lse is None else lse
-    _check(library().rib_window_attn_fwd(
+    name = "rib_window_attn_fwd_masked" if region_mask else "rib_window_attn_fwd"
+    _check(getattr(library(), name)(
         _ptr(qkv, torch.bfloat16, "qkv"), B, H, W, heads, d, int(window), int(shift),
         _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
         int(rank), float(scale), _ptr(out, torch.bfloat16, "out"),
-        _ptr(lse, torch.float32, "lse"), _stream(stream)), "rib_window_attn_fwd")
+        _ptr(lse, torch.float32, "lse"), _stream(stream)), name)
     return out, lse
 
 
@@ -314,8 +318,10 @@ def rib_window_attn_bwd_workspace(B, H, W, heads, head_dim, window, rank,
 def rib_window_attn_bwd(qkv, out, dout, lse, window: int, shift: int, qp_bf16=None,
                         kp_bf16=None, rank: int = 16, scale: float = 0.0,
                         mlp: Optional[PositionMLP] = None, dqkv=None, dqp=None, dkp=None,
-                        dmlp: Optional[PositionMLPGrad] = None, workspace=None, stream=None):
-    """Returns dict(dqkv, dqp, dkp, dmlp).  dmlp is computed when mlp is given."""
+                        dmlp: Optional[PositionMLPGrad] = None, workspace=None, stream=None,
+                        region_mask: bool = False):
+    """Returns dict(dqkv, dqp, dkp, dmlp).  dmlp is computed when mlp is given.
+    region_mask: as for rib_window_attn_fwd (rib_window_attn_bwd_masked)."""
     B, H, W, _, heads, d = qkv.shape
     dev = qkv.device
     dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
@@ -330,7 +336,8 @@ def rib_window_attn_bwd(qkv, out, dout, lse, window: int, shift: int, qp_bf16=No
         workspace = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
     c_mlp = mlp.c_struct() if mlp is not None else None
     c_dmlp = dmlp.c_struct() if (mlp is not None and dmlp is not None) else None
-    _check(library().rib_window_attn_bwd(
+    name = "rib_window_attn_bwd_masked" if region_mask else "rib_window_attn_bwd"
+    _check(getattr(library(), name)(
         _ptr(qkv, torch.bfloat16, "qkv"), _ptr(out, torch.bfloat16, "out"),
         _ptr(dout, torch.bfloat16, "dout"), _ptr(lse, torch.float32, "lse"),
         B, H, W, heads, d, int(window), int(shift),
@@ -340,7 +347,7 @@ def rib_window_attn_bwd(qkv, out, dout, lse, window: int, shift: int, qp_bf16=No
         ctypes.byref(c_mlp) if c_mlp is not None else None,
         ctypes.byref(c_dmlp) if c_dmlp is not None else None,
         _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
-        _stream(stream)), "rib_window_attn_bwd")
+        _stream(stream)), name)
     return {"dqkv": dqkv, "dqp": dqp, "dkp": dkp, "dmlp": dmlp}
 
 

@@ -50,6 +50,8 @@ _SIGS = {
                                         ctypes.POINTER(rib_mlp_grad_t), _p]),
     "rib_window_attn_fwd": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
                                  ctypes.c_float, _p, _p, _p]),
+    "rib_window_attn_fwd_masked": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
+                                        ctypes.c_float, _p, _p, _p]),
     "rib_window_attn_fwd_cla": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
                                      ctypes.c_float, _p, _p, _p, _p, _p]),
     "rib_cla_gate": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]),
@@ -63,6 +65,11 @@ _SIGS = {
                                  _i, ctypes.c_float, _p, _p, _p,
                                  ctypes.POINTER(rib_mlp_t),
                                  ctypes.POINTER(rib_mlp_grad_t), _p, ctypes.c_size_t, _p]),
+    "rib_window_attn_bwd_masked": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p,
+                                        _i, ctypes.c_float, _p, _p, _p,
+                                        ctypes.POINTER(rib_mlp_t),
+                                        ctypes.POINTER(rib_mlp_grad_t), _p, ctypes.c_size_t,
+                                        _p]),
     "rib_window_gather": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p]),
     "rib_window_scatter": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p]),
     "rib_status_string": (ctypes.c_char_p, [_i]),

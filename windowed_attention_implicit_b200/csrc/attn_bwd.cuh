@@ -89,6 +89,7 @@ constexpr uint64_t kBwdDrainNs = 200ull * 1000ull * 1000ull;
 
 struct BwdParams {
   int B, H, W, heads, M, s, rank, nWx, nW, tiles_x, n_tiles;
+  int region_mask;   // shifted-window region mask on (requires s > 0)
   float scale;       // tau
   float scale_log2;  // tau * log2(e)
   __nv_bfloat16* dqkv;
@@ -342,6 +343,7 @@ __device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdP
   if (leader) tma_store_wait_all();
 }
 
+template <bool kMask>
 __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const BwdParams& p,
                                             const UnitCoord& u, int unit, int kt, int g,
                                             int wq) {
@@ -354,9 +356,28 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
   const float sl = p.scale_log2;
   const uint64_t sl2 = pk2(sl, sl);
+  // region mask: bands of this thread's key token.  A warp's 32 keys are a
+  // 4 x 8 block and its 64 query columns an 8 x 8 block, so the mask is one
+  // warp-uniform decision per query tile (kv); masked blocks have P = dS = 0.
+  const bool mask_on = kMask && (u.wy == p.nW / p.nWx - 1 || u.wx == p.nWx - 1);
+  int kbr = 0, kbc = 0;
+  if (mask_on) {
+    int ki0, kj0, ki, kj;
+    tile_origin(kt, p.tiles_x, ki0, kj0);
+    tile_row_local(key, ki0, kj0, ki, kj);
+    kbr = region_band(u.wy * p.M + ki, p.H, p.M, p.s);
+    kbc = region_band(u.wx * p.M + kj, p.W, p.M, p.s);
+  }
   bool ok = true;
   for (int i = 0; i < n; ++i) {
     const int st = i % kBwdStages;
+    bool kv = true;
+    if (mask_on) {
+      int qi0, qj0;
+      tile_origin(i, p.tiles_x, qi0, qj0);
+      kv = region_band(u.wy * p.M + qi0, p.H, p.M, p.s) == kbr &&
+           region_band(u.wx * p.M + qj0 + 8 * g, p.W, p.M, p.s) == kbc;
+    }
     // S^T/dP^T of tile i, and the stage's lse / D rows (written by TMA)
     if (!(ok = warp_wait2(&sm.s_full, i & 1, &sm.q_full[st], (i / kBwdStages) & 1, ab, lim,
                           SITE_BWD_COMPUTE)))
@@ -411,20 +432,35 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     if (i > 0 && !(ok = warp_wait(&sm.pt_free, (i - 1) & 1, ab, lim, SITE_BWD_COMPUTE))) break;
     tc_fence_after();
     uint8_t* ds_row = sm.ds[i & 1];
+    if (kv) {
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t p8[8], d8[8];
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t p8[8], d8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        p8[e] = pk[8 * ch + e];
-        d8[e] = dk[8 * ch + e];
+        for (int e = 0; e < 8; ++e) {
+          p8[e] = pk[8 * ch + e];
+          d8[e] = dk[8 * ch + e];
+        }
+        tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, p8);
+        if (!kBwdDkSmem) tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, d8);
+        const int q = 64 * g + 16 * ch;
+        *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) =
+            make_uint4(d8[0], d8[1], d8[2], d8[3]);
+        *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q + 8)) =
+            make_uint4(d8[4], d8[5], d8[6], d8[7]);
       }
-      tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, p8);
-      if (!kBwdDkSmem) tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, d8);
-      const int q = 64 * g + 16 * ch;
-      *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) = make_uint4(d8[0], d8[1], d8[2], d8[3]);
-      *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q + 8)) =
-          make_uint4(d8[4], d8[5], d8[6], d8[7]);
+    } else {
+      // a masked block: P = dS = 0 (a store path of its own, so that the
+      // unmasked path carries no per-element selects)
+      const uint32_t z8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        tmem_st_x8(tmem + lane_off + kBColP + 32 * g + 8 * ch, z8);
+        if (!kBwdDkSmem) tmem_st_x8(tmem + lane_off + kBColDST + 32 * g + 8 * ch, z8);
+        const int q = 64 * g + 16 * ch;
+        *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(ds_row + ds_offset(key, q + 8)) = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     tmem_wait_st();
     fence_proxy_async_smem();
@@ -486,6 +522,8 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
 }
 
 // grid (n_tiles, units), block kBwdThreads, dynamic smem kBwdSmemBytes.
+// kMask: the shifted-window region mask (a separate instantiation).
+template <bool kMask>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                     const __grid_constant__ CUtensorMap tm_dout,
@@ -532,7 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   if (warp < 8) {
     regs_inc<kBwdComputeRegs>();
-    bwd_compute(sm, tmem, p, u, unit, kt, warp >> 2, warp & 3);
+    bwd_compute<kMask>(sm, tmem, p, u, unit, kt, warp >> 2, warp & 3);
   } else {
     regs_dec<kBwdServiceRegs>();
     if (warp < 12) {

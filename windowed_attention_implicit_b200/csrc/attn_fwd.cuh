@@ -83,6 +83,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct FwdParams {
   int B, H, W, heads, M, s, rank, nWx, nW, tiles_x, n_tiles;
+  int region_mask;   // shifted-window region mask on (requires s > 0)
   float scale_log2;  // softmax scale * log2(e)
   __nv_bfloat16* out;
   float* lse;
@@ -260,6 +261,7 @@ __device__ __forceinline__ bool wait_pv_count(FwdSmem& sm, int X, int need, cons
   return ok;
 }
 
+template <bool kMask>
 __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
                                             const UnitCoord& u, int tile0, int X, int h, int wq) {
   volatile int* ab = &sm.abort_flag;
@@ -271,10 +273,29 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   const float sl = p.scale_log2;
   const uint64_t sl2 = pk2(sl, sl);
   const int n = p.n_tiles;
+  // region mask: bands of this row's query token.  A warp's 32 rows are a
+  // 4 x 8 block of the window and its 64 key columns an 8 x 8 block, so the
+  // mask is one warp-uniform decision per key tile (kv).
+  const bool mask_on = kMask && (u.wy == p.nW / p.nWx - 1 || u.wx == p.nWx - 1);
+  int qbr = 0, qbc = 0;
+  if (mask_on) {
+    int qi0, qj0, qi, qj;
+    tile_origin(tile0 + X, p.tiles_x, qi0, qj0);
+    tile_row_local(row, qi0, qj0, qi, qj);
+    qbr = region_band(u.wy * p.M + qi, p.H, p.M, p.s);
+    qbc = region_band(u.wx * p.M + qj, p.W, p.M, p.s);
+  }
   float m_run = 0.f;
   bool ok = true;
   for (int j = 0; j < n; ++j) {
     const int k = 2 * j + X, r = k % kRegions;
+    bool kv = true;
+    if (mask_on) {
+      int ki0, kj0;
+      tile_origin(j, p.tiles_x, ki0, kj0);
+      kv = region_band(u.wy * p.M + ki0, p.H, p.M, p.s) == qbr &&
+           region_band(u.wx * p.M + kj0 + 8 * h, p.W, p.M, p.s) == qbc;
+    }
     const uint32_t tS = tl + r * 128 + 64 * h;  // this warp's 64 score columns
     const uint32_t tP = tl + r * 128 + 32 * h;  // its 64 bf16 P values, packed in pairs
     if (!(ok = warp_wait(&sm.s_full[r], (k / kRegions) & 1, ab, lim, SITE_FWD_SOFTMAX,
@@ -303,6 +324,7 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
       m4[q] = fmaxf(m, __uint_as_float(v[15]));
     }
     float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+    if (!kv) mx = -INFINITY;   // a masked key block adds nothing to the row maximum
     sm.red_max[j & 1][X][h][row] = mx;
     tc_fence_before();
     __syncwarp();
@@ -312,7 +334,9 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     tc_fence_after();
     mx = fmaxf(mx, sm.red_max[j & 1][X][h ^ 1][row]);
 
-    const float m_tile = mx * sl;
+    // (a key tile masked for both halves of a row leaves mx = -inf: the
+    // running maximum then stays at a finite floor, so no -inf - -inf arises)
+    const float m_tile = mask_on ? fmaxf(mx * sl, -1e30f) : mx * sl;
     float m_new = m_run, alpha = 1.f;
     bool resc = false;
     if (j == 0) {
@@ -341,7 +365,14 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
         }
         pk[e] = pack_bf16x2(p0, p1);
       }
-      tmem_st_x16(tP + c * 16, pk);
+      if (kv) {
+        tmem_st_x16(tP + c * 16, pk);
+      } else {
+        // a masked block: P = 0 exactly (its own store, so that the
+        // unmasked path carries no per-element selects)
+        const uint32_t z16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        tmem_st_x16(tP + c * 16, z16);
+      }
     }
     // the column-half-0 warp of each row pair rescales [O|L] (both halves
     // took the same decision from the same row maximum), once every PV step
@@ -416,6 +447,9 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
 }
 
 // grid (n_tiles / 2, units), block kFwdThreads, dynamic smem kFwdSmemBytes.
+// kMask: the shifted-window region mask (a separate instantiation, so that
+// the unmasked kernel carries none of its code).
+template <bool kMask>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                     const __grid_constant__ CUtensorMap tm_qp,
@@ -469,7 +503,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   if (warp < 16) {
     regs_inc<kFwdSoftmaxRegs>();
-    fwd_softmax(sm, tmem, p, u, tile0, warp >> 3, (warp >> 2) & 1, warp & 3);
+    fwd_softmax<kMask>(sm, tmem, p, u, tile0, warp >> 3, (warp >> 2) & 1, warp & 3);
   } else {
     regs_dec<kFwdServiceRegs>();
     if (warp == 16) {

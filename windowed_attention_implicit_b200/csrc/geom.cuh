@@ -33,6 +33,16 @@ __device__ __forceinline__ void tile_origin(int t, int tiles_x, int& i0, int& j0
   j0 = (t % tiles_x) * 16;
 }
 
+// Shifted-window region mask (optional; the pages describe none): on the map
+// rolled by -s, row band of rolled row y is 0 below H - M, 1 below H - s,
+// else 2 (columns alike with W).  A query attends only to keys of its own
+// (row band, column band).  Band boundaries fall on multiples of 8 (M % 16
+// and s % 8 are 0), so every 8 x 8 token block of a tile lies in one band
+// pair.  Only windows of the last window row or column hold more than one.
+__device__ __forceinline__ int region_band(int pos, int size, int M, int s) {
+  return pos < size - M ? 0 : (pos < size - s ? 1 : 2);
+}
+
 // v in [0, 2n) -> v mod n.
 __device__ __forceinline__ int wrap_once(int v, int n) { return v >= n ? v - n : v; }
 

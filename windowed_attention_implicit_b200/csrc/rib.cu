@@ -538,7 +538,7 @@ int rib_pos_tokens_bwd_noalloc(const rib_mlp_t* mlp, int window, const float* dq
 static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int head_dim,
                            int window, int shift, const void* qp_bf16, const void* kp_bf16,
                            int rank, float scale, void* out, float* lse, const void* gate,
-                           void* out_gated, void* stream) {
+                           void* out_gated, int region_mask, void* stream) {
   AttnGeom g;
   int rc = check_attn(B, H, W, heads, head_dim, window, shift, rank, &g);
   if (rc) return rc;
@@ -565,27 +565,29 @@ static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int 
   FwdParams p{};
   p.B = B; p.H = H; p.W = W; p.heads = heads; p.M = window; p.s = shift; p.rank = rank;
   p.nWx = g.nWx; p.nW = g.nW; p.tiles_x = g.tiles_x; p.n_tiles = g.n_tiles;
+  p.region_mask = region_mask != 0 && shift > 0;
   p.scale_log2 = tau * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.gate = static_cast<const __nv_bfloat16*>(gate);
   p.out_gated = static_cast<__nv_bfloat16*>(out_gated);
   p.wait_limit_ns = g_wait_limit_ns;
-  if ((rc = set_smem(attn_fwd_kernel, kFwdSmemBytes))) return rc;
+  auto* kern = p.region_mask ? attn_fwd_kernel<true> : attn_fwd_kernel<false>;
+  if ((rc = set_smem(kern, kFwdSmemBytes))) return rc;
   {
     // setmaxnreg split: only safe with the launch budget it was sized for
-    static int launch_regs = -1;
-    if (launch_regs < 0) {
+    static int launch_regs[2] = {-1, -1};
+    int& lr = launch_regs[p.region_mask ? 1 : 0];
+    if (lr < 0) {
       cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel) != cudaSuccess) return RIB_ERR_CUDA;
-      launch_regs = fa.numRegs;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return RIB_ERR_CUDA;
+      lr = fa.numRegs;
     }
-    if (launch_regs != kFwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
+    if (lr != kFwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
   }
   dim3 grid(g.n_tiles / 2, g.units);
   TraceScope ts(K_FWD, static_cast<cudaStream_t>(stream));
-  attn_fwd_kernel<<<grid, kFwdThreads, kFwdSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      tq, tqp, tkp, p);
+  kern<<<grid, kFwdThreads, kFwdSmemBytes, static_cast<cudaStream_t>(stream)>>>(tq, tqp, tkp, p);
   return launch_status();
 }
 
@@ -593,7 +595,14 @@ int rib_window_attn_fwd(const void* qkv, int B, int H, int W, int heads, int hea
                         int window, int shift, const void* qp_bf16, const void* kp_bf16,
                         int rank, float scale, void* out, float* lse, void* stream) {
   return attn_fwd_launch(qkv, B, H, W, heads, head_dim, window, shift, qp_bf16, kp_bf16, rank,
-                         scale, out, lse, nullptr, nullptr, stream);
+                         scale, out, lse, nullptr, nullptr, 0, stream);
+}
+
+int rib_window_attn_fwd_masked(const void* qkv, int B, int H, int W, int heads, int head_dim,
+                               int window, int shift, const void* qp_bf16, const void* kp_bf16,
+                               int rank, float scale, void* out, float* lse, void* stream) {
+  return attn_fwd_launch(qkv, B, H, W, heads, head_dim, window, shift, qp_bf16, kp_bf16, rank,
+                         scale, out, lse, nullptr, nullptr, 1, stream);
 }
 
 int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads, int head_dim,
@@ -602,7 +611,7 @@ int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads, int
                             float* lse, void* stream) {
   if (!gate || !out_gated) return RIB_ERR_ARG;
   return attn_fwd_launch(qkv, B, H, W, heads, head_dim, window, shift, qp_bf16, kp_bf16, rank,
-                         scale, out, lse, gate, out_gated, stream);
+                         scale, out, lse, gate, out_gated, 0, stream);
 }
 
 int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, const float* b_dw,
@@ -746,12 +755,12 @@ size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads, int head_di
   return bwd_ws_layout(B, H, W, heads, window, rank, mlp).total;
 }
 
-int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, const float* lse,
-                        int B, int H, int W, int heads, int head_dim, int window, int shift,
-                        const void* qp_bf16, const void* kp_bf16, int rank, float scale,
-                        void* dqkv, float* dqp, float* dkp, const rib_mlp_t* mlp,
-                        const rib_mlp_grad_t* dmlp, void* workspace, size_t workspace_bytes,
-                        void* stream) {
+static int attn_bwd_launch(const void* qkv, const void* out, const void* dout,
+                           const float* lse, int B, int H, int W, int heads, int head_dim,
+                           int window, int shift, const void* qp_bf16, const void* kp_bf16,
+                           int rank, float scale, void* dqkv, float* dqp, float* dkp,
+                           const rib_mlp_t* mlp, const rib_mlp_grad_t* dmlp, void* workspace,
+                           size_t workspace_bytes, int region_mask, void* stream) {
   AttnGeom g;
   int rc = check_attn(B, H, W, heads, head_dim, window, shift, rank, &g);
   if (rc) return rc;
@@ -836,6 +845,7 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
     if ((rc = launch_status())) return rc;
   }
   BwdParams p{};
+  p.region_mask = region_mask != 0 && shift > 0;
   p.B = B; p.H = H; p.W = W; p.heads = heads; p.M = window; p.s = shift; p.rank = rank;
   p.nWx = g.nWx; p.nW = g.nW; p.tiles_x = g.tiles_x; p.n_tiles = g.n_tiles;
   p.scale = tau;
@@ -844,22 +854,24 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
   p.dq_acc = a.dq_acc;
   p.dkp_part = reinterpret_cast<float*>(wsb + ws.dkp_part);
   p.wait_limit_ns = g_wait_limit_ns;
-  if ((rc = set_smem(attn_bwd_kernel, kBwdSmemBytes))) return rc;
+  auto* kern = p.region_mask ? attn_bwd_kernel<true> : attn_bwd_kernel<false>;
+  if ((rc = set_smem(kern, kBwdSmemBytes))) return rc;
   {
     // The kernel moves registers between warpgroups with setmaxnreg; that is
     // only safe if the compiled launch budget is the one the split assumes.
-    static int launch_regs = -1;
-    if (launch_regs < 0) {
+    static int launch_regs[2] = {-1, -1};
+    int& lr = launch_regs[p.region_mask ? 1 : 0];
+    if (lr < 0) {
       cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, attn_bwd_kernel) != cudaSuccess) return RIB_ERR_CUDA;
-      launch_regs = fa.numRegs;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return RIB_ERR_CUDA;
+      lr = fa.numRegs;
     }
-    if (launch_regs != kBwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
+    if (lr != kBwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
   }
   {
     TraceScope ts(K_BWD, st);
-    attn_bwd_kernel<<<dim3(g.n_tiles, g.units), kBwdThreads, kBwdSmemBytes, st>>>(
-        tq, tdo, tqp, tkp, tl, td, p);
+    kern<<<dim3(g.n_tiles, g.units), kBwdThreads, kBwdSmemBytes, st>>>(tq, tdo, tqp, tkp, tl,
+                                                                       td, p);
   }
   if ((rc = launch_status())) return rc;
   {
@@ -880,6 +892,28 @@ int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, cons
       return rc;
   }
   return RIB_OK;
+}
+
+int rib_window_attn_bwd(const void* qkv, const void* out, const void* dout, const float* lse,
+                        int B, int H, int W, int heads, int head_dim, int window, int shift,
+                        const void* qp_bf16, const void* kp_bf16, int rank, float scale,
+                        void* dqkv, float* dqp, float* dkp, const rib_mlp_t* mlp,
+                        const rib_mlp_grad_t* dmlp, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return attn_bwd_launch(qkv, out, dout, lse, B, H, W, heads, head_dim, window, shift, qp_bf16,
+                         kp_bf16, rank, scale, dqkv, dqp, dkp, mlp, dmlp, workspace,
+                         workspace_bytes, 0, stream);
+}
+
+int rib_window_attn_bwd_masked(const void* qkv, const void* out, const void* dout,
+                               const float* lse, int B, int H, int W, int heads, int head_dim,
+                               int window, int shift, const void* qp_bf16, const void* kp_bf16,
+                               int rank, float scale, void* dqkv, float* dqp, float* dkp,
+                               const rib_mlp_t* mlp, const rib_mlp_grad_t* dmlp,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_bwd_launch(qkv, out, dout, lse, B, H, W, heads, head_dim, window, shift, qp_bf16,
+                         kp_bf16, rank, scale, dqkv, dqp, dkp, mlp, dmlp, workspace,
+                         workspace_bytes, 1, stream);
 }
 
 static int window_copy(const void* src, void* dst, int B, int H, int W, int C, int eb, int M,
