@@ -156,6 +156,20 @@ def stored_traffic(kernel, workload):
     return d.get("dram_bytes_per_launch")
 
 
+def mask_line(w, ms_step, kern, f_fwd, f_bwd, peak):
+    """The training step with the shifted-window region mask (an optional
+    variant): its time and the two attention kernels' rates, counted with the
+    unmasked step's FLOPs (masked pairs still pass through the MMAs)."""
+    per = {k: v[1] / v[0] for k, v in kern.items()}
+    line = {"training_step_ms": ms_step, "kernels_ms": per,
+            "workload": f"{w.name} with the mask of shift {w.shifts[0]}"}
+    for k, f in (("attn_fwd_kernel", f_fwd), ("attn_bwd_kernel", f_bwd)):
+        if k in per:
+            line[k.replace("attn_", "").replace("_kernel", "") + "_frac"] = (
+                f / (per[k] * 1e-3) / 1e12 / peak)
+    return line
+
+
 def cla_line(w, kern_g, ms_gate_total, ms_fwd_cla_total, ms_fwd, pk, ms_cla_step_total,
              kern_cs, ms_step):
     """Convolutional local attention (measured beside the hot path, not part
@@ -338,6 +352,13 @@ def run_rib(args, w):
     def fwd_cla():
         R.rib_window_attn_fwd_cla(qkv, M, s, gate, q16, k16, out=out, out_gated=out_g, lse=lse)
 
+    # the same training step with the shifted-window region mask
+    def masked_step():
+        R.rib_pos_tokens(mlp, M, qp, kp, q16, k16)
+        R.rib_window_attn_fwd(qkv, M, s, q16, k16, out=out, lse=lse, region_mask=True)
+        R.rib_window_attn_bwd(qkv, out, dout, lse, M, s, q16, k16, mlp=mlp, dqkv=dqkv,
+                              dqp=dqp, dkp=dkp, dmlp=dmlp, workspace=ws, region_mask=True)
+
     def timed(fn, steps, trace=False):
         stream = torch.cuda.current_stream()
         if world > 1:
@@ -422,6 +443,9 @@ def run_rib(args, w):
     for _ in range(args.warmup):
         cla_step()
     ms_cs, kern_cs, _ = timed(cla_step, args.steps, trace=True)
+    for _ in range(args.warmup):
+        masked_step()
+    ms_m, kern_m, _ = timed(masked_step, args.steps, trace=True)
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
@@ -501,6 +525,7 @@ def run_rib(args, w):
                 "kernel_tflops": fwd_ach, "kernel_frac": fwd_ach / peak},
         "roofline": roof,
         "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk, ms_cs, kern_cs, ms_step),
+        "region_mask": mask_line(w, ms_m / args.steps, kern_m, f_fwd, f_bwd, peak),
         "kernels": per_kernel,
         "gpu_launches": launches,
         "cpu_baseline": cpu,
