@@ -468,10 +468,13 @@ def run_rib(args, w):
 
     e2e = None
     if not args.no_e2e:
-        # same step with the inputs copied from pinned host memory and the
-        # results read back, all inside the timed region
+        # the same step with the inputs copied from pinned host memory and the
+        # results read back, every step, all inside the timed region
         h_qkv = host["qkv"].pin_memory()
         h_dout = host["dout"].pin_memory()
+        nb = lambda t: t.numel() * t.element_size()
+
+        # (1) serialised: upload, step, read-back on one stream
         h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         h_dqkv = torch.empty(dqkv.shape, dtype=dqkv.dtype).pin_memory()
         h_flat = torch.empty(flat.shape, dtype=flat.dtype).pin_memory()
@@ -486,14 +489,90 @@ def run_rib(args, w):
 
         for _ in range(max(3, args.warmup // 2)):
             e2e_step()
-        ms_e, _, _ = timed(e2e_step, args.steps)
+        ms_serial, _, _ = timed(e2e_step, args.steps)
+
+        # (2) pipelined: uploads and read-backs on copy streams of their own,
+        # device tensors double-buffered, so step i+1's upload and step i-1's
+        # read-back overlap step i's kernels
+        b_qkv, b_dout = [qkv, torch.empty_like(qkv)], [dout, torch.empty_like(dout)]
+        b_out, b_dqkv = [out, torch.empty_like(out)], [dqkv, torch.empty_like(dqkv)]
+        b_flat = [flat, torch.empty_like(flat)]
+        b_dmlp = [dmlp]
+        views2, off2 = [], 0
+        for sh in shapes:
+            n = int(torch.Size(sh).numel())
+            views2.append(b_flat[1][off2:off2 + n].view(sh))
+            off2 += n
+        b_dmlp.append(R.PositionMLPGrad(*views2))
+        hb_out = [h_out, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
+        hb_dqkv = [h_dqkv, torch.empty(dqkv.shape, dtype=dqkv.dtype).pin_memory()]
+        hb_flat = [h_flat, torch.empty(flat.shape, dtype=flat.dtype).pin_memory()]
+        s_up, s_down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        comp = torch.cuda.current_stream()
+        ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("up", "comp", "down")}
+        used = {k: [False, False] for k in ev}
+
+        def piped_step(i):
+            bi = i % 2
+            with torch.cuda.stream(s_up):
+                if used["comp"][bi]:
+                    s_up.wait_event(ev["comp"][bi])   # step i-2 has read buffer bi
+                b_qkv[bi].copy_(h_qkv, non_blocking=True)
+                b_dout[bi].copy_(h_dout, non_blocking=True)
+                ev["up"][bi].record(s_up)
+            comp.wait_event(ev["up"][bi])
+            if used["down"][bi]:
+                comp.wait_event(ev["down"][bi])       # step i-2's results are read
+            R.rib_pos_tokens(mlp, M, qp, kp, q16, k16)
+            R.rib_window_attn_fwd(b_qkv[bi], M, s, q16, k16, out=b_out[bi], lse=lse)
+            R.rib_window_attn_bwd(b_qkv[bi], b_out[bi], b_dout[bi], lse, M, s, q16, k16,
+                                  mlp=mlp, dqkv=b_dqkv[bi], dqp=dqp, dkp=dkp,
+                                  dmlp=b_dmlp[bi], workspace=ws)
+            if world > 1:
+                dist.all_reduce(b_flat[bi])
+            ev["comp"][bi].record(comp)
+            used["comp"][bi] = True
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(ev["comp"][bi])
+                hb_out[bi].copy_(b_out[bi], non_blocking=True)
+                hb_dqkv[bi].copy_(b_dqkv[bi], non_blocking=True)
+                hb_flat[bi].copy_(b_flat[bi], non_blocking=True)
+                ev["down"][bi].record(s_down)
+            used["down"][bi] = True
+
+        def piped(steps):
+            for k in used:
+                used[k] = [False, False]
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(comp)
+            for i in range(steps):
+                piped_step(i)
+            comp.wait_event(ev["down"][(steps - 1) % 2])   # the last read-back is in
+            b.record(comp)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(b)
+            if world > 1:
+                dist.barrier()
+                tt = torch.tensor([t], device=dev)
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+                t = float(tt.item())
+            return t
+
+        piped(max(3, args.warmup // 2))
+        ms_e = piped(args.steps)
         e_step = ms_e / args.steps
-        nb = lambda t: t.numel() * t.element_size()
         e2e = {"value": world * (f_fwd + f_bwd) / (e_step * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_step,
                "tokens_per_s": world * w.tokens() / (e_step * 1e-3),
                "h2d_bytes_per_step": nb(h_qkv) + nb(h_dout),
-               "d2h_bytes_per_step": nb(h_out) + nb(h_dqkv) + nb(h_flat)}
+               "d2h_bytes_per_step": nb(h_out) + nb(h_dqkv) + nb(h_flat),
+               "pipelined": "uploads and read-backs on two copy streams, device tensors "
+                            "double-buffered; every step copies its inputs in and its "
+                            "results out",
+               "serial_ms_per_step": ms_serial / args.steps}
 
     clocks = sampler.stop() if sampler else None
     cpu = None
