@@ -47,10 +47,10 @@ constexpr int kPosThreads = 256;  // 4 threads per token
 // with the same address across the warp (broadcast).
 __host__ __device__ constexpr int pad1(int n) { return n + 1; }
 
-// Fourier features of tokens [t0, t0 + kPosTok) into g[kPosTok][pad1(4F)]
+// Fourier features of tokens [t0, t0 + kPosTok) into g[kPosTok][ld]
 // (fp64 math, fp32 store).
-__device__ __forceinline__ void fourier_tile(const PosParams& p, int t0, float* g) {
-  const int F = p.F, ld = pad1(4 * F);
+__device__ __forceinline__ void fourier_tile(const PosParams& p, int t0, float* g, int ld) {
+  const int F = p.F;
   for (int idx = threadIdx.x; idx < kPosTok * F; idx += blockDim.x) {
     const int t = idx % kPosTok, k = idx / kPosTok;
     const int tok = t0 + t;
@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   const int din = 4 * p.F, ldg = pad1(din), ldh = pad1(p.hid);
   float* g = sm_pos;                   // [kPosTok][din+1]
   float* h = g + kPosTok * ldg;        // [kPosTok][hid+1]
-  fourier_tile(p, t0, g);
+  fourier_tile(p, t0, g, ldg);
   __syncthreads();
   const int t = threadIdx.x % kPosTok, q = threadIdx.x / kPosTok;  // 4 threads per token
   const int nq = blockDim.x / kPosTok;
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
   float* h = g + T * ldg;        // [T][hid+1]  GELU(a)
   float* da = h + T * ldh;       // [T][hid+1]  dL/da
   float* go = da + T * ldh;      // [T][dout+1] dL/d(out)
-  fourier_tile(p, t0, g);
+  fourier_tile(p, t0, g, ldg);
   for (int idx = threadIdx.x; idx < T * dout; idx += blockDim.x) {
     const int o = idx / T, t = idx - o * T;
     const int tok = t0 + t;
@@ -207,6 +207,286 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
     float acc = 0.f;
     for (int t = 0; t < T; ++t) acc += go[t * ldo + o];
     o2[dout * hid + o] = acc;
+  }
+}
+
+// The same partial sums with register tiles (for hid % 8 == 0, dout % 4 ==
+// 0): each contraction runs as outer products of float4 rows, about ten
+// FMAs per load instead of one FMA per two loads.  Tile rows are padded by 4
+// floats; a thread's four tokens are t, t+16, t+32, t+48, so the 16 token
+// groups of a warp read different banks.  Every output is a sum over the
+// chunk's tokens in token order (deterministic).
+__host__ __device__ constexpr int pad4(int n) { return n + 4; }
+
+__host__ __device__ constexpr size_t mlp_bwd_tiled_smem_floats(int F, int hid, int dout) {
+  return static_cast<size_t>(kPosTok) * (pad4(4 * F) + 2 * pad4(hid) + pad4(dout));
+}
+
+__device__ __forceinline__ float f4get(const float4& v, int q) {
+  return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+
+// grid (n_chunks, 2), block kPosThreads, dynamic smem mlp_bwd_tiled_smem_floats.
+__global__ void __launch_bounds__(kPosThreads) mlp_bwd_tiled_kernel(PosParams p) {
+  extern __shared__ float4 sm_pos4[];
+  float* sm = reinterpret_cast<float*>(sm_pos4);
+  const int side = blockIdx.y;
+  const int chunk = blockIdx.x;
+  const int t0 = chunk * kPosTok;
+  const int din = 4 * p.F, hid = p.hid, dout = p.dout;
+  const int ldg = pad4(din), ldh = pad4(hid), ldo = pad4(dout);
+  constexpr int T = kPosTok;
+  float* g = sm;                 // [T][ldg]  Fourier features
+  float* h = g + T * ldg;        // [T][ldh]  GELU(a)
+  float* da = h + T * ldh;       // [T][ldh]  dL/da
+  float* go = da + T * ldh;      // [T][ldo]  dL/d(out)
+  fourier_tile(p, t0, g, ldg);
+  for (int idx = threadIdx.x; idx < T * dout; idx += blockDim.x) {
+    const int o = idx / T, t = idx - o * T;
+    const int tok = t0 + t;
+    const int head = o / p.rank, r = o - head * p.rank;
+    go[t * ldo + o] =
+        tok < p.N ? p.dtok[side][(static_cast<size_t>(head) * p.N + tok) * p.rank + r] : 0.f;
+  }
+  __syncthreads();
+  const float* w1 = p.w1[side];
+  const float* b1 = p.b1[side];
+  const float* w2 = p.w2[side];
+  // ---- a = g W1^T + b1 and dh = go W2 for tokens tg + 16 j (j < 4) and
+  // hidden units jh0 .. jh0 + 7; then h = GELU(a), da = dh * GELU'(a)
+  for (int tile = threadIdx.x; tile < 16 * (hid / 8); tile += blockDim.x) {
+    const int tg = tile % 16, jh0 = (tile / 16) * 8;
+    float acc[4][8], dh[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[j][i] = dh[j][i] = 0.f;
+    for (int k = 0; k < din; k += 4) {
+      float4 a4[4], b4[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        a4[j] = *reinterpret_cast<const float4*>(g + (tg + 16 * j) * ldg + k);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        b4[i] = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(jh0 + i) * din + k));
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[j][i] = fmaf(f4get(a4[j], q), f4get(b4[i], q), acc[j][i]);
+    }
+    for (int o = 0; o < dout; o += 4) {
+      float4 a4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        a4[j] = *reinterpret_cast<const float4*>(go + (tg + 16 * j) * ldo + o);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float* wr = w2 + static_cast<size_t>(o + q) * hid + jh0;
+        const float4 wa = __ldg(reinterpret_cast<const float4*>(wr));
+        const float4 wb = __ldg(reinterpret_cast<const float4*>(wr + 4));
+        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dh[j][i] = fmaf(f4get(a4[j], q), wv[i], dh[j][i]);
+      }
+    }
+    float bias[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bias[i] = __ldg(b1 + jh0 + i);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float hv[8], dv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float a = acc[j][i] + bias[i];
+        hv[i] = gelu_erf(a);
+        dv[i] = dh[j][i] * gelu_erf_grad(a);   // tokens past N have go == 0
+      }
+      float4* hr = reinterpret_cast<float4*>(h + (tg + 16 * j) * ldh + jh0);
+      float4* dr = reinterpret_cast<float4*>(da + (tg + 16 * j) * ldh + jh0);
+      hr[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+      hr[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
+      dr[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+      dr[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+    }
+  }
+  __syncthreads();
+  float* out = p.partial + (static_cast<size_t>(side) * p.n_chunks + chunk) * p.n_params;
+  // ---- dw1[jh][k] = sum_t da[t][jh] g[t][k]: tiles of 8 jh x 4 k
+  for (int tile = threadIdx.x; tile < (hid / 8) * (din / 4); tile += blockDim.x) {
+    const int k0 = 4 * (tile % (din / 4)), jh0 = (tile / (din / 4)) * 8;
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+    for (int t = 0; t < T; ++t) {
+      const float4 d0 = *reinterpret_cast<const float4*>(da + t * ldh + jh0);
+      const float4 d1 = *reinterpret_cast<const float4*>(da + t * ldh + jh0 + 4);
+      const float4 gv = *reinterpret_cast<const float4*>(g + t * ldg + k0);
+      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[i][0] = fmaf(dv[i], gv.x, acc[i][0]);
+        acc[i][1] = fmaf(dv[i], gv.y, acc[i][1]);
+        acc[i][2] = fmaf(dv[i], gv.z, acc[i][2]);
+        acc[i][3] = fmaf(dv[i], gv.w, acc[i][3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<float4*>(out + static_cast<size_t>(jh0 + i) * din + k0) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+  }
+  for (int jh = threadIdx.x; jh < hid; jh += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc += da[t * ldh + jh];
+    out[hid * din + jh] = acc;
+  }
+  float* o2 = out + hid * din + hid;
+  // ---- dw2[o][jh] = sum_t go[t][o] h[t][jh]: tiles of 4 o x 8 jh
+  for (int tile = threadIdx.x; tile < (dout / 4) * (hid / 8); tile += blockDim.x) {
+    const int jh0 = 8 * (tile % (hid / 8)), o0 = (tile / (hid / 8)) * 4;
+    float acc[4][8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[q][i] = 0.f;
+    for (int t = 0; t < T; ++t) {
+      const float4 gv = *reinterpret_cast<const float4*>(go + t * ldo + o0);
+      const float4 h0 = *reinterpret_cast<const float4*>(h + t * ldh + jh0);
+      const float4 h1 = *reinterpret_cast<const float4*>(h + t * ldh + jh0 + 4);
+      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[0][i] = fmaf(gv.x, hv[i], acc[0][i]);
+        acc[1][i] = fmaf(gv.y, hv[i], acc[1][i]);
+        acc[2][i] = fmaf(gv.z, hv[i], acc[2][i]);
+        acc[3][i] = fmaf(gv.w, hv[i], acc[3][i]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float4* dst = reinterpret_cast<float4*>(o2 + static_cast<size_t>(o0 + q) * hid + jh0);
+      dst[0] = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+      dst[1] = make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]);
+    }
+  }
+  for (int o = threadIdx.x; o < dout; o += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc += go[t * ldo + o];
+    o2[dout * hid + o] = acc;
+  }
+}
+
+// Position tokens with register tiles (hid % 8 == 0, rank % 8 == 0): the
+// two Linear layers as outer products of float4 rows, tiles of 4 tokens
+// (t, t+16, t+32, t+48) x 8 units.
+__host__ __device__ constexpr size_t pos_tiled_smem_floats(int F, int hid) {
+  return static_cast<size_t>(kPosTok) * (pad4(4 * F) + pad4(hid));
+}
+
+// grid (ceil(N / kPosTok), 2), block kPosThreads, dynamic smem pos_tiled_smem_floats.
+__global__ void __launch_bounds__(kPosThreads) pos_tokens_tiled_kernel(PosParams p) {
+  extern __shared__ float4 sm_pos4[];
+  float* sm = reinterpret_cast<float*>(sm_pos4);
+  const int side = blockIdx.y;
+  const int t0 = blockIdx.x * kPosTok;
+  const int din = 4 * p.F, hid = p.hid, dout = p.dout;
+  const int ldg = pad4(din), ldh = pad4(hid);
+  float* g = sm;                   // [kPosTok][ldg]
+  float* h = g + kPosTok * ldg;    // [kPosTok][ldh]
+  fourier_tile(p, t0, g, ldg);
+  __syncthreads();
+  const float* w1 = p.w1[side];
+  const float* b1 = p.b1[side];
+  const float* w2 = p.w2[side];
+  const float* b2 = p.b2[side];
+  // h = GELU(g W1^T + b1)
+  for (int tile = threadIdx.x; tile < 16 * (hid / 8); tile += blockDim.x) {
+    const int tg = tile % 16, jh0 = (tile / 16) * 8;
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[j][i] = 0.f;
+    for (int k = 0; k < din; k += 4) {
+      float4 a4[4], b4[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        a4[j] = *reinterpret_cast<const float4*>(g + (tg + 16 * j) * ldg + k);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        b4[i] = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(jh0 + i) * din + k));
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[j][i] = fmaf(f4get(a4[j], q), f4get(b4[i], q), acc[j][i]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float hv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hv[i] = gelu_erf(acc[j][i] + __ldg(b1 + jh0 + i));
+      float4* hr = reinterpret_cast<float4*>(h + (tg + 16 * j) * ldh + jh0);
+      hr[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+      hr[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
+    }
+  }
+  __syncthreads();
+  // out = h W2^T + b2; 8 consecutive outputs lie in one head (rank % 8 == 0)
+  for (int tile = threadIdx.x; tile < 16 * (dout / 8); tile += blockDim.x) {
+    const int tg = tile % 16, o0 = (tile / 16) * 8;
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[j][i] = 0.f;
+    for (int k = 0; k < hid; k += 4) {
+      float4 a4[4], b4[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        a4[j] = *reinterpret_cast<const float4*>(h + (tg + 16 * j) * ldh + k);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        b4[i] = __ldg(reinterpret_cast<const float4*>(w2 + static_cast<size_t>(o0 + i) * hid + k));
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[j][i] = fmaf(f4get(a4[j], q), f4get(b4[i], q), acc[j][i]);
+    }
+    const int head = o0 / p.rank, r0 = o0 - head * p.rank;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tok = t0 + tg + 16 * j;
+      if (tok >= p.N) continue;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = acc[j][i] + __ldg(b2 + o0 + i);
+      const size_t off = (static_cast<size_t>(head) * p.N + tok) * p.rank + r0;
+      float4* d32 = reinterpret_cast<float4*>(p.out32[side] + off);
+      d32[0] = make_float4(v[0], v[1], v[2], v[3]);
+      d32[1] = make_float4(v[4], v[5], v[6], v[7]);
+      if (p.out16[side]) {
+        uint32_t u[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 b2v = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+          u[e] = *reinterpret_cast<const uint32_t*>(&b2v);
+        }
+        *reinterpret_cast<uint4*>(p.out16[side] + off) = make_uint4(u[0], u[1], u[2], u[3]);
+      }
+    }
   }
 }
 

@@ -272,13 +272,22 @@ int launch_mlp_bwd(const rib_mlp_t* mlp, int window, const float* dqp, const flo
   pp.grads[0][2] = dmlp->q_dw2; pp.grads[0][3] = dmlp->q_db2;
   pp.grads[1][0] = dmlp->k_dw1; pp.grads[1][1] = dmlp->k_db1;
   pp.grads[1][2] = dmlp->k_dw2; pp.grads[1][3] = dmlp->k_db2;
-  const size_t smem = mlp_bwd_smem_floats(pp.F, pp.hid, pp.dout) * sizeof(float);
+  // register-tiled partial sums where the shapes and the weights' alignment
+  // allow float4 rows, else the general kernel
+  const size_t smem_t = mlp_bwd_tiled_smem_floats(pp.F, pp.hid, pp.dout) * sizeof(float);
+  const bool tiled = pp.hid % 8 == 0 && pp.dout % 4 == 0 && smem_t <= 200 * 1024 &&
+                     aligned16(pp.w1[0]) && aligned16(pp.w1[1]) && aligned16(pp.w2[0]) &&
+                     aligned16(pp.w2[1]);
+  const size_t smem = tiled ? smem_t : mlp_bwd_smem_floats(pp.F, pp.hid, pp.dout) * sizeof(float);
   if (smem > 200 * 1024) return RIB_ERR_UNSUPPORTED;
   int rc;
-  if ((rc = set_smem(mlp_bwd_partial_kernel, smem))) return rc;
+  if ((rc = set_smem(tiled ? mlp_bwd_tiled_kernel : mlp_bwd_partial_kernel, smem))) return rc;
   {
     TraceScope ts(K_MLP_PART, st);
-    mlp_bwd_partial_kernel<<<dim3(n_chunks, 2), kPosThreads, smem, st>>>(pp);
+    if (tiled)
+      mlp_bwd_tiled_kernel<<<dim3(n_chunks, 2), kPosThreads, smem, st>>>(pp);
+    else
+      mlp_bwd_partial_kernel<<<dim3(n_chunks, 2), kPosThreads, smem, st>>>(pp);
   }
   if ((rc = launch_status())) return rc;
   {
@@ -480,12 +489,21 @@ int rib_pos_tokens(const rib_mlp_t* mlp, int window, float* qp, float* kp, void*
   p.out32[1] = kp;
   p.out16[0] = static_cast<__nv_bfloat16*>(qp_bf16);
   p.out16[1] = static_cast<__nv_bfloat16*>(kp_bf16);
-  const size_t smem = pos_fwd_smem_floats(p.F, p.hid) * sizeof(float);
+  // register-tiled MLP where the shapes and alignments allow float4 rows
+  const size_t smem_t = pos_tiled_smem_floats(p.F, p.hid) * sizeof(float);
+  const bool tiled = p.hid % 8 == 0 && p.rank % 8 == 0 && smem_t <= 200 * 1024 &&
+                     aligned16(p.w1[0]) && aligned16(p.w1[1]) && aligned16(p.w2[0]) &&
+                     aligned16(p.w2[1]) && aligned16(qp) && aligned16(kp) &&
+                     (!qp_bf16 || aligned16(qp_bf16)) && (!kp_bf16 || aligned16(kp_bf16));
+  const size_t smem = tiled ? smem_t : pos_fwd_smem_floats(p.F, p.hid) * sizeof(float);
   if (smem > 200 * 1024) return RIB_ERR_UNSUPPORTED;
-  if ((rc = set_smem(pos_tokens_kernel, smem))) return rc;
+  if ((rc = set_smem(tiled ? pos_tokens_tiled_kernel : pos_tokens_kernel, smem))) return rc;
   dim3 grid((p.N + kPosTok - 1) / kPosTok, 2);
   TraceScope ts(K_POS, static_cast<cudaStream_t>(stream));
-  pos_tokens_kernel<<<grid, kPosThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  if (tiled)
+    pos_tokens_tiled_kernel<<<grid, kPosThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  else
+    pos_tokens_kernel<<<grid, kPosThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
   return launch_status();
 }
 
