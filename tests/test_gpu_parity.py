@@ -35,6 +35,32 @@ def test_pos_tokens_parity(M, strong):
     assert torch.equal(k16.cpu(), kp.cpu().to(torch.bfloat16))
 
 
+# Shapes for both kernel forms: the register-tiled one (hid % 8 == 0,
+# rank % 8 == 0) and the general one (the other shapes).
+MLP_SHAPES = [  # heads, rank, hid, F
+    (4, 12, 60, 16),    # general: hid and rank not multiples of 8
+    (3, 6, 36, 8),      # general
+    (2, 8, 64, 5),      # tiled, 20 Fourier inputs
+    (1, 16, 8, 1),      # tiled, smallest
+]
+
+
+@pytest.mark.parametrize("heads,rank,hid,F", MLP_SHAPES)
+def test_pos_tokens_parity_both_kernel_forms(heads, rank, hid, F):
+    M = 12
+    freqs = I.default_freqs(F)
+    mq = I.make_mlp(F, hid, heads, rank, 31, 0, strong=True)
+    mk = I.make_mlp(F, hid, heads, rank, 31, 1, strong=True)
+    mlp = R.PositionMLP.from_params(freqs, mq, mk, heads, rank)
+    qp, kp, q16, k16 = R.rib_pos_tokens(mlp, M)
+    torch.cuda.synchronize()
+    rq, rk = O.pos_tokens(freqs, mq, mk, M, heads, rank)
+    for got, ref, name in ((qp, rq, "qp"), (kp, rk, "kp")):
+        rel = np.abs(to_np(got) - ref).max() / np.abs(ref).max()
+        assert rel <= POS_REL, f"{name}: rel {rel:.3e}"
+    assert torch.equal(q16.cpu(), qp.cpu().to(torch.bfloat16))
+
+
 # ---------------------------------------------------------------- gather/scatter
 
 @pytest.mark.parametrize("B,H,W,C,dtype,M,s", [
@@ -168,6 +194,27 @@ def test_pos_tokens_bwd_parity(M, hid):
             got = to_np(getattr(dm, f"{side}_{name}"))
             rel = np.abs(got - r).max() / np.abs(r).max()
             print(f"{side}_{name}: rel {rel:.3e}")
+            if rel > MLP_REL:
+                bad.append(f"{side}_{name} rel {rel:.3e}")
+    assert not bad, bad
+
+
+@pytest.mark.parametrize("heads,rank,hid,F", MLP_SHAPES)
+def test_pos_tokens_bwd_parity_both_kernel_forms(heads, rank, hid, F):
+    M = 20   # 400 tokens: seven chunks of 64, the last one partial
+    freqs = I.default_freqs(F)
+    mq = I.make_mlp(F, hid, heads, rank, 37, 0, strong=True)
+    mk = I.make_mlp(F, hid, heads, rank, 37, 1, strong=True)
+    mlp = R.PositionMLP.from_params(freqs, mq, mk, heads, rank)
+    gq = I.randn((heads, M, M, rank), seed=M, tag=7)
+    gk = I.randn((heads, M, M, rank), seed=M, tag=8)
+    dm = R.rib_pos_tokens_bwd(mlp, M, gq.cuda(), gk.cuda())
+    torch.cuda.synchronize()
+    (rq, rk) = O.pos_tokens_backward(freqs, mq, mk, M, gq.double().numpy(), gk.double().numpy())
+    bad = []
+    for side, ref in (("q", rq), ("k", rk)):
+        for name, r in zip(("dw1", "db1", "dw2", "db2"), ref):
+            rel = np.abs(to_np(getattr(dm, f"{side}_{name}")) - r).max() / np.abs(r).max()
             if rel > MLP_REL:
                 bad.append(f"{side}_{name} rel {rel:.3e}")
     assert not bad, bad
