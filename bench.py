@@ -156,6 +156,41 @@ def stored_traffic(kernel, workload):
     return d.get("dram_bytes_per_launch")
 
 
+def copy_line(kern_ga, kern_sc, x_map, pk):
+    """rib_window_gather / rib_window_scatter of the qkv map: each call reads
+    and writes the whole map once (bf16), against the measured HBM copy."""
+    byt = 2 * x_map.numel() * x_map.element_size()
+    ga = kern_ga["window_copy_kernel"]
+    sc = kern_sc["window_copy_kernel"]
+    g_ms, s_ms = ga[1] / ga[0], sc[1] / sc[0]
+    return {"kernel": "window_copy_kernel", "bound": "hbm", "bytes_per_call": byt,
+            "gather_ms": g_ms, "scatter_ms": s_ms,
+            "gather_gbs": byt / (g_ms * 1e-3) / 1e9, "scatter_gbs": byt / (s_ms * 1e-3) / 1e9,
+            "gather_frac_hbm": byt / (g_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "scatter_frac_hbm": byt / (s_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "map": list(x_map.shape)}
+
+
+def pos_line(w, per_kernel, pk):
+    """The position-token kernel inside the step: both MLPs over the M*M
+    window tokens.  FMA-bound: FLOPs of the two Linear layers per token and
+    MLP, against the fp32 FMA rate of 148 SMs x 128 lanes x 2 at the measured
+    clock; bytes written (Qp, Kp in fp32 and bf16) as its HBM figure."""
+    k = per_kernel.get("pos_tokens_kernel")
+    if k is None:
+        return None
+    N = w.windows[0] ** 2
+    din, out = 4 * w.n_freq, w.heads * w.rank
+    flops = 2 * N * 2 * (din * w.hidden + w.hidden * out)
+    byt = 2 * N * out * (4 + 2)
+    t = k["avg_ms"] * 1e-3
+    fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    return {"kernel_ms": k["avg_ms"], "bound": "fma", "flops": flops,
+            "tflops_fp32": flops / t / 1e12, "fma_peak_tflops": fma_peak,
+            "frac_fma": flops / t / 1e12 / fma_peak, "bytes_written": byt,
+            "gbs": byt / t / 1e9}
+
+
 def mask_line(w, ms_step, kern, f_fwd, f_bwd, peak):
     """The training step with the shifted-window region mask (an optional
     variant): its time and the two attention kernels' rates, counted with the
@@ -446,6 +481,25 @@ def run_rib(args, w):
     for _ in range(args.warmup):
         masked_step()
     ms_m, kern_m, _ = timed(masked_step, args.steps, trace=True)
+
+    # the window gather / scatter of the workload's qkv map (the partition
+    # with cyclic shift as a standalone TMA copy), against the HBM roofline
+    C3 = 3 * heads * d
+    x_map = qkv.view(B, H, W, C3)
+    xw = torch.empty((B, (H // M) * (W // M), M * M, C3), device=dev, dtype=torch.bfloat16)
+    x_back = torch.empty_like(x_map)
+
+    def gather_only():
+        R.rib_window_gather(x_map, M, s, out=xw)
+
+    def scatter_only():
+        R.rib_window_scatter(xw, H, W, M, s, out=x_back)
+
+    for _ in range(args.warmup):
+        gather_only()
+        scatter_only()
+    _, kern_ga, _ = timed(gather_only, args.steps, trace=True)
+    _, kern_sc, _ = timed(scatter_only, args.steps, trace=True)
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
@@ -605,6 +659,8 @@ def run_rib(args, w):
         "roofline": roof,
         "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk, ms_cs, kern_cs, ms_step),
         "region_mask": mask_line(w, ms_m / args.steps, kern_m, f_fwd, f_bwd, peak),
+        "gather": copy_line(kern_ga, kern_sc, x_map, pk),
+        "pos_tokens": pos_line(w, per_kernel, pk),
         "kernels": per_kernel,
         "gpu_launches": launches,
         "cpu_baseline": cpu,
