@@ -156,6 +156,25 @@ def stored_traffic(kernel, workload):
     return d.get("dram_bytes_per_launch")
 
 
+def infer_line(wi, ms_pass, kern, steps, world, peak):
+    """The 12-layer forward pass of the large-image inference workload."""
+    M = wi.windows[0]
+    N = M * M
+    units = wi.batch * (wi.height // M) * (wi.width // M) * wi.heads
+    f_layer = 160.0 * N * N * units
+    fwd = kern.get("attn_fwd_kernel", (1, 0.0))
+    k_ms = fwd[1] / max(fwd[0], 1)
+    return {"workload": f"{wi.name}: B={wi.batch} {wi.height}x{wi.width} map, {M}x{M} windows, "
+                        f"{wi.layers} layers, shifts {'/'.join(str(x) for x in wi.shifts[:2])}, "
+                        "forward only, Qp/Kp computed once and reused",
+            "ms_per_pass": ms_pass,
+            "tflops": world * wi.layers * f_layer / (ms_pass * 1e-3) / 1e12,
+            "tokens_per_s": world * wi.layers * wi.batch * wi.height * wi.width / (ms_pass * 1e-3),
+            "fwd_kernel_ms": k_ms,
+            "fwd_kernel_frac": f_layer / (k_ms * 1e-3) / 1e12 / peak if k_ms else None,
+            "pos_tokens_launches_per_pass": kern.get("pos_tokens_kernel", (0, 0.0))[0] / steps}
+
+
 def copy_line(kern_ga, kern_sc, x_map, pk):
     """rib_window_gather / rib_window_scatter of the qkv map: each call reads
     and writes the whole map once (bf16), against the measured HBM copy."""
@@ -500,6 +519,28 @@ def run_rib(args, w):
         scatter_only()
     _, kern_ga, _ = timed(gather_only, args.steps, trace=True)
     _, kern_sc, _ = timed(scatter_only, args.steps, trace=True)
+    del xw, x_back
+
+    # large-image inference: 12 forward layers (shifts alternating 0 / M/2)
+    # over a 576 x 384 map, Qp/Kp computed once and reused by every window
+    # and layer (the stack's geometry cache)
+    from windowed_attention_implicit_b200.schedule import LayerSpec, RIBLayerStack
+    wi = I.get_workload("w96infer", seed=I.get_workload("w96infer").seed + 7919 * rank)
+    inp0 = I.make_layer_inputs(wi, 0, with_dout=False)
+    mlp_i = R.PositionMLP.from_params(inp0["freqs"], inp0["mlp_q"], inp0["mlp_k"], wi.heads,
+                                      wi.rank, device=dev)
+    stack = RIBLayerStack([LayerSpec(wi.windows[l], wi.shifts[l], mlp_i)
+                           for l in range(wi.layers)])
+    qkvs = [inp0["qkv"].to(dev)] + [I.make_layer_inputs(wi, l, with_dout=False)["qkv"].to(dev)
+                                    for l in range(1, wi.layers)]
+
+    def infer_pass():
+        stack.forward(qkvs)
+
+    for _ in range(args.warmup):
+        infer_pass()
+    ms_inf, kern_inf, _ = timed(infer_pass, args.steps, trace=True)
+    del qkvs
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
@@ -660,6 +701,7 @@ def run_rib(args, w):
         "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk, ms_cs, kern_cs, ms_step),
         "region_mask": mask_line(w, ms_m / args.steps, kern_m, f_fwd, f_bwd, peak),
         "gather": copy_line(kern_ga, kern_sc, x_map, pk),
+        "inference": infer_line(wi, ms_inf / args.steps, kern_inf, args.steps, world, peak),
         "pos_tokens": pos_line(w, per_kernel, pk),
         "kernels": per_kernel,
         "gpu_launches": launches,
