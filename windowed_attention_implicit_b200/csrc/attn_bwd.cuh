@@ -33,25 +33,28 @@
 // that no group's waits hold back another's.  The compute warps neither
 // drain dQ (dedicated warps do) nor wait for the previous tile's gradient
 // MMAs before their exponentials (they form the whole tile in registers
-// first, then wait for the P^T/dS^T buffers).
+// first, then wait for the P^T buffer).
 // Per query tile i:  S^T = K_aug Q_aug^T and dP^T = V dO^T (MMA, TMEM) ->
-// compute warps form P^T and dS^T (to TMEM) and dS (to shared memory,
-// core-matrix layout, double-buffered) -> MMA: dV += P^T dO and
-// dK_aug += dS^T [Qc|Qp] (A from TMEM), dQ_aug = dS [Kc|Kp] (A from shared
-// memory) -> drain warps fold dQ into the fp32 accumulator with one bulk
-// reduce-add per tile (per-thread vector atomics cost more L2 time than the
-// whole rest of the kernel).
+// compute warps form P^T (to TMEM) and dS (to shared memory as 8 x 8 core
+// matrices, double-buffered) -> MMA: dV += P^T dO (A from TMEM),
+// dK_aug += dS^T [Qc|Qp] (A = the dS core matrices read K-major) and
+// dQ_aug = dS [Kc|Kp] (A = the same core matrices read MN-major) -> drain
+// warps fold dQ into the fp32 accumulator with one bulk reduce-add per tile
+// (per-thread vector atomics cost more L2 time than the whole rest of the
+// kernel).
 // At d = 32 the MMAs are narrow: a tcgen05.mma of M=128, K=16 costs ~40-50
 // cycles however small N is, and with both operands in shared memory an
-// N <= 64 MMA moves more bytes than its flops cover.  So the A operand comes
-// from TMEM wherever the lane layout allows (P^T, dS^T), the positional
+// N <= 64 MMA moves more bytes than its flops cover.  So P^T, the A of the
+// dV MMA, comes from TMEM; dS^T is read from the shared dS tile instead (a
+// TMEM copy would cost the compute warps a store per element), the positional
 // tiles are fetched zero-padded to 32 channels (TMA fills the out-of-bounds
 // half with zeros) so that [Qc|Qp] and [Kc|Kp] form one N=48 B operand of two
 // 64B-swizzle atoms, and dK_aug, dQ_aug are one MMA chain each (29 MMAs per
 // tile).  S/dP of tile i+1 are issued as soon as the compute warps have
-// pulled tile i into registers; P^T/dS^T are released right after the dV/dK
-// MMAs and dS is double-buffered, so the compute warps rarely wait on the
-// gradient MMAs of the previous tile.  Exponentials are split between MUFU
+// pulled tile i into registers; P^T is released right after the dV/dK MMAs
+// and dS is double-buffered, so the compute warps never wait on the
+// gradient MMAs of the previous tile (what they do wait on is the latency
+// of testing barriers that are already complete).  Exponentials are split between MUFU
 // and the FMA pipe (exp2_fma2), with packed f32x2 arithmetic.
 #pragma once
 
@@ -69,8 +72,8 @@ static_assert(2 * 128 * kBwdComputeRegs + 2 * 128 * kBwdServiceRegs <=
                   kBwdThreads * kBwdLaunchRegs,
               "register split exceeds the launch budget");
 constexpr uint32_t kBwdTmemCols = 512;
-// TMEM columns (512): S^T, dP^T fp32; P^T, dS^T bf16; dV; dK = [dKc | dKp];
-// dQ = [dQc | dQp]
+// TMEM columns (512): S^T, dP^T fp32; P^T bf16; (dS^T bf16, used only when
+// RIB_BWD_DK_SMEM is 0); dV; dK = [dKc | dKp]; dQ = [dQc | dQp]
 constexpr uint32_t kBColS = 0, kBColDP = 128, kBColP = 256, kBColDST = 320, kBColDV = 384,
                    kBColDK = 416, kBColDQ = 464;
 // Of every 8 element pairs, how many exponentials run on the FMA pipe.  The
