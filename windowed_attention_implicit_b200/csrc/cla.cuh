@@ -19,7 +19,8 @@
 //   warp 1       TMEM allocator; issues the point-wise convolution as C/16
 //                tcgen05.mma steps (M = 128 pixels, N = C, K = C), W_pw
 //                having been rounded to bf16 into shared memory once per CTA
-//   warps 2-9    depth-wise 3x3 in fp32 from the halo (lane = channel pair),
+//   warps 2-9    depth-wise 3x3 in fp32 from the halo (lane = channel quad
+//                of one of two neighbouring pixels),
 //                y written as bf16 into one of two A tiles in the canonical
 //                no-swizzle K-major core-matrix layout
 //   warps 10-17  epilogue: accumulator (one of two in tensor memory) + b_pw,
@@ -205,38 +206,37 @@ __global__ void __launch_bounds__(kClaThreads, 1)
       for (int g = 0; g < chunks; ++g, ++q) {
         const int st = q & 1;
         if (!(ok = warp_wait(&bb.halo_full[st], (q >> 1) & 1, ab, lim, SITE_CLA))) break;
-        const int c = g * 64 + 2 * lane;
+        // lane = (channel quad cq of the chunk, pixel parity pp): 16 lanes read
+        // one pixel's 128 bytes, the warp two neighbouring pixels at a time
+        const int cq = lane & 15, pp = lane >> 4;
+        const int c = g * 64 + 4 * cq;
         if (c < C) {
-          float w0[9], w1[9];
+          float4 w4[9];
 #pragma unroll
-          for (int tp = 0; tp < 9; ++tp) {
-            const float2 wv = *reinterpret_cast<const float2*>(sWdw + tp * C + c);
-            w0[tp] = wv.x;
-            w1[tp] = wv.y;
-          }
-          const float bias0 = sBdw[c], bias1 = sBdw[c + 1];
-          const uint8_t* h = sH(st) + lane * 4;   // halo [10 rows][18 cols][64 ch]
-#pragma unroll 4
-          for (int r = dw; r < 128; r += kClaDwWarps) {
+          for (int tp = 0; tp < 9; ++tp) w4[tp] = *reinterpret_cast<const float4*>(sWdw + tp * C + c);
+          const float4 b4 = *reinterpret_cast<const float4*>(sBdw + c);
+          const uint8_t* h = sH(st) + cq * 8;     // halo [10 rows][18 cols][64 ch]
+#pragma unroll 2
+          for (int m = 0; m < 128 / (2 * kClaDwWarps); ++m) {
+            const int r = 2 * (dw + kClaDwWarps * m) + pp;
             const int i = r >> 4, j = r & 15;     // tile-local; halo row i+u, col j+v
-            // two partial sums per channel shorten the dependent FMA chains
-            float a0 = bias0, a1 = bias1, e0 = 0.f, e1 = 0.f;
+            float a0 = b4.x, a1 = b4.y, a2 = b4.z, a3 = b4.w;
 #pragma unroll
             for (int u = 0; u < 3; ++u)
 #pragma unroll
               for (int v = 0; v < 3; ++v) {
-                const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
-                    h + ((i + u) * 18 + (j + v)) * 128));
-                if ((u * 3 + v) & 1) {
-                  e0 = fmaf(w0[u * 3 + v], xf.x, e0);
-                  e1 = fmaf(w1[u * 3 + v], xf.y, e1);
-                } else {
-                  a0 = fmaf(w0[u * 3 + v], xf.x, a0);
-                  a1 = fmaf(w1[u * 3 + v], xf.y, a1);
-                }
+                const uint2 xv =
+                    *reinterpret_cast<const uint2*>(h + ((i + u) * 18 + (j + v)) * 128);
+                const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv.x));
+                const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv.y));
+                const float4 w = w4[u * 3 + v];
+                a0 = fmaf(w.x, x01.x, a0);
+                a1 = fmaf(w.y, x01.y, a1);
+                a2 = fmaf(w.z, x23.x, a2);
+                a3 = fmaf(w.w, x23.y, a3);
               }
-            *reinterpret_cast<uint32_t*>(sA(s) + cla_kmajor_offset(r, c, C)) =
-                pack_bf16x2(a0 + e0, a1 + e1);
+            *reinterpret_cast<uint2*>(sA(s) + cla_kmajor_offset(r, c, C)) =
+                make_uint2(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3));
           }
         }
         __syncwarp();
