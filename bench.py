@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--workload", default="w96train")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the table of every workload definition")
     ap.add_argument("--step-only", action="store_true",
                     help="run only warm-up + timed training steps (for profiler launch lists)")
     ap.add_argument("--cla-only", action="store_true",
@@ -154,6 +156,78 @@ def stored_traffic(kernel, workload):
     if d.get("source_hash") != kernel_source_hash():
         return None
     return d.get("dram_bytes_per_launch")
+
+
+def config_sweep(I, R, dev, rank, world, timed, steps, warmup, peak, pk):
+    """Every workload definition through the public API: the forward of all
+    its layers (position tokens cached per geometry) and, for the training
+    ones, the training step (position tokens, forward, backward with the MLP
+    gradients, per layer).  Algorithmic FLOPs: 160 N^2 (fwd) and 416 N^2 (bwd)
+    per unit; tokens = B*H*W per layer."""
+    import torch
+    from windowed_attention_implicit_b200.schedule import LayerSpec, RIBLayerStack
+    res = {}
+    for name in ("tiny", "w32", "cyclic", "w96train", "w96infer"):
+        w0 = I.get_workload(name)
+        w = I.get_workload(name, seed=w0.seed + 7919 * rank)
+        layers = []
+        for l in range(w.layers):
+            inp = I.make_layer_inputs(w, l, with_dout=w.backward)
+            mlp = R.PositionMLP.from_params(inp["freqs"], inp["mlp_q"], inp["mlp_k"], w.heads,
+                                            w.rank, device=dev)
+            layers.append((inp["qkv"].to(dev), inp["dout"].to(dev) if w.backward else None, mlp))
+        if w.shared_mlp:
+            layers = [(q, g, layers[0][2]) for q, g, _ in layers]
+        specs = [LayerSpec(w.windows[l], w.shifts[l], layers[l][2]) for l in range(w.layers)]
+        stack = RIBLayerStack(specs)
+        qkvs = [q for q, _, _ in layers]
+        f_fwd = sum(160.0 * (w.windows[l] ** 2) ** 2 * w.units(l) for l in range(w.layers))
+        f_bwd = sum(416.0 * (w.windows[l] ** 2) ** 2 * w.units(l) for l in range(w.layers))
+        tok = w.layers * w.tokens()
+
+        def fwd_pass():
+            stack.forward(qkvs)
+
+        for _ in range(warmup):
+            fwd_pass()
+        ms_f, kern_f, _ = timed(fwd_pass, steps, trace=True)
+        ms_f /= steps
+        line = {"layers": w.layers, "windows": list(w.windows), "shifts": list(w.shifts),
+                "map": [w.batch, w.height, w.width], "heads": w.heads,
+                "fwd_ms": ms_f, "fwd_tflops": world * f_fwd / (ms_f * 1e-3) / 1e12,
+                "fwd_tokens_per_s": world * tok / (ms_f * 1e-3),
+                "fwd_frac_sustained": f_fwd / (ms_f * 1e-3) / 1e12 / peak}
+        if w.backward:
+            ws = {}
+
+            def train_step():
+                for l, (qkv, dout, mlp) in enumerate(layers):
+                    M, sh = w.windows[l], w.shifts[l]
+                    _, _, q16, k16 = R.rib_pos_tokens(mlp, M)
+                    out, lse = R.rib_window_attn_fwd(qkv, M, sh, q16, k16)
+                    if l not in ws:
+                        ws[l] = torch.empty(max(R.rib_window_attn_bwd_workspace(
+                            w.batch, w.height, w.width, w.heads, w.head_dim, M, w.rank,
+                            mlp if w.mlp_grads else None), 256), device=dev, dtype=torch.uint8)
+                    R.rib_window_attn_bwd(qkv, out, dout, lse, M, sh, q16, k16,
+                                          mlp=mlp if w.mlp_grads else None, workspace=ws[l])
+
+            for _ in range(warmup):
+                train_step()
+            ms_t, _, _ = timed(train_step, steps)
+            ms_t /= steps
+            line.update({"step_ms": ms_t,
+                         "step_tflops": world * (f_fwd + f_bwd) / (ms_t * 1e-3) / 1e12,
+                         "step_tokens_per_s": world * tok / (ms_t * 1e-3),
+                         "step_frac_sustained": (f_fwd + f_bwd) / (ms_t * 1e-3) / 1e12 / peak})
+        # bytes of one forward (qkv read, out written, lse written) against HBM
+        byt = w.layers * w.tokens() * w.heads * (3 * 64 + 64 + 4)
+        line["fwd_gbs"] = byt / (ms_f * 1e-3) / 1e9
+        line["fwd_frac_hbm"] = line["fwd_gbs"] / pk["hbm_gbs"]
+        res[name] = line
+        del layers, qkvs, stack
+        torch.cuda.empty_cache()
+    return res
 
 
 def infer_line(wi, ms_pass, kern, steps, world, peak):
@@ -540,7 +614,10 @@ def run_rib(args, w):
     for _ in range(args.warmup):
         infer_pass()
     ms_inf, kern_inf, _ = timed(infer_pass, args.steps, trace=True)
-    del qkvs
+    del qkvs, stack
+    pk_s = peaks()
+    sweep = config_sweep(I, R, dev, rank, world, timed, min(args.steps, 10), args.warmup,
+                         pk_s["bf16_tflops_sustained"], pk_s) if not args.no_sweep else None
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
@@ -702,6 +779,7 @@ def run_rib(args, w):
         "region_mask": mask_line(w, ms_m / args.steps, kern_m, f_fwd, f_bwd, peak),
         "gather": copy_line(kern_ga, kern_sc, x_map, pk),
         "inference": infer_line(wi, ms_inf / args.steps, kern_inf, args.steps, world, peak),
+        "configs": sweep,
         "pos_tokens": pos_line(w, per_kernel, pk),
         "kernels": per_kernel,
         "gpu_launches": launches,
