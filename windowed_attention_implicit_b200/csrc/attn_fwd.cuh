@@ -83,6 +83,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct FwdParams {
   int B, H, W, heads, M, s, rank, nWx, nW, tiles_x, n_tiles;
+  int n_items;       // work items: (unit, pair of query tiles), units * n_tiles / 2
   int region_mask;   // shifted-window region mask on (requires s > 0)
   float scale_log2;  // softmax scale * log2(e)
   __nv_bfloat16* out;
@@ -93,13 +94,14 @@ struct FwdParams {
 };
 
 struct __align__(1024) FwdSmem {
-  uint8_t qc[2][8192];            // [128 rows][64 B], 64B swizzle
+  uint8_t qc[2][2][8192];         // [item parity][tile X] [128 rows][64 B], 64B swizzle
   uint8_t kc[kFwdStages][8192];
   uint8_t v[kFwdStages][8192];
   uint8_t ones[8192];             // bf16 1.0 everywhere: B atom that yields the row sums
-  uint8_t qp[2][4096];            // [128 rows][32 B], 32B swizzle
+  uint8_t qp[2][2][4096];         // [item parity][tile X] [128 rows][32 B], 32B swizzle
   uint8_t kp[kFwdStages][4096];
-  uint64_t q_full;
+  uint64_t q_full[2], q_free[2];  // Q buffers (item parity): loaded / read by every score MMA
+  uint64_t o_free[2];             // [O|L]_X read by the epilogue of the tile's last item
   uint64_t kv_full[kFwdStages];
   uint64_t kv_empty[kFwdStages];  // both PV threads release a stage
   uint64_t s_full[kRegions], r_free[kRegions];
@@ -118,80 +120,120 @@ static_assert(kFwdSmemBytes <= 227 * 1024, "forward shared memory exceeds the pe
 constexpr uint32_t kIdescS = make_idesc_bf16(128, 128, false, false);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, kOCols, false, true);
 
+// The CTA's work items, in order: item li is it = blockIdx.x + li * gridDim.x,
+// unit it / (n_tiles / 2), query tiles 2 (it % (n_tiles / 2)) and the next.
+// Every barrier phase below is counted across items (key tile J = li n + j,
+// score tile K = 2 J + X), so the pipeline runs on from one item to the next.
+__device__ __forceinline__ void fwd_item(const FwdParams& p, int it, UnitCoord& u, int& tile0) {
+  const int pairs = p.n_tiles / 2;
+  u = decode_unit(it / pairs, p.heads, p.nW, p.nWx);
+  tile0 = 2 * (it % pairs);
+}
+
+// Warp 16, lane 0: Q of each item into the buffer of its parity (once the
+// score MMAs of the item two back have read it), then its K/V/Kp tiles
+// through the ring.
 __device__ __forceinline__ void fwd_producer(FwdSmem& sm, const CUtensorMap* tq,
                                              const CUtensorMap* tqp, const CUtensorMap* tkp,
-                                             const FwdParams& p, const UnitCoord& u, int tile0) {
+                                             const FwdParams& p) {
   volatile int* ab = &sm.abort_flag;
-  const int hh = u.head;
-  const int by = u.wy * p.M + p.s, bx = u.wx * p.M + p.s;
   const bool pos = p.rank > 0;
-  mbar_arrive_expect_tx(&sm.q_full, 2u * (8192u + (pos ? 4096u : 0u)));
-  for (int X = 0; X < 2; ++X) {
-    int i0, j0;
-    tile_origin(tile0 + X, p.tiles_x, i0, j0);
-    const int y = wrap_once(by + i0, p.H);
-    for (int c = 0; c < 2; ++c) {
-      const int x = wrap_once(bx + j0 + 8 * c, p.W);
-      tma_load_5d(sm.qc[X] + c * 4096, tq, &sm.q_full, 0, hh, x, y, u.b);
-      if (pos) tma_load_4d(sm.qp[X] + c * 2048, tqp, &sm.q_full, 0, j0 + 8 * c, i0, hh);
-    }
-  }
+  const int n = p.n_tiles;
   const uint32_t kv_bytes = 2u * 8192u + (pos ? 4096u : 0u);
-  int j = 0;
-  for (; j < p.n_tiles; ++j) {
-    const int st = j % kFwdStages, use = j / kFwdStages;
-    if (use > 0 &&
-        !mbar_wait(&sm.kv_empty[st], (use - 1) & 1, ab, p.wait_limit_ns, SITE_FWD_PRODUCER))
+  int J = 0, li = 0, q_issued = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++li) {
+    UnitCoord u;
+    int tile0;
+    fwd_item(p, it, u, tile0);
+    const int hh = u.head;
+    const int by = u.wy * p.M + p.s, bx = u.wx * p.M + p.s;
+    const int qb = li & 1;
+    if (li >= 2 &&
+        !(ok = mbar_wait(&sm.q_free[qb], ((li >> 1) - 1) & 1, ab, p.wait_limit_ns,
+                         SITE_FWD_PRODUCER)))
       break;
-    mbar_arrive_expect_tx(&sm.kv_full[st], kv_bytes);
-    int i0, j0;
-    tile_origin(j, p.tiles_x, i0, j0);
-    const int y = wrap_once(by + i0, p.H);
-    for (int c = 0; c < 2; ++c) {
-      const int x = wrap_once(bx + j0 + 8 * c, p.W);
-      tma_load_5d(sm.kc[st] + c * 4096, tq, &sm.kv_full[st], 0, p.heads + hh, x, y, u.b);
-      tma_load_5d(sm.v[st] + c * 4096, tq, &sm.kv_full[st], 0, 2 * p.heads + hh, x, y, u.b);
-      if (pos) tma_load_4d(sm.kp[st] + c * 2048, tkp, &sm.kv_full[st], 0, j0 + 8 * c, i0, hh);
+    mbar_arrive_expect_tx(&sm.q_full[qb], 2u * (8192u + (pos ? 4096u : 0u)));
+    for (int X = 0; X < 2; ++X) {
+      int i0, j0;
+      tile_origin(tile0 + X, p.tiles_x, i0, j0);
+      const int y = wrap_once(by + i0, p.H);
+      for (int c = 0; c < 2; ++c) {
+        const int x = wrap_once(bx + j0 + 8 * c, p.W);
+        tma_load_5d(sm.qc[qb][X] + c * 4096, tq, &sm.q_full[qb], 0, hh, x, y, u.b);
+        if (pos)
+          tma_load_4d(sm.qp[qb][X] + c * 2048, tqp, &sm.q_full[qb], 0, j0 + 8 * c, i0, hh);
+      }
+    }
+    ++q_issued;
+    for (int j = 0; j < n; ++j, ++J) {
+      const int st = J % kFwdStages, use = J / kFwdStages;
+      if (use > 0 &&
+          !(ok = mbar_wait(&sm.kv_empty[st], (use - 1) & 1, ab, p.wait_limit_ns,
+                           SITE_FWD_PRODUCER)))
+        break;
+      mbar_arrive_expect_tx(&sm.kv_full[st], kv_bytes);
+      int i0, j0;
+      tile_origin(j, p.tiles_x, i0, j0);
+      const int y = wrap_once(by + i0, p.H);
+      for (int c = 0; c < 2; ++c) {
+        const int x = wrap_once(bx + j0 + 8 * c, p.W);
+        tma_load_5d(sm.kc[st] + c * 4096, tq, &sm.kv_full[st], 0, p.heads + hh, x, y, u.b);
+        tma_load_5d(sm.v[st] + c * 4096, tq, &sm.kv_full[st], 0, 2 * p.heads + hh, x, y, u.b);
+        if (pos) tma_load_4d(sm.kp[st] + c * 2048, tkp, &sm.kv_full[st], 0, j0 + 8 * c, i0, hh);
+      }
     }
   }
   if (*ab) {
-    // Aborted: let every copy this thread started land before the CTA exits.
+    // Aborted: let every copy this thread started land before the CTA exits
+    // (the latest phase of each Q buffer and of each ring stage).
     volatile int no_abort = 0;
-    mbar_wait(&sm.q_full, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
-    for (int jj = j - 1; jj >= 0 && jj >= j - kFwdStages; --jj)
+    for (int q = q_issued - 1; q >= 0 && q >= q_issued - 2; --q)
+      mbar_wait(&sm.q_full[q & 1], (q >> 1) & 1, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
+    for (int jj = J - 1; jj >= 0 && jj >= J - kFwdStages; --jj)
       mbar_wait(&sm.kv_full[jj % kFwdStages], (jj / kFwdStages) & 1, &no_abort, kFwdDrainNs,
                 SITE_FWD_DRAIN);
   }
 }
 
-// Warp 17: S(k) = Q_X K_j^T into region k % 3 for k = 2j + X, in order,
-// each once the region has been freed by the PV MMA of score tile k - 3.
+// Warp 17: S(K) = Q_X K_J^T into region K % 3 for the score tiles
+// K = 2 J + X of every item, in order, each once the region has been freed
+// by the PV MMA of score tile K - 3.  After an item's last score tile the
+// commit to q_free releases its Q buffer.
 // Phase arithmetic: a region's barriers complete once per use, and use
-// k + 3 cannot start before use k has been consumed, so no barrier is ever
+// K + 3 cannot start before use K has been consumed, so no barrier is ever
 // more than one phase ahead of the parity a waiter asks for.
 __device__ __forceinline__ void fwd_mma_scores(FwdSmem& sm, uint32_t tmem, const FwdParams& p) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const bool pos = p.rank > 0;
-  const int n = 2 * p.n_tiles;
-  bool ok = warp_wait(&sm.q_full, 0, ab, lim, SITE_FWD_MMA);
-  for (int k = 0; ok && k < n; ++k) {
-    const int X = k & 1, j = k >> 1, r = k % kRegions, st = j % kFwdStages;
-    if (X == 0 && !(ok = warp_wait(&sm.kv_full[st], (j / kFwdStages) & 1, ab, lim, SITE_FWD_MMA)))
-      break;
-    if (k >= kRegions &&
-        !(ok = warp_wait(&sm.r_free[r], (k / kRegions - 1) & 1, ab, lim, SITE_FWD_MMA)))
-      break;
-    tc_fence_after();
-    const uint32_t d = tmem + r * 128;
-    const uint64_t a = make_sdesc(smem_u32(sm.qc[X]), 16, 512, kLayoutSW64);
-    const uint64_t b = make_sdesc(smem_u32(sm.kc[st]), 16, 512, kLayoutSW64);
-    umma_ss_elect(d, a, b, kIdescS, 0u);
-    umma_ss_elect(d, a + 2, b + 2, kIdescS, 1u);  // channels 16..31: start address + 32 B
-    if (pos)
-      umma_ss_elect(d, make_sdesc(smem_u32(sm.qp[X]), 16, 256, kLayoutSW32),
-                    make_sdesc(smem_u32(sm.kp[st]), 16, 256, kLayoutSW32), kIdescS, 1u);
-    umma_commit_elect(&sm.s_full[r]);
+  const int n = p.n_tiles;
+  bool ok = true;
+  int li = 0;
+  for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++li) {
+    const int qb = li & 1;
+    if (!(ok = warp_wait(&sm.q_full[qb], (li >> 1) & 1, ab, lim, SITE_FWD_MMA))) break;
+    for (int k = 0; ok && k < 2 * n; ++k) {
+      const int X = k & 1, J = li * n + (k >> 1), K = 2 * J + X;
+      const int r = K % kRegions, st = J % kFwdStages;
+      if (X == 0 &&
+          !(ok = warp_wait(&sm.kv_full[st], (J / kFwdStages) & 1, ab, lim, SITE_FWD_MMA)))
+        break;
+      if (K >= kRegions &&
+          !(ok = warp_wait(&sm.r_free[r], (K / kRegions - 1) & 1, ab, lim, SITE_FWD_MMA)))
+        break;
+      tc_fence_after();
+      const uint32_t d = tmem + r * 128;
+      const uint64_t a = make_sdesc(smem_u32(sm.qc[qb][X]), 16, 512, kLayoutSW64);
+      const uint64_t b = make_sdesc(smem_u32(sm.kc[st]), 16, 512, kLayoutSW64);
+      umma_ss_elect(d, a, b, kIdescS, 0u);
+      umma_ss_elect(d, a + 2, b + 2, kIdescS, 1u);  // channels 16..31: start address + 32 B
+      if (pos)
+        umma_ss_elect(d, make_sdesc(smem_u32(sm.qp[qb][X]), 16, 256, kLayoutSW32),
+                      make_sdesc(smem_u32(sm.kp[st]), 16, 256, kLayoutSW32), kIdescS, 1u);
+      umma_commit_elect(&sm.s_full[r]);
+    }
+    if (ok) umma_commit_elect(&sm.q_free[qb]);
   }
   // Every MMA issued above must finish before the tensor memory is freed.
   umma_commit_elect(&sm.drain);
@@ -199,14 +241,17 @@ __device__ __forceinline__ void fwd_mma_scores(FwdSmem& sm, uint32_t tmem, const
   mbar_wait(&sm.drain, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
 }
 
-// Warps 18 (X = 0) and 19 (X = 1), all lanes, one elected lane issuing: [O|L]_X += P(k) [V_j | 1] for k = 2j + X
-// once group X has written P(k).  The commits free the region and release
-// K/V stage j (kv_empty counts one arrival per PV thread); the warp then
-// waits for its own MMAs (on the region's barrier) and publishes how many PV steps of tile X are
-// complete in pv_count[X], which the softmax warps read before touching
-// [O|L]_X (the rare rescale, and the epilogue).  The accumulation into
-// [O|L]_X is serial anyway, and the next P arrives much later, so the wait
-// costs this thread nothing.
+// Warps 18 (X = 0) and 19 (X = 1), all lanes, one elected lane issuing:
+// [O|L]_X (+)= P(K) [V_J | 1] for K = 2 J + X once group X has written P(K);
+// the first key tile of an item overwrites [O|L]_X, once the epilogue of the
+// previous item has read it (o_free).  The commits free the region and
+// release K/V stage J (kv_empty counts one arrival per PV thread); the warp
+// then waits for its own MMAs (on the region's barrier) and publishes how
+// many PV steps of tile X are complete in pv_count[X] (counted across
+// items), which the softmax warps read before touching [O|L]_X (the rare
+// rescale, and the epilogue).  The accumulation into [O|L]_X is serial
+// anyway, and the next P arrives much later, so the wait costs this thread
+// nothing.
 __device__ __forceinline__ void fwd_mma_pv(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
                                            int X) {
   volatile int* ab = &sm.abort_flag;
@@ -214,24 +259,30 @@ __device__ __forceinline__ void fwd_mma_pv(FwdSmem& sm, uint32_t tmem, const Fwd
   const int n = p.n_tiles;
   const uint32_t d = tmem + kColO + X * kOCols;
   bool ok = true;
-  for (int j = 0; ok && j < n; ++j) {
-    const int k = 2 * j + X, r = k % kRegions, st = j % kFwdStages;
-    // p_full(k) implies K/V stage st has landed: S(k) was computed from it
-    if (!(ok = warp_wait(&sm.p_full[X][j & 1], (j >> 1) & 1, ab, lim, SITE_FWD_MMA))) break;
-    tc_fence_after();
-    const uint32_t vaddr = smem_u32(sm.v[st]);
-    // B = [V | ones]: two MN-major 64B-swizzle atoms, the second LBO bytes
-    // on; step k reads the next 16 keys (1 KB of V further)
-    const uint32_t lbo = smem_u32(sm.ones) - vaddr;
-    umma_ts8_elect(d, tmem + r * 128, make_sdesc(vaddr, lbo, 512, kLayoutSW64), 1024 >> 4,
-                   kIdescPV, j > 0 ? 1u : 0u);
-    umma_commit_elect(&sm.r_free[r]);
-    umma_commit_elect(&sm.kv_empty[st]);
-    // r_free[r] is exact for this thread: its next phase needs S(k + 3),
-    // which needs this phase
-    if (!(ok = warp_wait(&sm.r_free[r], (k / kRegions) & 1, ab, lim, SITE_FWD_MMA))) break;
-    tc_fence_before();
-    if ((threadIdx.x & 31) == 0) st_release_shared(&sm.pv_count[X], j + 1);
+  int li = 0;
+  for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++li) {
+    for (int j = 0; ok && j < n; ++j) {
+      const int J = li * n + j, K = 2 * J + X, r = K % kRegions, st = J % kFwdStages;
+      if (j == 0 && li > 0 &&
+          !(ok = warp_wait(&sm.o_free[X], (li - 1) & 1, ab, lim, SITE_FWD_MMA)))
+        break;
+      // p_full(K) implies K/V stage st has landed: S(K) was computed from it
+      if (!(ok = warp_wait(&sm.p_full[X][J & 1], (J >> 1) & 1, ab, lim, SITE_FWD_MMA))) break;
+      tc_fence_after();
+      const uint32_t vaddr = smem_u32(sm.v[st]);
+      // B = [V | ones]: two MN-major 64B-swizzle atoms, the second LBO bytes
+      // on; step k reads the next 16 keys (1 KB of V further)
+      const uint32_t lbo = smem_u32(sm.ones) - vaddr;
+      umma_ts8_elect(d, tmem + r * 128, make_sdesc(vaddr, lbo, 512, kLayoutSW64), 1024 >> 4,
+                     kIdescPV, j > 0 ? 1u : 0u);
+      umma_commit_elect(&sm.r_free[r]);
+      umma_commit_elect(&sm.kv_empty[st]);
+      // r_free[r] is exact for this thread: its next phase needs S(K + 3),
+      // which needs this phase
+      if (!(ok = warp_wait(&sm.r_free[r], (K / kRegions) & 1, ab, lim, SITE_FWD_MMA))) break;
+      tc_fence_before();
+      if ((threadIdx.x & 31) == 0) st_release_shared(&sm.pv_count[X], J + 1);
+    }
   }
   umma_commit_elect(&sm.drain);
   volatile int no_abort = 0;
@@ -261,9 +312,13 @@ __device__ __forceinline__ bool wait_pv_count(FwdSmem& sm, int X, int need, cons
   return ok;
 }
 
+// One work item (the CTA's li-th) of a softmax warp: tile X of the item's
+// pair, 32 rows (quarter wq), key columns 64 h .. 64 h + 63.  Returns false
+// on abort.
 template <bool kMask>
-__device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
-                                            const UnitCoord& u, int tile0, int X, int h, int wq) {
+__device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
+                                                 const UnitCoord& u, int tile0, int X, int h,
+                                                 int wq, int li) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int lane = threadIdx.x & 31;
@@ -288,7 +343,8 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   float m_run = 0.f;
   bool ok = true;
   for (int j = 0; j < n; ++j) {
-    const int k = 2 * j + X, r = k % kRegions;
+    const int J = li * n + j;   // key tile counted across items
+    const int k = 2 * J + X, r = k % kRegions;
     bool kv = true;
     if (mask_on) {
       int ki0, kj0;
@@ -325,14 +381,14 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     }
     float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
     if (!kv) mx = -INFINITY;   // a masked key block adds nothing to the row maximum
-    sm.red_max[j & 1][X][h][row] = mx;
+    sm.red_max[J & 1][X][h][row] = mx;
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.pair_bar[X][wq]);
-    if (!(ok = warp_wait(&sm.pair_bar[X][wq], j & 1, ab, lim, SITE_FWD_SOFTMAX, kFwdSleepNs)))
+    if (!(ok = warp_wait(&sm.pair_bar[X][wq], J & 1, ab, lim, SITE_FWD_SOFTMAX, kFwdSleepNs)))
       break;
     tc_fence_after();
-    mx = fmaxf(mx, sm.red_max[j & 1][X][h ^ 1][row]);
+    mx = fmaxf(mx, sm.red_max[J & 1][X][h ^ 1][row]);
 
     // (a key tile masked for both halves of a row leaves mx = -inf: the
     // running maximum then stays at a finite floor, so no -inf - -inf arises)
@@ -378,7 +434,7 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     // took the same decision from the same row maximum), once every PV step
     // accumulated so far has completed
     if (h == 0 && __any_sync(0xffffffffu, resc)) {
-      if (!(ok = wait_pv_count(sm, X, j, p))) break;
+      if (!(ok = wait_pv_count(sm, X, J, p))) break;
       uint32_t o[32], l[16];
       tmem_ld_x32(tO, o);
       tmem_ld_x16(tO + 32, l);
@@ -395,17 +451,22 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.p_full[X][j & 1]);
+    if (lane == 0) mbar_arrive(&sm.p_full[X][J & 1]);
     m_run = m_new;
   }
-  if (!ok || h != 0) return;
-  if (!wait_pv_count(sm, X, n, p)) return;
+  if (!ok) return false;
+  if (h != 0) return true;
+  if (!wait_pv_count(sm, X, (li + 1) * n, p)) return false;
   uint32_t o[32], l[16];
   tmem_ld_x32(tO, o);
   tmem_ld_x16(tO + 32, l);
   tmem_wait_ld();
   reg_fence_x32(o);
   reg_fence_x16(l);
+  // [O|L]_X is read: the next item's first PV MMA may overwrite it
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sm.o_free[X]);
   const float l_run = __uint_as_float(l[0]);
   const float inv = 1.f / l_run;
   uint32_t pk[16];
@@ -444,9 +505,24 @@ __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const Fw
   }
   p.lse[(static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x] =
       (m_run + log2f(l_run)) * 0.69314718055994531f;
+  return true;
 }
 
-// grid (n_tiles / 2, units), block kFwdThreads, dynamic smem kFwdSmemBytes.
+// Warps 0-15: the softmax of every work item of the CTA in turn.
+template <bool kMask>
+__device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const FwdParams& p, int X,
+                                            int h, int wq) {
+  int li = 0;
+  for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++li) {
+    UnitCoord u;
+    int tile0;
+    fwd_item(p, it, u, tile0);
+    if (!fwd_softmax_item<kMask>(sm, tmem, p, u, tile0, X, h, wq, li)) return;
+  }
+}
+
+// grid min(n_items, SMs) (each CTA walks the work items it, it + gridDim.x,
+// ...), block kFwdThreads, dynamic smem kFwdSmemBytes.
 // kMask: the shifted-window region mask (a separate instantiation, so that
 // the unmasked kernel carries none of its code).
 template <bool kMask>
@@ -457,10 +533,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   extern __shared__ uint8_t sm_raw_fwd[];
   FwdSmem& sm = *align1024<FwdSmem>(sm_raw_fwd);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const UnitCoord u = decode_unit(blockIdx.y, p.heads, p.nW, p.nWx);
-  const int tile0 = blockIdx.x * 2;
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.q_full[b], 1);
+      mbar_init(&sm.q_free[b], 1);  // the score-MMA thread's commit after an item
+      mbar_init(&sm.o_free[b], 4);  // the four epilogue warps of tile b
+    }
     for (int st = 0; st < kFwdStages; ++st) {
       mbar_init(&sm.kv_full[st], 1);
       mbar_init(&sm.kv_empty[st], 2);  // one commit from each PV thread
@@ -503,11 +581,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   if (warp < 16) {
     regs_inc<kFwdSoftmaxRegs>();
-    fwd_softmax<kMask>(sm, tmem, p, u, tile0, warp >> 3, (warp >> 2) & 1, warp & 3);
+    fwd_softmax<kMask>(sm, tmem, p, warp >> 3, (warp >> 2) & 1, warp & 3);
   } else {
     regs_dec<kFwdServiceRegs>();
     if (warp == 16) {
-      if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p, u, tile0);
+      if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p);
     } else if (warp == 17) {
       fwd_mma_scores(sm, tmem, p);
     } else {

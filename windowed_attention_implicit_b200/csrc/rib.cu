@@ -603,7 +603,11 @@ static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int 
     }
     if (lr != kFwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
   }
-  dim3 grid(g.n_tiles / 2, g.units);
+  // one CTA per SM walks the work items (unit, pair of query tiles)
+  int sms = 0;
+  if ((rc = device_sms(&sms))) return rc;
+  p.n_items = g.units * (g.n_tiles / 2);
+  dim3 grid(std::min(p.n_items, sms));
   TraceScope ts(K_FWD, static_cast<cudaStream_t>(stream));
   kern<<<grid, kFwdThreads, kFwdSmemBytes, static_cast<cudaStream_t>(stream)>>>(tq, tqp, tkp, p);
   return launch_status();
