@@ -12,14 +12,17 @@
 // content tiles and one over the positional tiles, accumulating into the
 // same TMEM score tile.
 //
-// CTA = one unit (batch, window, head) x two 128-query tiles (A, B), 640
-// threads (5 warpgroups):
+// Persistent CTAs, one per SM, each walking work items = one unit (batch,
+// window, head) x two 128-query tiles (A, B); every barrier phase is counted
+// across items, so the next item's loads and score MMAs overlap the end of
+// the current one.  640 threads (5 warpgroups):
 //   warps 0-7    softmax group A: warp w owns TMEM lanes 32(w%4).. (query
 //                rows) and key columns 64((w/4)%2).. of each score tile; the
 //                two warps sharing a row exchange partial row maxima
 //   warps 8-15   softmax group B, the same for the second query tile
-//   warp  16     TMA producer: Q tiles once, then K/V/Kp tiles through a
-//                3-stage shared-memory ring; boxes at rolled map coordinates
+//   warp  16     TMA producer: each item's Q tiles (two buffers, by item
+//                parity), then its K/V/Kp tiles through a 3-stage
+//                shared-memory ring; boxes at rolled map coordinates
 //   warp  17     TMEM allocator; issues the score MMAs
 //   warp  18     issues the PV MMAs of query tile A
 //   warp  19     issues the PV MMAs of query tile B
@@ -27,10 +30,11 @@
 // exponential chains; the softmax warpgroups take 104 registers and the
 // service warpgroup 64 (setmaxnreg).
 //
-// One thread issues at most one tcgen05.mma every ~90 cycles, whatever its
-// shape, while the tensor pipe retires an M=128, N=48, K=16 MMA in ~24
-// cycles; so the MMAs of a key tile (3 score MMAs per query tile, 8 PV MMAs
-// per query tile) are spread over three issuing threads.
+// One thread issues at most one tcgen05.mma every ~43 cycles (an elected
+// lane of a converged warp; ~90 from a divergent branch), while the tensor
+// pipe retires an M=128, N=48, K=16 MMA in ~24 cycles; so the MMAs of a key
+// tile (3 score MMAs per query tile, 8 PV MMAs per query tile) are spread
+// over three issuing threads.
 //
 // TMEM (512 columns): three score regions R0..R2 of 128 fp32 columns, then
 // [O|L]_A and [O|L]_B (48 columns each).  Score tiles are numbered
@@ -41,7 +45,8 @@
 // operand (the second swizzle atom of the B operand is an all-ones tile, so
 // the tensor core also accumulates the softmax denominators L from the very
 // bf16 P it multiplies with V) and frees the region.  The score MMA of
-// k + 3 reuses the region once that PV has completed.  The softmax warps
+// k + 3 reuses the region once that PV has completed; an item's first PV
+// overwrites [O|L]_X once the previous item's epilogue has read it.  The softmax warps
 // therefore never wait for a PV MMA, except before the rare rescale of O:
 // the running max is updated lazily, O and L being rescaled only when the
 // max grows by more than 2^8.

@@ -19,7 +19,8 @@
 //   cla_bwd_dwpw_kernel  dW_pw partials = sum over the CTA's tiles of
 //                        dz^T y, y recomputed from x; both operands MN-major
 //                        in shared memory, the C x C partial in TMEM
-//   cla_bwd_dx_kernel    dx, and dW_dw / db_dw partials (FMA pipe, two CTAs per SM)
+//   cla_bwd_dx_kernel    dx, and dW_dw / db_dw partials (FMA pipe, two CTAs per SM,
+//                        x and dy halos staged by TMA)
 //   cla_bwd_reduce_kernel fixed-order sums of the partials
 #pragma once
 
@@ -414,23 +415,56 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1)
 }
 
 // -------------------------------------------------------------- dx, dW_dw, db_dw
-// grid p.grid_dx, block kClaDxThreads, static smem.  Lanes along channel
-// pairs (one 64-channel group at a time over all of the CTA's tiles, so each
-// thread keeps 20 partial sums); a warp walks down one column of a tile at a
-// time with the 3 x 3 neighbourhoods of x and dy in registers, loading only
-// the new row of each per pixel.
-__device__ __forceinline__ float2 cla_ld2(const __nv_bfloat16* ptr, bool valid) {
-  if (!valid) return make_float2(0.f, 0.f);
-  const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(ptr));
+// grid p.grid_dx (two CTAs per SM), block kClaDxThreads, dynamic smem
+// cla_dx_smem_bytes().  One 64-channel group at a time over all of the CTA's
+// tiles (lanes along channel pairs, so each thread keeps 20 partial sums);
+// per tile, the 10 x 18-pixel halos of x and dy come by TMA into one of two
+// shared-memory stages (the next tile's load overlaps this tile's work; the
+// zero padding is the TMA's out-of-range fill), and a warp walks down a
+// tile column with the 3 x 3 neighbourhoods of x and dy in registers,
+// reading only the new row of each per pixel.
+__host__ __device__ __forceinline__ size_t cla_dx_smem_bytes() {
+  return 4ull * kDwpwHaloChunk + 64 + 1024;
+}
+
+__device__ __forceinline__ float2 cla_lds2(const uint8_t* ptr) {
+  const uint32_t v = *reinterpret_cast<const uint32_t*>(ptr);
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
 }
 
-__global__ void __launch_bounds__(kClaDxThreads, 2) cla_bwd_dx_kernel(const ClaBwdParams p) {
-  __shared__ float red[kClaDxThreads / 32][10][64];
+__global__ void __launch_bounds__(kClaDxThreads, 2)
+    cla_bwd_dx_kernel(const __grid_constant__ CUtensorMap tm_x,
+                      const __grid_constant__ CUtensorMap tm_dy, const ClaBwdParams p) {
+  extern __shared__ uint8_t dx_raw[];
+  uint8_t* base = dx_raw + ((1024u - (smem_u32(dx_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + 4 * kDwpwHaloChunk);   // [2] stages
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.C;
-  const size_t row_stride = static_cast<size_t>(p.W) * C;   // elements between map rows
-  for (int g = 0; g * 64 < C; ++g) {
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  const int G = gridDim.x;
+  const int my_tiles = (p.n_tiles - static_cast<int>(blockIdx.x) + G - 1) / G;
+  // stage s: x halo at base + s * chunk, dy halo at base + (2 + s) * chunk
+  auto hx = [&](int st) { return base + st * kDwpwHaloChunk; };
+  auto hdy = [&](int st) { return base + (2 + st) * kDwpwHaloChunk; };
+  int issued = 0, consumed = 0;   // halo loads (thread 0 issues; all threads consume)
+  auto issue = [&](int g, int k) {
+    int b, i0, j0;
+    cla_tile(p, static_cast<int>(blockIdx.x) + k * G, b, i0, j0);
+    const int st = issued & 1;
+    mbar_arrive_expect_tx(&full[st], 2 * kClaHaloBytes);
+    tma_load_4d(hx(st), &tm_x, &full[st], 64 * g, j0 - 1, i0 - 1, b);
+    tma_load_4d(hdy(st), &tm_dy, &full[st], 64 * g, j0 - 1, i0 - 1, b);
+    ++issued;
+  };
+  bool ok = true;
+  for (int g = 0; ok && g * 64 < C; ++g) {
     const int c = g * 64 + 2 * lane;
     const bool act = c < C;
     float w0[9], w1[9], aw0[9], aw1[9], ab0 = 0.f, ab1 = 0.f;
@@ -440,31 +474,35 @@ __global__ void __launch_bounds__(kClaDxThreads, 2) cla_bwd_dx_kernel(const ClaB
       w1[tp] = act ? p.w_dw[(c + 1) * 9 + tp] : 0.f;
       aw0[tp] = aw1[tp] = 0.f;
     }
-    for (int t = blockIdx.x; act && t < p.n_tiles; t += gridDim.x) {
+    if (threadIdx.x == 0 && my_tiles > 0) issue(g, 0);
+    for (int k = 0; k < my_tiles; ++k) {
+      // the other stage was released by the barrier at the end of tile k-1
+      if (threadIdx.x == 0 && k + 1 < my_tiles) issue(g, k + 1);
+      const int st = consumed & 1;
+      ok = mbar_wait(&full[st], (consumed >> 1) & 1, abort_flag, p.wait_limit_ns, SITE_CLA);
+      if (!__syncthreads_and(ok)) {
+        ok = false;
+        break;
+      }
+      ++consumed;
       int b, i0, j0;
-      cla_tile(p, t, b, i0, j0);
-      for (int jc = warp; jc < 16; jc += kClaDxThreads / 32) {
-        const int j = j0 + jc;
-        const bool cv[3] = {j > 0, true, j + 1 < p.W};
-        // xw[u][v] = x(i + u - 1, j + v - 1), dw[u][v] = dy(i + u - 1, j + v - 1)
+      cla_tile(p, static_cast<int>(blockIdx.x) + k * G, b, i0, j0);
+      const uint8_t* xs = hx(st) + lane * 4;     // halo [10 rows][18 cols][64 ch]
+      const uint8_t* ys = hdy(st) + lane * 4;
+      for (int jc = warp; act && jc < 16; jc += kClaDxThreads / 32) {
+        // xw[u][v] = x(i + u - 1, jc + v - 1), dw[u][v] = dy(i + u - 1, jc + v - 1):
+        // halo row i + u, halo column jc + v
         float2 xw[3][3], dw[3][3];
-        // element offset of (row i0 - 1, column j - 1), channel c; only
-        // dereferenced where the row and column are inside the map
-        const long long o0 = (static_cast<long long>(b) * p.H + (i0 - 1)) * p.W * C +
-                             static_cast<long long>(j - 1) * C + c;
 #pragma unroll
-        for (int u = 0; u < 3; ++u) {
-          const bool rv = i0 - 1 + u >= 0 && i0 - 1 + u < p.H;
+        for (int u = 0; u < 3; ++u)
 #pragma unroll
           for (int v = 0; v < 3; ++v) {
-            const long long o = o0 + u * static_cast<long long>(row_stride) + v * C;
-            xw[u][v] = cla_ld2(p.x + o, rv && cv[v]);
-            dw[u][v] = cla_ld2(p.dy + o, rv && cv[v]);
+            const int o = (u * 18 + jc + v) * 128;
+            xw[u][v] = cla_lds2(xs + o);
+            dw[u][v] = cla_lds2(ys + o);
           }
-        }
 #pragma unroll
         for (int ii = 0; ii < 8; ++ii) {
-          const int i = i0 + ii;
           const float2 d = dw[1][1];
           ab0 += d.x;
           ab1 += d.y;
@@ -481,41 +519,50 @@ __global__ void __launch_bounds__(kClaDxThreads, 2) cla_bwd_dx_kernel(const ClaB
               dx0 = fmaf(w0[tp], dw[2 - u][2 - v].x, dx0);
               dx1 = fmaf(w1[tp], dw[2 - u][2 - v].y, dx1);
             }
-          *reinterpret_cast<uint32_t*>(p.dx + cla_pix(p, b, i, j) * C + c) = pack_bf16x2(dx0, dx1);
+          *reinterpret_cast<uint32_t*>(p.dx + cla_pix(p, b, i0 + ii, j0 + jc) * C + c) =
+              pack_bf16x2(dx0, dx1);
           if (ii < 7) {
-            // slide down one row: drop row i - 1, load row i + 2
-            const bool rv = i + 2 < p.H;
 #pragma unroll
             for (int v = 0; v < 3; ++v) {
               xw[0][v] = xw[1][v];
               xw[1][v] = xw[2][v];
               dw[0][v] = dw[1][v];
               dw[1][v] = dw[2][v];
-              const long long o = o0 + (ii + 3) * static_cast<long long>(row_stride) + v * C;
-              xw[2][v] = cla_ld2(p.x + o, rv && cv[v]);
-              dw[2][v] = cla_ld2(p.dy + o, rv && cv[v]);
+              const int o = ((ii + 3) * 18 + jc + v) * 128;
+              xw[2][v] = cla_lds2(xs + o);
+              dw[2][v] = cla_lds2(ys + o);
             }
           }
         }
       }
+      __syncthreads();   // stage st is read: it may be refilled
     }
-    // this group's partials: the warps' sums, added in warp order
+    if (!ok) break;
+    // this group's partials: the warps' sums, added in warp order, staged in
+    // the (now idle) first x halo
+    float* red = reinterpret_cast<float*>(hx(0));   // [warp][10][64]
 #pragma unroll
     for (int tp = 0; tp < 9; ++tp) {
-      red[warp][tp][2 * lane] = aw0[tp];
-      red[warp][tp][2 * lane + 1] = aw1[tp];
+      red[(warp * 10 + tp) * 64 + 2 * lane] = aw0[tp];
+      red[(warp * 10 + tp) * 64 + 2 * lane + 1] = aw1[tp];
     }
-    red[warp][9][2 * lane] = ab0;
-    red[warp][9][2 * lane + 1] = ab1;
+    red[(warp * 10 + 9) * 64 + 2 * lane] = ab0;
+    red[(warp * 10 + 9) * 64 + 2 * lane + 1] = ab1;
     __syncthreads();
     for (int e = threadIdx.x; e < 10 * 64; e += blockDim.x) {
       const int tp = e / 64, cc = e % 64;
       if (g * 64 + cc >= C) continue;
-      float s = 0.f;
-      for (int w = 0; w < kClaDxThreads / 32; ++w) s += red[w][tp][cc];
-      p.part_dw[(static_cast<size_t>(blockIdx.x) * 10 + tp) * C + g * 64 + cc] = s;
+      float sacc = 0.f;
+      for (int w = 0; w < kClaDxThreads / 32; ++w) sacc += red[(w * 10 + tp) * 64 + cc];
+      p.part_dw[(static_cast<size_t>(blockIdx.x) * 10 + tp) * C + g * 64 + cc] = sacc;
     }
-    __syncthreads();
+    __syncthreads();   // red is read before the next group's first halo lands there
+  }
+  if (!ok && threadIdx.x == 0) {
+    // a halo still in flight lands before the CTA exits
+    volatile int no_abort = 0;
+    for (int q = consumed; q < issued; ++q)
+      mbar_wait(&full[q & 1], (q >> 1) & 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
   }
 }
 

@@ -746,9 +746,21 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
                   CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   }
+  // dy (workspace, [B][H][W][C] bf16) as the same kind of map, for the dx kernel
+  CUtensorMap tm_dy;
+  {
+    const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {2ull * C, 2ull * C * W, 2ull * C * W * H};
+    const uint32_t box[4] = {64, 18, 10, 1};
+    rc = make_map(&tm_dy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.dy, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+  }
   const size_t smem_dz = cla_dz_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
+  const size_t smem_dx = cla_dx_smem_bytes();
   if ((rc = set_smem(cla_bwd_dz_kernel, smem_dz))) return rc;
   if ((rc = set_smem(cla_bwd_dwpw_kernel, smem_dw))) return rc;
+  if ((rc = set_smem(cla_bwd_dx_kernel, smem_dx))) return rc;
   {
     TraceScope ts(K_CLA_DZ, st);
     cla_bwd_dz_kernel<<<L.grid, kClaBwdThreads, smem_dz, st>>>(p);
@@ -761,7 +773,7 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   }
   {
     TraceScope ts(K_CLA_DX, st);
-    cla_bwd_dx_kernel<<<L.grid_dx, kClaDxThreads, 0, st>>>(p);
+    cla_bwd_dx_kernel<<<L.grid_dx, kClaDxThreads, smem_dx, st>>>(tm_x, tm_dy, p);
     if ((rc = launch_status())) return rc;
   }
   TraceScope ts(K_CLA_RED, st);
