@@ -27,8 +27,9 @@
 //   warp  18     issues the PV MMAs of query tile A
 //   warp  19     issues the PV MMAs of query tile B
 // Four softmax warps per SM sub-partition hide the latency of the
-// exponential chains; the softmax warpgroups take 104 registers and the
-// service warpgroup 64 (setmaxnreg).
+// exponential chains; the softmax warpgroups take 112 registers (with 104
+// the polynomial exponentials spill) and the service warpgroup 32
+// (setmaxnreg).
 //
 // One thread issues at most one tcgen05.mma every ~43 cycles (an elected
 // lane of a converged warp; ~90 from a divergent branch), while the tensor
@@ -65,8 +66,8 @@ namespace rib {
 constexpr int kFwdStages = 3;
 constexpr int kFwdThreads = 640;
 constexpr int kFwdLaunchRegs = 96;      // what the host checks ptxas gave (65536 / 640)
-constexpr int kFwdSoftmaxRegs = 104;    // warpgroups 0-3
-constexpr int kFwdServiceRegs = 64;     // warpgroup 4
+constexpr int kFwdSoftmaxRegs = 112;    // warpgroups 0-3
+constexpr int kFwdServiceRegs = 32;     // warpgroup 4
 static_assert(4 * 128 * kFwdSoftmaxRegs + 128 * kFwdServiceRegs <= kFwdThreads * kFwdLaunchRegs,
               "register split exceeds the launch budget");
 constexpr uint32_t kFwdTmemCols = 512;
