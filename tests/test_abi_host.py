@@ -140,3 +140,115 @@ def test_pos_tokens_validation():
     assert lib.rib_pos_tokens(ctypes.byref(m), 16, None, FAKE, None, None, None) == _abi.RIB_ERR_ARG
     m.n_freq = 0
     assert lib.rib_pos_tokens(ctypes.byref(m), 16, FAKE, FAKE, None, None, None) == _abi.RIB_ERR_ARG
+
+
+def fwd_masked(**kw):
+    a = dict(qkv=FAKE, B=1, H=64, W=64, heads=2, d=32, M=16, s=8, qp=FAKE, kp=FAKE, r=16,
+             scale=0.0, out=FAKE, lse=FAKE)
+    a.update(kw)
+    return R.library().rib_window_attn_fwd_masked(
+        a["qkv"], a["B"], a["H"], a["W"], a["heads"], a["d"], a["M"], a["s"], a["qp"],
+        a["kp"], a["r"], a["scale"], a["out"], a["lse"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qkv=None), _abi.RIB_ERR_ARG),
+    (dict(H=72), _abi.RIB_ERR_SHAPE),
+    (dict(s=16), _abi.RIB_ERR_SHAPE),
+    (dict(s=4), _abi.RIB_ERR_UNSUPPORTED),
+    (dict(d=64), _abi.RIB_ERR_UNSUPPORTED),
+    (dict(qp=None), _abi.RIB_ERR_ARG),
+    (dict(lse=FAKE + 4), _abi.RIB_ERR_ALIGN),
+    (dict(scale=float("inf")), _abi.RIB_ERR_ARG),
+    (dict(B=0, qkv=None, out=None, lse=None, qp=None, kp=None), _abi.RIB_OK),
+])
+def test_fwd_masked_validation(kw, code):
+    assert fwd_masked(**kw) == code
+
+
+def fwd_cla(**kw):
+    a = dict(B=1, H=64, M=16, gate=FAKE, out=FAKE, out_gated=FAKE)
+    a.update(kw)
+    return R.library().rib_window_attn_fwd_cla(
+        FAKE, a["B"], a["H"], 64, 2, 32, a["M"], 0, FAKE, FAKE, 16, 0.0, a["gate"], a["out"],
+        a["out_gated"], FAKE, None)
+
+
+def test_fwd_cla_validation():
+    assert fwd_cla(gate=None) == _abi.RIB_ERR_ARG
+    assert fwd_cla(out_gated=None) == _abi.RIB_ERR_ARG
+    assert fwd_cla(gate=FAKE + 8) == _abi.RIB_ERR_ALIGN
+    assert fwd_cla(out_gated=FAKE + 2) == _abi.RIB_ERR_ALIGN
+    assert fwd_cla(H=72) == _abi.RIB_ERR_SHAPE
+    assert fwd_cla(out=None) == _abi.RIB_ERR_ARG
+
+
+def cla_gate(**kw):
+    a = dict(x=FAKE, B=1, H=16, W=32, C=96, w_dw=FAKE, b_dw=FAKE, w_pw=FAKE, b_pw=FAKE,
+             gate=FAKE)
+    a.update(kw)
+    return R.library().rib_cla_gate(a["x"], a["B"], a["H"], a["W"], a["C"], a["w_dw"],
+                                    a["b_dw"], a["w_pw"], a["b_pw"], a["gate"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=0), _abi.RIB_ERR_ARG),
+    (dict(C=-32), _abi.RIB_ERR_ARG),
+    (dict(C=48), _abi.RIB_ERR_UNSUPPORTED),       # channels in multiples of 32
+    (dict(H=12), _abi.RIB_ERR_SHAPE),             # tiles of 8 rows
+    (dict(W=24), _abi.RIB_ERR_SHAPE),             # and 16 columns
+    (dict(x=None), _abi.RIB_ERR_ARG),
+    (dict(b_pw=None), _abi.RIB_ERR_ARG),
+    (dict(gate=None), _abi.RIB_ERR_ARG),
+    (dict(x=FAKE + 8), _abi.RIB_ERR_ALIGN),
+    (dict(gate=FAKE + 8), _abi.RIB_ERR_ALIGN),
+    (dict(w_pw=FAKE + 4), _abi.RIB_ERR_ALIGN),
+    (dict(w_dw=FAKE + 2), _abi.RIB_ERR_ALIGN),
+    (dict(B=0, H=12), _abi.RIB_ERR_SHAPE),        # an empty batch is still shape-checked
+])
+def test_cla_gate_validation(kw, code):
+    assert cla_gate(**kw) == code
+
+
+def test_cla_bwd_validation():
+    lib = R.library()
+
+    def call(**kw):
+        a = dict(x=FAKE, B=1, H=16, W=32, C=96, w_dw=FAKE, b_dw=FAKE, w_pw=FAKE, gate=FAKE,
+                 out=FAKE, dog=FAKE, do=FAKE, dx=FAKE, dw_dw=FAKE, db_dw=FAKE, dw_pw=FAKE,
+                 db_pw=FAKE, ws=FAKE * 256, wsb=1 << 40)
+        a.update(kw)
+        return lib.rib_cla_bwd(a["x"], a["B"], a["H"], a["W"], a["C"], a["w_dw"], a["b_dw"],
+                               a["w_pw"], a["gate"], a["out"], a["dog"], a["do"], a["dx"],
+                               a["dw_dw"], a["db_dw"], a["dw_pw"], a["db_pw"], a["ws"],
+                               a["wsb"], None)
+    assert call(C=40) == _abi.RIB_ERR_UNSUPPORTED
+    assert call(W=40) == _abi.RIB_ERR_SHAPE
+    assert call(B=-1) == _abi.RIB_ERR_ARG
+    assert call(dw_pw=None) == _abi.RIB_ERR_ARG
+    assert call(B=0, dw_dw=None) == _abi.RIB_ERR_ARG
+    assert call(dog=None) == _abi.RIB_ERR_ARG
+    assert call(dx=None) == _abi.RIB_ERR_ARG
+    assert call(out=FAKE + 8) == _abi.RIB_ERR_ALIGN
+    assert call(dw_pw=FAKE + 4) == _abi.RIB_ERR_ALIGN
+    assert call(db_pw=FAKE + 2) == _abi.RIB_ERR_ALIGN
+    assert lib.rib_cla_bwd_workspace(1, 12, 32, 96) == 0    # bad shape -> 0
+    assert lib.rib_cla_bwd_workspace(1, 16, 32, 40) == 0    # unsupported -> 0
+
+
+def test_bwd_masked_validation():
+    lib = R.library()
+
+    def call(ws_bytes=1 << 40, **kw):
+        a = dict(M=16, s=8, r=16, d=32, dqp=FAKE, ws=FAKE * 256)
+        a.update(kw)
+        return lib.rib_window_attn_bwd_masked(FAKE, FAKE, FAKE, FAKE, 1, 64, 64, 2, a["d"],
+                                              a["M"], a["s"], FAKE, FAKE, a["r"], 0.0, FAKE,
+                                              a["dqp"], FAKE, None, None, a["ws"], ws_bytes,
+                                              None)
+    assert call(ws_bytes=16) == _abi.RIB_ERR_WORKSPACE
+    assert call(dqp=None) == _abi.RIB_ERR_ARG
+    assert call(M=24) == _abi.RIB_ERR_SHAPE
+    assert call(s=4) == _abi.RIB_ERR_UNSUPPORTED
+    assert call(d=16) == _abi.RIB_ERR_UNSUPPORTED
+    assert call(ws=FAKE * 256 + 16) == _abi.RIB_ERR_ALIGN
