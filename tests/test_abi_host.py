@@ -252,3 +252,32 @@ def test_bwd_masked_validation():
     assert call(s=4) == _abi.RIB_ERR_UNSUPPORTED
     assert call(d=16) == _abi.RIB_ERR_UNSUPPORTED
     assert call(ws=FAKE * 256 + 16) == _abi.RIB_ERR_ALIGN
+
+
+def test_work_entry_points_run_inside_nvtx_ranges(monkeypatch):
+    log = []
+    monkeypatch.setattr(R, "_nvtx_calls",
+                        lambda: (lambda n: log.append(("push", n)), lambda: log.append("pop")))
+
+    class FakeLib:
+        pass
+    fake = FakeLib()
+    for name in _abi._SIGS:
+        setattr(fake, name, (lambda n: (lambda *a: (n, a)))(name))
+
+    def boom(*a):
+        raise ValueError("from the library")
+    fake.rib_window_scatter = boom
+    lib = R._RangedLibrary(fake)
+    assert lib.rib_window_attn_fwd(1, 2) == ("rib_window_attn_fwd", (1, 2))
+    assert log == [("push", "rib_window_attn_fwd"), "pop"]
+    log.clear()
+    for quiet in ("rib_window_attn_bwd_workspace", "rib_cla_bwd_workspace", "rib_status_string",
+                  "rib_last_status", "rib_trace_collect"):
+        getattr(lib, quiet)()
+    assert log == []
+    with pytest.raises(ValueError):
+        lib.rib_window_scatter()
+    assert log == [("push", "rib_window_scatter"), "pop"]
+    # the real library: the wrapped entry points keep their names
+    assert R.library().rib_cla_bwd.__name__ == "rib_cla_bwd"

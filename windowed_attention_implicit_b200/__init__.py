@@ -39,8 +39,60 @@ class RibError(RuntimeError):
         super().__init__(f"{where}: {rib_status_string(code)} ({code})")
 
 
-def library() -> ctypes.CDLL:
-    return _abi.load()
+# Entry points that enqueue GPU work get an NVTX range named after them, so a
+# profiler's timeline (ncu --nvtx, Nsight Systems) shows which call launched
+# which kernels.  Without a tool attached a range costs well under a
+# microsecond; where torch has no NVTX support the ranges are left out.
+_NO_RANGE = ("_workspace", "rib_status_string", "rib_last_status", "rib_version",
+             "rib_set_wait_limit_ns", "rib_trace_enable", "rib_trace_collect")
+
+
+def _nvtx_calls():
+    try:
+        torch.cuda.nvtx.range_push("rib")
+        torch.cuda.nvtx.range_pop()
+        return torch.cuda.nvtx.range_push, torch.cuda.nvtx.range_pop
+    except Exception:  # pragma: no cover - a torch build without NVTX
+        return None
+
+
+class _RangedLibrary:
+    """librib.so with every work-enqueuing entry point wrapped in an NVTX
+    range; other attributes are the ctypes library's own."""
+
+    def __init__(self, cdll: ctypes.CDLL):
+        self._cdll = cdll
+        calls = _nvtx_calls()
+        for name in _abi._SIGS:
+            fn = getattr(cdll, name)
+            if calls is not None and not any(t in name for t in _NO_RANGE):
+                fn = self._ranged(name, fn, *calls)
+            setattr(self, name, fn)
+
+    @staticmethod
+    def _ranged(name, fn, push, pop):
+        def call(*args):
+            push(name)
+            try:
+                return fn(*args)
+            finally:
+                pop()
+        call.__name__ = name
+        return call
+
+    def __getattr__(self, name):
+        return getattr(self._cdll, name)
+
+
+_ranged_lib: Optional[_RangedLibrary] = None
+
+
+def library() -> _RangedLibrary:
+    """The loaded librib.so (raises if it is missing)."""
+    global _ranged_lib
+    if _ranged_lib is None:
+        _ranged_lib = _RangedLibrary(_abi.load())
+    return _ranged_lib
 
 
 def _check(code: int, where: str) -> None:
