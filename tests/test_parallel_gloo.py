@@ -84,3 +84,86 @@ def test_two_rank_gloo_allreduce_matches_single_process():
     ref = _grads(*_inputs())
     for g, r in zip(got, ref):
         assert np.allclose(g, r, rtol=1e-12, atol=1e-12)
+
+
+# With the convolutional local attention gate in the step, its weight
+# gradients (sums over every pixel) share the MLP gradients' buffer: still one
+# all-reduce per step.
+C_CLA = HEADS * 5
+
+
+def _cla_inputs():
+    x = I.make_features(B, H, W, C_CLA, seed=31).float().numpy()
+    o = I.make_features(B, H, W, C_CLA, seed=32).float().numpy()
+    dog = I.make_features(B, H, W, C_CLA, seed=33).float().numpy()
+    return x, o, dog, I.make_cla(C_CLA, seed=31)
+
+
+def _cla_grads(x, o, dog, p):
+    from oracle.cla_oracle import cla_backward
+    g = cla_backward(x, p.w_dw.numpy(), p.b_dw.numpy(), p.w_pw.numpy(), p.b_pw.numpy(), o, dog)
+    return [g["dw_dw"], g["db_dw"], g["dw_pw"], g["db_pw"]]
+
+
+def _worker_mlp_cla(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        qkv, dout, freqs, mq, mk = _inputs()
+        x, o, dog, p = _cla_inputs()
+        sl = shard_batch(B, world, rank)
+        local = _grads(qkv[sl], dout[sl], freqs, mq, mk) + _cla_grads(x[sl], o[sl], dog[sl], p)
+        fg = FlatGrads([g.shape for g in local], device="cpu", dtype=torch.float64,
+                       names=FlatGrads.ORDER + FlatGrads.CLA_ORDER)
+        for v, g in zip(fg.views, local):
+            v.copy_(torch.from_numpy(np.ascontiguousarray(g)))
+        allreduce_grads(fg.flat)
+        if rank == 0:
+            q.put([v.numpy().copy() for v in fg.views])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gloo_allreduce_with_cla_gradients():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_mlp_cla, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = q.get(timeout=240)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ref = _grads(*_inputs()) + _cla_grads(*_cla_inputs())
+    assert len(got) == len(ref) == 12
+    for g, r in zip(got, ref):
+        assert g.shape == r.shape
+        assert np.allclose(g, r, rtol=1e-12, atol=1e-12)
+    # a shard's CLA gradient alone is not the whole sum
+    part = _cla_grads(*(a[:1] for a in _cla_inputs()[:3]), _cla_inputs()[3])
+    assert not np.allclose(part[2], ref[10])
+
+
+def test_flat_layouts():
+    from windowed_attention_implicit_b200 import PositionMLP
+    mq = I.make_mlp(F, HID, HEADS, R, 21, 0)
+    mk = I.make_mlp(F, HID, HEADS, R, 21, 1)
+    mlp = PositionMLP(torch.tensor([1.0]),
+                      *(t.contiguous() for t in (mq.w1, mq.b1, mq.w2, mq.b2,
+                                                 mk.w1, mk.b1, mk.w2, mk.b2)), HEADS, R)
+    both = FlatGrads.for_mlp_and_cla(mlp, C_CLA)
+    n_mlp = sum(t.numel() for t in (mq.w1, mq.b1, mq.w2, mq.b2, mk.w1, mk.b1, mk.w2, mk.b2))
+    assert both.flat.numel() == n_mlp + 9 * C_CLA + C_CLA + C_CLA * C_CLA + C_CLA
+    assert tuple(both.cla()["dw_dw"].shape) == (C_CLA, 3, 3)
+    assert tuple(both.cla()["dw_pw"].shape) == (C_CLA, C_CLA)
+    assert both.as_grad().q_dw1.shape == mq.w1.shape
+    both.cla()["db_pw"].fill_(2.0)                  # views of the one buffer
+    assert both.flat[-C_CLA:].eq(2.0).all()
+    with pytest.raises(ValueError):
+        FlatGrads.for_cla(C_CLA, "cpu").as_grad()
+    with pytest.raises(ValueError):
+        FlatGrads.for_mlp(mlp).cla()
+    with pytest.raises(ValueError):
+        FlatGrads([(2,), (3,)], "cpu", names=("a",))
