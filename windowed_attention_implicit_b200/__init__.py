@@ -166,9 +166,26 @@ class PositionMLP:
             p(self.q_b2, "q_b2"), p(self.k_w1, "k_w1"), p(self.k_b1, "k_b1"),
             p(self.k_w2, "k_w2"), p(self.k_b2, "k_b2"))
 
+    def tensors(self) -> Tuple[torch.Tensor, ...]:
+        """Every tensor the position tokens depend on."""
+        return (self.freqs, self.q_w1, self.q_b1, self.q_w2, self.q_b2,
+                self.k_w1, self.k_b1, self.k_w2, self.k_b2)
+
     def key(self) -> Tuple[int, ...]:
-        return tuple(t.data_ptr() for t in (self.freqs, self.q_w1, self.q_w2, self.k_w1,
-                                            self.k_w2))
+        """Addresses of those tensors (which storage the tokens come from)."""
+        return tuple(t.data_ptr() for t in self.tensors())
+
+    def versions(self) -> Tuple[int, ...]:
+        """Their in-place modification counters (an optimizer step that
+        updates the weights in place moves them on)."""
+        return tuple(_tensor_version(t) for t in self.tensors())
+
+
+def _tensor_version(t: torch.Tensor) -> int:
+    try:
+        return t._version
+    except RuntimeError:  # an inference-mode tensor carries no version counter
+        return -1
 
 
 @dataclass
@@ -466,16 +483,26 @@ def rib_trace_collect() -> Dict[str, Tuple[int, float]]:
 
 class PosTokenCache:
     """Qp/Kp per window geometry, computed once and reused across windows,
-    batch entries and layers (they depend only on the geometry and the MLP)."""
+    batch entries and layers (they depend only on the geometry and the MLP).
+
+    An entry is keyed by the window and the addresses of the MLP's tensors
+    (frequencies, weights and biases), and holds references to them, so no
+    other tensor can take those addresses while it lives.  It is recomputed
+    when any of them has been modified in place since (an optimizer step),
+    and replaced, not kept beside the new one."""
 
     def __init__(self):
         self._cache = {}
 
     def get(self, mlp: PositionMLP, window: int, stream=None):
         k = (mlp.key(), int(window))
-        if k not in self._cache:
-            self._cache[k] = rib_pos_tokens(mlp, window, stream=stream)
-        return self._cache[k]
+        ver = mlp.versions()
+        e = self._cache.get(k)
+        if e is None or e[0] != ver:
+            tokens = rib_pos_tokens(mlp, window, stream=stream)
+            self._cache[k] = (ver, tokens, mlp.tensors())
+            e = self._cache[k]
+        return e[1]
 
     def clear(self):
         self._cache.clear()
