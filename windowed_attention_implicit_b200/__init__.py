@@ -118,6 +118,34 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
     return t.data_ptr()
 
 
+def _sizes(where: str, dev, **buffers) -> None:
+    """Buffers handed to the library must hold exactly the elements the call
+    reads or writes, on the device of the call's other tensors: the library
+    takes bare pointers and can check neither.  buffers: name=(tensor or
+    None, element count)."""
+    for name, (t, n) in buffers.items():
+        if t is None:
+            continue
+        if t.numel() != n:
+            raise RibError(_abi.RIB_ERR_ARG,
+                           f"{where}: {name} holds {t.numel()} elements, the call needs {n}")
+        if t.device != dev:
+            raise RibError(_abi.RIB_ERR_ARG, f"{where}: {name} is on {t.device}, not {dev}")
+
+
+def _grad_sizes(dmlp: Optional["PositionMLPGrad"], mlp: Optional["PositionMLP"]):
+    """Each position-MLP gradient sized like its weight."""
+    if dmlp is None or mlp is None:
+        return {}
+    return {f"dmlp.{n}": (getattr(dmlp, n), getattr(mlp, n[:2] + n[3:]).numel())
+            for n in ("q_dw1", "q_db1", "q_dw2", "q_db2", "k_dw1", "k_db1", "k_dw2", "k_db2")}
+
+
+def _cla_sizes(cla: "ClaGate", C: int):
+    return {"w_dw": (cla.w_dw, 9 * C), "b_dw": (cla.b_dw, C), "w_pw": (cla.w_pw, C * C),
+            "b_pw": (cla.b_pw, C)}
+
+
 def rib_status_string(code: int) -> str:
     return library().rib_status_string(int(code)).decode()
 
@@ -225,6 +253,9 @@ def rib_pos_tokens(mlp: PositionMLP, window: int, qp=None, kp=None, qp_bf16=None
     if with_bf16:
         qp_bf16 = torch.empty(shape, device=dev, dtype=torch.bfloat16) if qp_bf16 is None else qp_bf16
         kp_bf16 = torch.empty(shape, device=dev, dtype=torch.bfloat16) if kp_bf16 is None else kp_bf16
+    n = mlp.heads * int(window) ** 2 * mlp.rank
+    _sizes("rib_pos_tokens", dev, qp=(qp, n), kp=(kp, n), qp_bf16=(qp_bf16, n),
+           kp_bf16=(kp_bf16, n))
     c = mlp.c_struct()
     _check(library().rib_pos_tokens(
         ctypes.byref(c), int(window), _ptr(qp, torch.float32, "qp"), _ptr(kp, torch.float32, "kp"),
@@ -242,6 +273,9 @@ def rib_pos_tokens_bwd(mlp: PositionMLP, window: int, dqp: torch.Tensor, dkp: to
                        dmlp: Optional["PositionMLPGrad"] = None, workspace=None, stream=None):
     """Position-MLP gradients from dL/dQp, dL/dKp ([heads][M][M][rank] fp32)."""
     dmlp = PositionMLPGrad.empty_like(mlp) if dmlp is None else dmlp
+    n = mlp.heads * int(window) ** 2 * mlp.rank
+    _sizes("rib_pos_tokens_bwd", mlp.freqs.device, dqp=(dqp, n), dkp=(dkp, n),
+           **_grad_sizes(dmlp, mlp))
     need = rib_pos_tokens_bwd_workspace(mlp, window)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=dqp.device, dtype=torch.uint8)
@@ -262,6 +296,9 @@ def rib_pos_tokens_bwd_noalloc(mlp: PositionMLP, window: int, dqp: torch.Tensor,
     of a workspace; `dmlp` must be given (preallocated).  Calls that overlap
     on the GPU share that scratch and race; the first call on a device should
     precede any stream capture."""
+    n = mlp.heads * int(window) ** 2 * mlp.rank
+    _sizes("rib_pos_tokens_bwd_noalloc", mlp.freqs.device, dqp=(dqp, n), dkp=(dkp, n),
+           **_grad_sizes(dmlp, mlp))
     c, cg = mlp.c_struct(), dmlp.c_struct()
     _check(library().rib_pos_tokens_bwd_noalloc(
         ctypes.byref(c), int(window), _ptr(dqp, torch.float32, "dqp"),
@@ -283,6 +320,10 @@ def rib_window_attn_fwd(qkv: torch.Tensor, window: int, shift: int, qp_bf16=None
     out = torch.empty((B, H, W, heads, d), device=qkv.device, dtype=torch.bfloat16) if out is None else out
     lse = torch.empty((B, heads, H, W), device=qkv.device, dtype=torch.float32) if lse is None else lse
     name = "rib_window_attn_fwd_masked" if region_mask else "rib_window_attn_fwd"
+    nt = heads * int(window) ** 2 * int(rank)
+    _sizes(name, qkv.device, out=(out, B * H * W * heads * d), lse=(lse, B * heads * H * W),
+           qp_bf16=(qp_bf16 if rank > 0 else None, nt),
+           kp_bf16=(kp_bf16 if rank > 0 else None, nt))
     _check(getattr(library(), name)(
         _ptr(qkv, torch.bfloat16, "qkv"), B, H, W, heads, d, int(window), int(shift),
         _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
@@ -315,6 +356,7 @@ def rib_cla_gate(x: torch.Tensor, cla: ClaGate, gate=None, stream=None) -> torch
     """G bf16 [B][H][W][C] = sigmoid(PW1x1(DW3x3(x))) for x bf16 [B][H][W][C]."""
     B, H, W, C = x.shape
     gate = torch.empty_like(x) if gate is None else gate
+    _sizes("rib_cla_gate", x.device, gate=(gate, x.numel()), **_cla_sizes(cla, C))
     f32 = torch.float32
     _check(library().rib_cla_gate(
         _ptr(x, torch.bfloat16, "x"), B, H, W, C, _ptr(cla.w_dw, f32, "w_dw"),
@@ -337,6 +379,11 @@ def rib_window_attn_fwd_cla(qkv: torch.Tensor, window: int, shift: int, gate: to
     out = torch.empty(shape, device=qkv.device, dtype=torch.bfloat16) if out is None else out
     out_gated = torch.empty(shape, device=qkv.device, dtype=torch.bfloat16) if out_gated is None else out_gated
     lse = torch.empty((B, heads, H, W), device=qkv.device, dtype=torch.float32) if lse is None else lse
+    n_out, nt = B * H * W * heads * d, heads * int(window) ** 2 * int(rank)
+    _sizes("rib_window_attn_fwd_cla", qkv.device, gate=(gate, n_out), out=(out, n_out),
+           out_gated=(out_gated, n_out), lse=(lse, B * heads * H * W),
+           qp_bf16=(qp_bf16 if rank > 0 else None, nt),
+           kp_bf16=(kp_bf16 if rank > 0 else None, nt))
     _check(library().rib_window_attn_fwd_cla(
         _ptr(qkv, torch.bfloat16, "qkv"), B, H, W, heads, d, int(window), int(shift),
         _ptr(qp_bf16, torch.bfloat16, "qp_bf16"), _ptr(kp_bf16, torch.bfloat16, "kp_bf16"),
@@ -361,6 +408,9 @@ def rib_cla_bwd(x: torch.Tensor, cla: ClaGate, gate: torch.Tensor, out: torch.Te
     dx = torch.empty_like(x) if dx is None else dx
     g = {k: torch.empty_like(getattr(cla, k.replace("d", "", 1)))
          for k in ("dw_dw", "db_dw", "dw_pw", "db_pw")}
+    n = x.numel()
+    _sizes("rib_cla_bwd", dev, gate=(gate, n), out=(out, n), dout_gated=(dout_gated, n),
+           dout=(dout, n), dx=(dx, n), **_cla_sizes(cla, C))
     need = rib_cla_bwd_workspace(B, H, W, C)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
@@ -400,12 +450,18 @@ def rib_window_attn_bwd(qkv, out, dout, lse, window: int, shift: int, qp_bf16=No
         dkp = torch.empty(pshape, device=dev, dtype=torch.float32) if dkp is None else dkp
     if mlp is not None and dmlp is None:
         dmlp = PositionMLPGrad.empty_like(mlp)
+    name = "rib_window_attn_bwd_masked" if region_mask else "rib_window_attn_bwd"
+    n_out, nt = B * H * W * heads * d, heads * int(window) ** 2 * int(rank)
+    pos = rank > 0
+    _sizes(name, dev, out=(out, n_out), dout=(dout, n_out), lse=(lse, B * heads * H * W),
+           dqkv=(dqkv, qkv.numel()), qp_bf16=(qp_bf16 if pos else None, nt),
+           kp_bf16=(kp_bf16 if pos else None, nt), dqp=(dqp if pos else None, nt),
+           dkp=(dkp if pos else None, nt), **_grad_sizes(dmlp, mlp))
     need = rib_window_attn_bwd_workspace(B, H, W, heads, d, window, rank, mlp)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
     c_mlp = mlp.c_struct() if mlp is not None else None
     c_dmlp = dmlp.c_struct() if (mlp is not None and dmlp is not None) else None
-    name = "rib_window_attn_bwd_masked" if region_mask else "rib_window_attn_bwd"
     _check(getattr(library(), name)(
         _ptr(qkv, torch.bfloat16, "qkv"), _ptr(out, torch.bfloat16, "out"),
         _ptr(dout, torch.bfloat16, "dout"), _ptr(lse, torch.float32, "lse"),
@@ -425,6 +481,7 @@ def rib_window_gather(x: torch.Tensor, window: int, shift: int, out=None, stream
     B, H, W, C = x.shape
     nW = (H // window) * (W // window)
     out = torch.empty((B, nW, window * window, C), device=x.device, dtype=x.dtype) if out is None else out
+    _sizes("rib_window_gather", x.device, out=(out, B * nW * window * window * C))
     _check(library().rib_window_gather(
         _ptr(x, None, "x"), B, H, W, C, x.element_size(), int(window), int(shift),
         _ptr(out, x.dtype, "out"), _stream(stream)), "rib_window_gather")
@@ -436,6 +493,12 @@ def rib_window_scatter(xw: torch.Tensor, H: int, W: int, window: int, shift: int
     """Inverse of rib_window_gather."""
     B, nW, N, C = xw.shape
     out = torch.empty((B, H, W, C), device=xw.device, dtype=xw.dtype) if out is None else out
+    _sizes("rib_window_scatter", xw.device, out=(out, B * H * W * C))
+    if (window > 0 and H % window == 0 and W % window == 0 and
+            (nW, N) != ((H // window) * (W // window), window * window)):
+        raise RibError(_abi.RIB_ERR_ARG, f"rib_window_scatter: xw is [B][{nW}][{N}][C], the "
+                       f"{window}x{window} windows of a {H}x{W} map need "
+                       f"[B][{(H // window) * (W // window)}][{window * window}][C]")
     _check(library().rib_window_scatter(
         _ptr(xw, None, "xw"), B, H, W, C, xw.element_size(), int(window), int(shift),
         _ptr(out, xw.dtype, "out"), _stream(stream)), "rib_window_scatter")
