@@ -58,7 +58,7 @@ def assert_all(checks):
 
 
 def mlp_grad_checks(dmlp, ref_q, ref_k):
-    """Position-MLP weight grads of one side are judged on that side's common
+    """Position-MLP weight grads of one side are measured against that side's common
     scale, max(1, max|ref| over its four tensors): the key MLP's output-bias
     gradient is a sum that cancels exactly (rows of dS sum to zero), so its
     own magnitude says nothing about the size of the terms summed."""

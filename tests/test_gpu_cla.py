@@ -98,10 +98,10 @@ def _cla_bwd_case(B, H, W, C, seed):
     ref = O.cla_backward(x, p.w_dw, p.b_dw, p.w_pw, p.b_pw, o, dout_g)
     # dO = dO' * G has the magnitude of the upstream gradient (up to ~5 for
     # N(0,1) draws over 28 M elements), where one bf16 half-ulp is 0.016:
-    # judged, like the sums below, on max(1, max|ref|)
+    # measured, like the sums below, against max(1, max|ref|)
     checks = [check_close(to_np(g["dout"]), ref["d_o"], "dO", normalize=True),
               check_close(to_np(g["dx"]), ref["dx"], "dx")]
-    # sums over every pixel: judged on their magnitude (bf16 operands)
+    # sums over every pixel: measured against their magnitude (bf16 operands)
     for k in ("dw_pw", "db_pw", "dw_dw", "db_dw"):
         checks.append(check_close(to_np(g[k]), ref[k], k, normalize=True))
     assert_all(checks)
