@@ -142,3 +142,14 @@ def test_gather_scatter_buffers():
     _rejects(R.rib_window_scatter, "out holds", xw, H, W, M, S, out=x[:, :16])
     # windows of another size than the call's
     _rejects(R.rib_window_scatter, "xw is", torch.zeros((B, 16, 64, C), dtype=bf), H, W, M, S)
+
+
+def test_tensors_off_the_current_device_are_refused(monkeypatch):
+    # the library launches on the current device; a call whose tensors live
+    # on another GPU is refused before any pointer is handed over
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(R.RibError, match="current device is cuda:0") as e:
+        R._sizes("rib_window_attn_fwd", torch.device("cuda", 1))
+    assert e.value.code == _abi.RIB_ERR_ARG
+    R._sizes("rib_window_attn_fwd", torch.device("cuda", 0))
+    R._sizes("rib_window_attn_fwd", torch.device("cpu"))

@@ -122,7 +122,11 @@ def _sizes(where: str, dev, **buffers) -> None:
     """Buffers handed to the library must hold exactly the elements the call
     reads or writes, on the device of the call's other tensors: the library
     takes bare pointers and can check neither.  buffers: name=(tensor or
-    None, element count)."""
+    None, element count).  The library launches on the current CUDA device,
+    so the call's tensors must live there (torch.cuda.set_device)."""
+    if dev is not None and dev.type == "cuda" and dev.index != torch.cuda.current_device():
+        raise RibError(_abi.RIB_ERR_ARG, f"{where}: tensors are on {dev}, the current device "
+                       f"is cuda:{torch.cuda.current_device()}")
     for name, (t, n) in buffers.items():
         if t is None:
             continue
