@@ -48,10 +48,13 @@ Memory: rows of the N x N score matrix are processed in row blocks when N is
 large; every row's softmax is independent, so a block changes no row's
 arithmetic, and the key-side gradient sums still run over every row.
 
-Pins: every function here is checked, in tests/test_oracle_pins.py, against
-closed forms, brute force on tiny windows, library routines (torch SDPA and
-autograd in fp64) and central finite differences; no function is "parity
-unpinned".
+Pins: every function here is checked, in tests/test_oracle_pins.py and
+tests/test_region_mask_oracle.py, against closed forms, brute force on tiny
+windows (the unit read pixel by pixel through the modular roll index, each
+requested query row attended on its own), library routines (torch SDPA and
+autograd in fp64) and central finite differences; tests/test_oracle_mutations.py
+plants a plausible mistake in each and checks that a pin fails.  No function
+is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -63,7 +66,7 @@ __all__ = [
     "mlp_backward", "pos_tokens", "pos_tokens_backward", "window_partition",
     "window_reverse", "unit_scores", "attention_unit", "attention_unit_rows",
     "attention_unit_backward", "attn_fwd", "attn_bwd", "default_scale",
-    "unit_index", "gather_unit", "region_labels",
+    "gather_unit", "region_labels",
 ]
 
 _ROW_BLOCK = 2048
@@ -219,12 +222,6 @@ def window_reverse(xw, M: int, s: int, H: int, W: int):
     x = np.moveaxis(x, 2, 3)             # B, H/M, M, W/M, M, ...
     x = x.reshape((B, H, W) + rest)
     return np.roll(x, shift=(s, s), axis=(1, 2))
-
-
-def unit_index(H, W, M, heads, b, w, h):
-    """Flat (batch, window, head) unit id used by the tests' sampling."""
-    nW = (H // M) * (W // M)
-    return (b * nW + w) * heads + h
 
 
 # --------------------------------------------------------------------------

@@ -4,6 +4,8 @@ Each case monkeypatches one oracle function with a plausible bug (dropped
 term, wrong sign, transposed operand, swapped index) and runs the pin tests
 that should catch it; at least one of them must fail.
 """
+import inspect
+
 import numpy as np
 import pytest
 
@@ -74,6 +76,46 @@ def _mlp_bwd_no_gelu_grad(gamma, w1, b1, w2, b2, d_out):
     return dh.T @ gamma, dh.sum(0), g.T @ h, g.sum(0)
 
 
+def _gather_wrong_head_pos(qkv, qp, kp, M, s, b, w, h):
+    g = list(_orig_gather(qkv, qp, kp, M, s, b, w, h))
+    g[3] = R._f64(qp)[0].reshape(M * M, -1)          # Qp of head 0 for every head
+    return tuple(g)
+
+
+def _gather_wrong_batch(qkv, qp, kp, M, s, b, w, h):
+    return _orig_gather(qkv, qp, kp, M, s, 0, w, h)   # batch entry ignored
+
+
+def _gather_k_v_swapped(qkv, qp, kp, M, s, b, w, h):
+    qc, kc, v, qpf, kpf = _orig_gather(qkv, qp, kp, M, s, b, w, h)
+    return qc, v, kc, qpf, kpf
+
+
+_orig_gather = R.gather_unit
+
+
+def _allowed_ignores_rows(labels, r0, r1, rows=None):
+    return _orig_allowed(labels, r0, r1)              # labels of rows 0.. instead of `rows`
+
+
+_orig_allowed = R._allowed
+
+
+def _rows_positional_unsliced(qc, kc, v, qp, kp, scale, rows=None, labels=None):
+    qc, kc, v, qp, kp = map(R._f64, (qc, kc, v, qp, kp))
+    if rows is not None:
+        qc = qc[rows]                                 # Qp left in token order
+        qp = qp[: len(rows)]
+    n = qc.shape[0]
+    out, lse = np.empty((n, v.shape[1])), np.empty(n)
+    for r0 in range(0, n, R._ROW_BLOCK):
+        r1 = min(n, r0 + R._ROW_BLOCK)
+        sc = R.unit_scores(qc[r0:r1], kc, qp[r0:r1], kp, scale, R._allowed(labels, r0, r1, rows))
+        p, lse[r0:r1] = R._softmax_rows(sc)
+        out[r0:r1] = p @ v
+    return out, lse
+
+
 MUTATIONS = [
     ("unit_scores", _scores_bias_sign,
      [P.test_golden_closed_forms, P.test_attention_matches_torch_sdpa_augmented]),
@@ -94,6 +136,16 @@ MUTATIONS = [
      [P.test_attn_bwd_matches_torch_autograd]),
     ("mlp_backward", _mlp_bwd_no_gelu_grad,
      [P.test_mlp_backward_finite_differences, P.test_pos_tokens_backward_finite_differences]),
+    ("gather_unit", _gather_wrong_head_pos,
+     [P.test_gather_unit_matches_pixel_index, P.test_gather_unit_then_attention_is_the_map_output]),
+    ("gather_unit", _gather_wrong_batch,
+     [P.test_gather_unit_matches_pixel_index, P.test_gather_unit_then_attention_is_the_map_output]),
+    ("gather_unit", _gather_k_v_swapped,
+     [P.test_gather_unit_matches_pixel_index]),
+    ("_allowed", _allowed_ignores_rows,
+     [P.test_attention_unit_rows_matches_per_row_brute_force]),
+    ("attention_unit_rows", _rows_positional_unsliced,
+     [P.test_attention_unit_rows_matches_per_row_brute_force]),
 ]
 
 _PARAMS = {
@@ -101,6 +153,8 @@ _PARAMS = {
     P.test_concatenated_dot_product_equals_content_plus_bias: {"r": 3},
     P.test_attention_matches_torch_sdpa_augmented: {"r": 16},
     P.test_partition_matches_modular_index_and_inverts: {"M": 4, "s": 3},
+    P.test_gather_unit_matches_pixel_index: {"M": 2, "s": 1, "b": 1, "w": 5, "h": 2},
+    P.test_attention_unit_rows_matches_per_row_brute_force: {"masked": True},
 }
 
 
@@ -108,11 +162,30 @@ _PARAMS = {
                          ids=[f"{m[0]}:{m[1].__name__}" for m in MUTATIONS])
 def test_planted_mistake_is_caught(monkeypatch, name, bad, pins):
     monkeypatch.setattr(R, name, bad)
-    monkeypatch.setattr(O, name, bad)
+    if hasattr(O, name):
+        monkeypatch.setattr(O, name, bad)
     caught = 0
     for pin in pins:
+        kw = dict(_PARAMS.get(pin, {}))
+        if "monkeypatch" in inspect.signature(pin).parameters:
+            kw["monkeypatch"] = monkeypatch
         try:
-            pin(**_PARAMS.get(pin, {}))
+            pin(**kw)
         except AssertionError:
             caught += 1
     assert caught >= 1, f"no pin caught the planted mistake in {name}"
+
+
+_PIN_FILES = ("test_oracle_pins.py", "test_region_mask_oracle.py", "test_cla_oracle.py")
+
+
+def test_every_exported_oracle_function_is_called_by_a_pin_file():
+    """No exported oracle function goes without a CPU pin: each name appears as
+    a call in at least one of the pin files (closed forms, brute force,
+    library routines, finite differences)."""
+    import os
+    import re
+    here = os.path.dirname(__file__)
+    text = "".join(open(os.path.join(here, f)).read() for f in _PIN_FILES)
+    missing = [n for n in O.__all__ if not re.search(r"\bO\.%s\(" % n, text)]
+    assert not missing, missing

@@ -471,3 +471,86 @@ def test_golden_closed_forms():
                                     c["scale"])
         assert np.allclose(out, c["expect"]["out"], atol=1e-12), c["name"]
         assert np.allclose(lse, c["expect"]["lse"], atol=1e-12), c["name"]
+
+
+# ---------------------------------------------------------------- unit helpers
+
+def _brute_unit(qkv, qp, kp, M, s, b, w, h):
+    """Unit (b, w, h) read pixel by pixel: token t = i*M + j of window
+    w = wy*(W/M) + wx sits at map pixel ((wy*M+i+s) mod H, (wx*M+j+s) mod W)
+    (the roll by -s, then the partition); its position tokens are row (i, j)
+    of head h."""
+    H, W = qkv.shape[1:3]
+    wy, wx = divmod(w, W // M)
+    N = M * M
+    d, r = qkv.shape[-1], qp.shape[-1]
+    qc, kc, v = np.empty((N, d)), np.empty((N, d)), np.empty((N, d))
+    qpu, kpu = np.empty((N, r)), np.empty((N, r))
+    for i, j in itertools.product(range(M), range(M)):
+        t = i * M + j
+        y, x = (wy * M + i + s) % H, (wx * M + j + s) % W
+        qc[t], kc[t], v[t] = qkv[b, y, x, 0, h], qkv[b, y, x, 1, h], qkv[b, y, x, 2, h]
+        qpu[t], kpu[t] = qp[h, i, j], kp[h, i, j]
+    return qc, kc, v, qpu, kpu
+
+
+@pytest.mark.parametrize("M,s,b,w,h", [(2, 1, 1, 5, 2), (4, 2, 0, 3, 1), (4, 0, 1, 0, 0),
+                                       (4, 3, 1, 2, 2)])
+def test_gather_unit_matches_pixel_index(M, s, b, w, h):
+    B, H, W, heads, d, r = 2, 8, 12, 3, 5, 2
+    qkv = rnd(B, H, W, 3, heads, d)
+    qp, kp = rnd(heads, M, M, r), rnd(heads, M, M, r)
+    got = O.gather_unit(qkv, qp, kp, M, s, b, w, h)
+    want = _brute_unit(qkv, qp, kp, M, s, b, w, h)
+    for g, e in zip(got, want):
+        assert np.array_equal(g, e)
+
+
+def test_gather_unit_then_attention_is_the_map_output():
+    """The unit read by gather_unit, attended, lands at the map pixels that
+    attn_fwd (checked pixel by pixel above) writes for that unit."""
+    B, H, W, heads, d, M, r, s = 2, 8, 8, 2, 3, 4, 2, 2
+    qkv = rnd(B, H, W, 3, heads, d)
+    qp, kp = rnd(heads, M, M, r), rnd(heads, M, M, r)
+    tau = 0.4
+    out, lse = O.attn_fwd(qkv, M, s, qp, kp, tau)
+    for b, w, h in ((1, 3, 1), (0, 1, 0)):
+        o, l = O.attention_unit(*O.gather_unit(qkv, qp, kp, M, s, b, w, h), tau)
+        wy, wx = divmod(w, W // M)
+        for i, j in itertools.product(range(M), range(M)):
+            y, x = (wy * M + i + s) % H, (wx * M + j + s) % W
+            assert np.allclose(out[b, y, x, h], o[i * M + j], atol=1e-14)
+            assert abs(lse[b, h, y, x] - l[i * M + j]) < 1e-14
+
+
+def _brute_rows(qc, kc, v, qp, kp, tau, rows, labels):
+    """Each requested query row on its own: scores over the keys it may see
+    (all, or those sharing its region label), softmax, weighted sum of V."""
+    outs, lses = [], []
+    for t in rows:
+        keys = [u for u in range(kc.shape[0]) if labels is None or labels[u] == labels[t]]
+        logits = np.array([tau * (qc[t] @ kc[u] + qp[t] @ kp[u]) for u in keys])
+        p = np.exp(logits - logits.max())
+        outs.append((p[:, None] * v[keys]).sum(0) / p.sum())
+        lses.append(logsumexp(logits))
+    return np.array(outs), np.array(lses)
+
+
+@pytest.mark.parametrize("masked", [False, True])
+def test_attention_unit_rows_matches_per_row_brute_force(monkeypatch, masked):
+    """A row subset that is unsorted, repeats a row and, with a small row
+    block, straddles block edges and every region band of a corner window."""
+    H = W = 32
+    M, s = 16, 8
+    N, d, r = M * M, 4, 3
+    qc, kc, v, qp, kp = rnd(N, d), rnd(N, d), rnd(N, d), rnd(N, r), rnd(N, r)
+    lab = O.region_labels(H, W, M, s, 1, 1) if masked else None
+    if masked:
+        assert len(set(lab.tolist())) == 4
+    rows = np.array([255, 0, 7, 8, 9, 120, 136, 17, 250, 8, 64, 191])
+    monkeypatch.setattr(O.rib_oracle, "_ROW_BLOCK", 5)
+    out, lse = O.attention_unit_rows(qc, kc, v, qp, kp, 0.35, rows=rows, labels=lab)
+    ref_o, ref_l = _brute_rows(qc, kc, v, qp, kp, 0.35, rows, lab)
+    assert out.shape == (len(rows), d)
+    assert np.allclose(out, ref_o, atol=1e-13)
+    assert np.allclose(lse, ref_l, atol=1e-13)
