@@ -9,8 +9,16 @@ Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rib|reference]
 
+--gpus N runs N ranks, one per GPU: under an outer torchrun launch WORLD_SIZE
+must equal N; without one, N > 1 re-launches this script under
+torch.distributed.run with N processes on this node.
+
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on this host's cores (rank 0 only).
+
+Roofline fractions divide by the measured burst bf16 peak: the timed loops
+are a fraction of a second long and the sampled SM clock stays at its
+maximum, so the seconds-long, power-capped sustained figure does not apply.
 """
 from __future__ import annotations
 
@@ -48,6 +56,70 @@ def parse():
                     help="run only the convolutional local attention gate and the gated "
                          "forward, warm-up + timed (for profiler captures)")
     return ap.parse_args()
+
+
+def world_plan(gpus: int, env=None):
+    """What to do with --gpus N given the launcher's environment.
+
+    Returns "run" (the ranks are in place), "relaunch" (no outer launcher and
+    N > 1: start N ranks under torch.distributed.run) or raises ValueError
+    when an outer launcher started a different number of ranks than N."""
+    env = os.environ if env is None else env
+    if gpus < 1:
+        raise ValueError(f"--gpus must be >= 1, got {gpus}")
+    ws = env.get("WORLD_SIZE")
+    if ws is None:
+        return "relaunch" if gpus > 1 else "run"
+    if int(ws) != gpus:
+        raise ValueError(f"--gpus {gpus} but the launcher started WORLD_SIZE={ws} ranks")
+    return "run"
+
+
+def relaunch_cmd(gpus: int, argv, port: int):
+    """torch.distributed.run command that starts `gpus` ranks of this script
+    on this node (rendezvous on 127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (all ranks must call it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bench_config(w, world: int):
+    """The `config` object of the bench line, the same for both arms."""
+    return {"workload": workload_desc(w), "global_batch": w.batch * world,
+            "map": [w.height, w.width], "window": w.windows[0], "shift": w.shifts[0],
+            "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
+            "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2 (qkv 170 MB + dout 57 MB per rank)"
+                  if w.name == "w96train" else "per-step inputs as generated"}
+
+
+def roofline_entry(kernel, flop_per_launch, avg_ms, pk, traffic=None):
+    """Achieved algorithmic TFLOP/s of one launch against the measured burst
+    bf16 peak."""
+    ach = flop_per_launch / (avg_ms * 1e-3) / 1e12
+    return {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": traffic,
+            "flop_per_launch": flop_per_launch, "avg_ms": avg_ms,
+            "frac_of_sustained": ach / pk["bf16_tflops_sustained"],
+            "peak_source": f"{pk['source']} bf16_tflops (burst)"}
 
 
 def flops(w, layer=0):
@@ -196,7 +268,7 @@ def config_sweep(I, R, dev, rank, world, timed, steps, warmup, peak, pk):
                 "map": [w.batch, w.height, w.width], "heads": w.heads,
                 "fwd_ms": ms_f, "fwd_tflops": world * f_fwd / (ms_f * 1e-3) / 1e12,
                 "fwd_tokens_per_s": world * tok / (ms_f * 1e-3),
-                "fwd_frac_sustained": f_fwd / (ms_f * 1e-3) / 1e12 / peak}
+                "fwd_frac": f_fwd / (ms_f * 1e-3) / 1e12 / peak}
         if w.backward:
             ws = {}
 
@@ -219,7 +291,7 @@ def config_sweep(I, R, dev, rank, world, timed, steps, warmup, peak, pk):
             line.update({"step_ms": ms_t,
                          "step_tflops": world * (f_fwd + f_bwd) / (ms_t * 1e-3) / 1e12,
                          "step_tokens_per_s": world * tok / (ms_t * 1e-3),
-                         "step_frac_sustained": (f_fwd + f_bwd) / (ms_t * 1e-3) / 1e12 / peak})
+                         "step_frac": (f_fwd + f_bwd) / (ms_t * 1e-3) / 1e12 / peak})
         # bytes of one forward (qkv read, out written, lse written) against HBM
         byt = w.layers * w.tokens() * w.heads * (3 * 64 + 64 + 4)
         line["fwd_gbs"] = byt / (ms_f * 1e-3) / 1e9
@@ -353,6 +425,8 @@ def oracle_cores():
 
 
 def run_reference(args, w):
+    """The oracle on this host's cores; under N ranks only rank 0 works and
+    prints, the others exit 0 at once."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -381,8 +455,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(w), "global_batch": w.batch, "window": w.windows[0],
-                   "shift": w.shifts[0], "parallelism": "host cores"},
+        "config": bench_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -407,6 +480,8 @@ def run_rib(args, w):
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
+        if torch.cuda.device_count() < world:
+            raise SystemExit(f"{world} ranks but only {torch.cuda.device_count()} GPUs visible")
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     R.library()
 
@@ -506,9 +581,7 @@ def run_rib(args, w):
         ms = a.elapsed_time(b)
         if world > 1:
             dist.barrier()
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
+            ms = max_over_ranks(ms, dev)
         return ms, kern, None
 
     props = torch.cuda.get_device_properties(dev)
@@ -617,24 +690,24 @@ def run_rib(args, w):
     del qkvs, stack
     pk_s = peaks()
     sweep = config_sweep(I, R, dev, rank, world, timed, min(args.steps, 10), args.warmup,
-                         pk_s["bf16_tflops_sustained"], pk_s) if not args.no_sweep else None
+                         pk_s["bf16_tflops"], pk_s) if not args.no_sweep else None
     code, site = R.rib_last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {R.rib_status_string(code)} at site {site}")
 
     pk = peaks()
-    peak = pk["bf16_tflops_sustained"]
+    peak = pk["bf16_tflops"]
     launches = sum(n for n, _ in kern.values())
     per_kernel = {k: {"launches": n, "total_ms": t, "avg_ms": t / n,
                       "share": t / sum(x for _, x in kern.values())} for k, (n, t) in kern.items()}
     top = max(per_kernel, key=lambda k: per_kernel[k]["total_ms"])
     kflops = {"attn_bwd_kernel": f_bwd, "attn_fwd_kernel": f_fwd}
+    both = {k: roofline_entry(k, f, per_kernel[k]["avg_ms"], pk, stored_traffic(k, w.name))
+            for k, f in kflops.items() if k in per_kernel}
     roof = None
-    if top in kflops:
-        ach = kflops[top] / (per_kernel[top]["avg_ms"] * 1e-3) / 1e12
-        roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": peak,
-                "unit": "TFLOP/s", "frac": ach / peak, "traffic": stored_traffic(top, w.name),
-                "peak_source": f"{pk['source']} bf16_tflops_sustained (kernel inside a long step)"}
+    if top in both:
+        roof = dict(both[top])
+        roof["kernels"] = both
     fwd_k = kern_f.get("attn_fwd_kernel", (1, ms_f))
     fwd_ach = f_fwd / (fwd_k[1] / fwd_k[0] * 1e-3) / 1e12
 
@@ -728,9 +801,7 @@ def run_rib(args, w):
             t = a.elapsed_time(b)
             if world > 1:
                 dist.barrier()
-                tt = torch.tensor([t], device=dev)
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-                t = float(tt.item())
+                t = max_over_ranks(t, dev)
             return t
 
         piped(max(3, args.warmup // 2))
@@ -766,14 +837,12 @@ def run_rib(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) features and upstream grads, N(0,0.02) MLP weights)",
-        "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
-                   "map": [w.height, w.width], "window": M, "shift": s, "heads": heads,
-                   "head_dim": d, "rank": w.rank, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (qkv 170 MB + dout 57 MB per rank)"},
+        "config": bench_config(w, world),
         "tokens_per_s": tokens_s,
         "fwd": {"tflops": world * f_fwd / (ms_fwd * 1e-3) / 1e12, "ms": ms_fwd,
                 "tokens_per_s": world * w.tokens() / (ms_fwd * 1e-3),
-                "kernel_tflops": fwd_ach, "kernel_frac": fwd_ach / peak},
+                "kernel_tflops": fwd_ach, "kernel_frac": fwd_ach / peak,
+                "kernel_frac_of": "measured burst bf16 peak"},
         "roofline": roof,
         "cla": cla_line(w, kern_g, ms_g, ms_c, ms_fwd, pk, ms_cs, kern_cs, ms_step),
         "region_mask": mask_line(w, ms_m / args.steps, kern_m, f_fwd, f_bwd, peak),
@@ -794,6 +863,13 @@ def run_rib(args, w):
 
 def main():
     args = parse()
+    try:
+        plan = world_plan(args.gpus)
+    except ValueError as e:
+        print(f"bench.py: {e}", file=sys.stderr)
+        return 2
+    if plan == "relaunch":
+        return subprocess.call(relaunch_cmd(args.gpus, sys.argv[1:], free_port()))
     import rib_inputs as I
     w = I.get_workload(args.workload)
     if args.impl == "reference":

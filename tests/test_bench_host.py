@@ -138,3 +138,72 @@ def test_committed_traffic_records_are_well_formed():
         assert d["dram_bytes_per_launch"] == d["dram_bytes_read"] + d["dram_bytes_write"]
         assert len(d["source_hash"]) == 16
         assert "--clock-control none" in d["command"] and d["command"].startswith("ncu ")
+
+
+# ---------------------------------------------------------------- ranks
+
+def test_world_plan():
+    assert bench.world_plan(1, {}) == "run"
+    assert bench.world_plan(4, {}) == "relaunch"
+    assert bench.world_plan(2, {"WORLD_SIZE": "2"}) == "run"
+    assert bench.world_plan(1, {"WORLD_SIZE": "1"}) == "run"
+    with pytest.raises(ValueError, match="WORLD_SIZE=2"):
+        bench.world_plan(8, {"WORLD_SIZE": "2"})
+    with pytest.raises(ValueError, match="WORLD_SIZE=4"):
+        bench.world_plan(1, {"WORLD_SIZE": "4"})
+    with pytest.raises(ValueError):
+        bench.world_plan(0, {})
+
+
+def test_relaunch_command_starts_n_ranks_of_this_script():
+    cmd = bench.relaunch_cmd(8, ["--gpus", "8", "--steps", "3"], 29511)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=8" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[cmd.index("--master-port") + 1] == "29511"
+    assert cmd[-4:] == ["--gpus", "8", "--steps", "3"]
+    assert os.path.samefile(cmd[-5], os.path.join(ROOT, "bench.py"))
+
+
+def test_both_arms_share_one_config_object():
+    w = get_workload("w96train")
+    c = bench.bench_config(w, 2)
+    assert c["global_batch"] == 8 and c["parallelism"] == "dp2"
+    assert c["map"] == [192, 192] and (c["window"], c["shift"]) == (96, 48)
+    assert (c["heads"], c["head_dim"], c["rank"]) == (6, 32, 16)
+    assert c["workload"].startswith("w96train:")
+
+
+def test_roofline_divides_by_the_burst_peak():
+    pk = {"bf16_tflops": 1665.3, "bf16_tflops_sustained": 1404.1, "source": "measured"}
+    e = bench.roofline_entry("attn_bwd_kernel", 3.392e12, 4.655, pk)
+    assert e["achieved"] == pytest.approx(3.392e12 / 4.655e-3 / 1e12)
+    assert e["peak"] == 1665.3
+    assert e["frac"] == pytest.approx(0.4376, abs=1e-4)
+    assert e["frac_of_sustained"] == pytest.approx(e["achieved"] / 1404.1)
+    assert "burst" in e["peak_source"]
+
+
+def _max_over_ranks_worker(rank, world, port, q):
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        q.put((rank, bench.max_over_ranks([3.5, 7.25][rank], "cpu")))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = bench.free_port()
+    ps = [ctx.Process(target=_max_over_ranks_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == {0: 7.25, 1: 7.25}

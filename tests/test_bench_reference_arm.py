@@ -55,3 +55,29 @@ def test_reference_arm_under_torchrun_prints_once():
     lines = _lines(r.stdout)
     assert len(lines) == 1
     _check_line(lines[0], 2, 1, 3)
+
+
+def test_gpus_n_without_launcher_starts_n_ranks():
+    """--gpus 2 with no outer launcher re-launches itself as two ranks; only
+    rank 0 prints, and the line reports both."""
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3"], cwd=ROOT,
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _lines(r.stdout)
+    assert len(lines) == 1
+    _check_line(lines[0], 2, 1, 3)
+    assert lines[0]["config"]["parallelism"] == "dp2"
+
+
+def test_gpus_n_mismatching_the_launcher_fails():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "8", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3"], cwd=ROOT,
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode == 2
+    assert "WORLD_SIZE=2" in r.stderr
+    assert not _lines(r.stdout)
