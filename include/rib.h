@@ -266,6 +266,15 @@ size_t rib_window_attn_bwd_workspace(int B, int H, int W, int heads,
  * weight gradients are computed from dqp/dkp as well (sums over tokens in a
  * fixed order).
  *
+ * Reproducibility: dKc, dV, dkp and the key MLP's gradients are bit-identical
+ * from call to call (each key tile's sums run in query-tile order inside one
+ * CTA; dkp and the MLP sums are fixed-order reductions).  dQc, dqp and the
+ * query MLP's gradients are NOT: every key tile of a unit adds its dQ_aug
+ * partial to one fp32 accumulator per query tile with a bulk reduce-add, and
+ * the order of those adds depends on how the CTAs are scheduled.  Repeated
+ * calls agree to fp32 rounding of the accumulator (within the stated
+ * tolerance), not bit for bit.
+ *
  *   qkv, out, lse : as produced for / by rib_window_attn_fwd
  *   dout     : bf16 [B][H][W][heads][head_dim]
  *   dqkv     : out, bf16 [B][H][W][3][heads][head_dim]

@@ -25,3 +25,19 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With RIB_PARITY_LOG set, every parity comparison of the run (absolute
+    and normalised error figures) is written there as JSON lines."""
+    path = os.environ.get("RIB_PARITY_LOG")
+    if not path:
+        return
+    try:
+        from tests.rib_testlib import RECORDS
+    except Exception:  # pragma: no cover
+        return
+    import json
+    with open(path, "w") as f:
+        for r in RECORDS:
+            f.write(json.dumps(r) + "\n")

@@ -7,6 +7,8 @@ compared on exactly the values it consumes.
 """
 from __future__ import annotations
 
+import re
+
 import numpy as np
 import torch
 
@@ -25,24 +27,50 @@ def stats(got, ref):
     return float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0
 
 
-def check_close(got, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS, normalize=False):
-    """Returns an error message ('' if within bounds).  normalize=True divides
-    the errors by max(1, max|ref|) first, and a number divides them by
-    max(1, that number): used for fp32 sums whose magnitude grows with the
-    number of windows or tokens summed (dQp, dKp, MLP weight gradients),
-    whose bf16-level errors grow in proportion."""
+# Tensors whose error may be judged relative to their magnitude (besides the
+# absolute figure, which is always computed and reported): fp32 sums over
+# windows or tokens (dQp, dKp, the position-MLP and CLA weight gradients) and
+# the CLA's dO = dO' * G, which carries the upstream gradient's magnitude.
+NORMALISED = {"dqp", "dkp", "dw1", "db1", "dw2", "db2", "dw", "db", "do"}
+
+# every comparison made in this process: name, absolute and normalised
+# figures (written out as JSON lines when RIB_PARITY_LOG names a file)
+RECORDS = []
+
+
+def check_close(got, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS, normalize=False,
+                grown_inputs=False):
+    """Returns an error message ('' if within bounds).
+
+    The absolute max/mean errors are always computed, reported and recorded.
+    normalize=True divides the errors by max(1, max|ref|) before the bounds
+    are applied, and a number divides them by max(1, that number).  It is
+    allowed only for the tensors named in NORMALISED, whose magnitude grows
+    with the number of windows or tokens summed, and for cases whose inputs
+    are scaled up on purpose (grown_inputs=True)."""
     mx, mn = stats(got, ref)
+    refmax = float(np.abs(np.asarray(ref, dtype=np.float64)).max()) if np.size(ref) else 0.0
+    if normalize:
+        tokens = set(re.split(r"[ _]", what.lower()))
+        assert grown_inputs or tokens & NORMALISED, \
+            f"{what}: a magnitude-relative bound is not allowed for this tensor"
     if normalize is True:
-        scale = max(1.0, float(np.abs(np.asarray(ref, dtype=np.float64)).max()))
+        scale = max(1.0, refmax)
     elif normalize:
         scale = max(1.0, float(normalize))
     else:
         scale = 1.0
+    abs_ok = mx <= max_abs and mn <= mean_abs
     ok = mx / scale <= max_abs and mn / scale <= mean_abs
-    msg = (f"{what}: max|d|={mx:.3e}, mean|d|={mn:.3e}, max|ref|="
-           f"{float(np.abs(np.asarray(ref, dtype=np.float64)).max()):.3e}"
-           f"{' (normalised by %.3e)' % scale if normalize else ''} bounds {max_abs}/{mean_abs}")
+    msg = (f"{what}: abs max|d|={mx:.3e} mean|d|={mn:.3e} "
+           f"({'within' if abs_ok else 'beyond'} {max_abs}/{mean_abs}), max|ref|={refmax:.3e}")
+    if normalize:
+        msg += (f"; normalised by {scale:.3e}: max {mx / scale:.3e} mean {mn / scale:.3e} "
+                f"({'within' if ok else 'beyond'} bounds)")
     print(msg)
+    RECORDS.append({"what": what, "max_abs": mx, "mean_abs": mn, "max_ref": refmax,
+                    "abs_within": abs_ok, "normalised_by": scale if normalize else None,
+                    "within": ok})
     return "" if ok else msg
 
 

@@ -1,0 +1,56 @@
+"""Repeatability of the backward.
+
+The key-side gradients (dKc, dV, dKp, the key MLP's weight gradients) come
+from sums in a fixed order and must be bit-identical from call to call.  The
+query-side ones (dQc, dQp, the query MLP's weight gradients) are folded into
+an fp32 accumulator by every key tile of a unit, in an order set by CTA
+scheduling: two calls must agree within the parity tolerance, and the test
+reports how far apart they are.  The forward (one CTA owns each query tile)
+must be bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+import rib_inputs as I
+import windowed_attention_implicit_b200 as R
+from tests.rib_testlib import assert_all, check_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name,B", [("w32", 2), ("w96train", 4)])
+def test_backward_repeatability(name, B):
+    w = I.get_workload(name)
+    inp = I.make_layer_inputs(w, 0, strong=True)
+    M, s = w.windows[0], w.shifts[0]
+    qkv, dout = inp["qkv"][:B].cuda(), inp["dout"][:B].cuda()
+    mlp = R.PositionMLP.from_params(inp["freqs"], inp["mlp_q"], inp["mlp_k"], w.heads, w.rank)
+    _, _, q16, k16 = R.rib_pos_tokens(mlp, M)
+    runs = []
+    for _ in range(3):
+        out, lse = R.rib_window_attn_fwd(qkv, M, s, q16, k16)
+        g = R.rib_window_attn_bwd(qkv, out, dout, lse, M, s, q16, k16, mlp=mlp)
+        torch.cuda.synchronize()
+        assert R.rib_last_status()[0] == 0
+        runs.append((out.clone(), lse.clone(), g))
+    (o0, l0, g0) = runs[0]
+    checks = []
+    for o, l, g in runs[1:]:
+        assert torch.equal(o, o0) and torch.equal(l, l0), "forward must be bit-identical"
+        assert torch.equal(g["dqkv"][:, :, :, 1:], g0["dqkv"][:, :, :, 1:]), "dKc / dV"
+        assert torch.equal(g["dkp"], g0["dkp"]), "dKp"
+        for n in ("k_dw1", "k_db1", "k_dw2", "k_db2"):
+            assert torch.equal(getattr(g["dmlp"], n), getattr(g0["dmlp"], n)), n
+        checks.append(check_close(to_np(g["dqkv"][:, :, :, 0]), to_np(g0["dqkv"][:, :, :, 0]),
+                                  "dQc call to call"))
+        checks.append(check_close(to_np(g["dqp"]), to_np(g0["dqp"]), "dQp call to call",
+                                  normalize=True))
+        for n in ("q_dw1", "q_db1", "q_dw2", "q_db2"):
+            a, b = to_np(getattr(g["dmlp"], n)), to_np(getattr(g0["dmlp"], n))
+            rel = np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)
+            print(f"{n} call to call: rel {rel:.3e}")
+            checks.append("" if rel <= 1e-4 else f"{n} rel {rel:.3e}")
+        same = torch.equal(g["dqkv"][:, :, :, 0], g0["dqkv"][:, :, :, 0])
+        print(f"{name}: dQc bit-identical across calls: {same}")
+    assert_all(checks)

@@ -5,8 +5,9 @@ gradients: code running while a CUDA graph is captured, hosts whose allocator
 owns all device memory, or loops that cannot afford the synchronisation of a
 cudaMalloc/cudaFree pair.  This entry point serves them with a scratch array
 compiled into the library.  The test calls it through the C ABI twice in a
-row, on different inputs, and checks each result against the workspace-based
-rib_pos_tokens_bwd, with the same bound the other MLP-backward tests use.
+row, on different inputs, and checks each result against the fp64 oracle's
+MLP backward and against the workspace-based rib_pos_tokens_bwd, with the
+same bound the other MLP-backward tests use.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import rib_inputs as I
 import windowed_attention_implicit_b200 as R
 from windowed_attention_implicit_b200 import _abi
@@ -48,11 +50,17 @@ def test_noalloc_matches_workspace_version_twice(M, hid):
         ref = R.rib_pos_tokens_bwd(mlp, M, gq, gk)
         torch.cuda.synchronize()
         assert R.rib_last_status()[0] == 0
-        for name in ("q_dw1", "q_db1", "q_dw2", "q_db2", "k_dw1", "k_db1", "k_dw2", "k_db2"):
+        rq, rk = O.pos_tokens_backward(freqs, mq, mk, M, gq.double().cpu().numpy(),
+                                       gk.double().cpu().numpy())
+        exact = dict(zip(("q_dw1", "q_db1", "q_dw2", "q_db2"), rq))
+        exact.update(zip(("k_dw1", "k_db1", "k_dw2", "k_db2"), rk))
+        for name, e in exact.items():
             a = getattr(got, name).double().cpu().numpy()
             b = getattr(ref, name).double().cpu().numpy()
+            rel = np.abs(a - e).max() / np.abs(e).max()
+            assert rel <= MLP_REL, f"call {call} {name} vs oracle: rel {rel:.3e}"
             rel = np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)
-            assert rel <= MLP_REL, f"call {call} {name}: rel {rel:.3e}"
+            assert rel <= MLP_REL, f"call {call} {name} vs workspace call: rel {rel:.3e}"
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

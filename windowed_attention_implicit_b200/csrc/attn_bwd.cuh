@@ -13,7 +13,9 @@
 //   attn_bwd_kernel  one CTA per (key tile, unit): keeps K, V, Kp of its 128
 //                    keys in shared memory and streams the unit's query
 //                    tiles; dK, dV accumulate in TMEM; dQ partials go to an
-//                    fp32 accumulator with vector atomics
+//                    fp32 accumulator through one bulk TMA reduce-add per
+//                    query tile (the order of the key tiles' adds follows
+//                    CTA scheduling, so dQ is not bit-reproducible)
 //   dq_finalize      dQ content channels -> bf16 dqkv at the rolled pixels
 //   posgrad_reduce   fixed-order sums over (batch, window) of dQp, dKp
 //

@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -553,6 +554,22 @@ int rib_pos_tokens_bwd_noalloc(const rib_mlp_t* mlp, int window, const float* dq
                         static_cast<cudaStream_t>(stream));
 }
 
+// Kernels that move registers between warpgroups with setmaxnreg are only
+// safe when compiled to the per-thread launch budget their split assumes.
+// The count is a property of the library's one sm_100a image, so it is read
+// once per kernel variant and cached (atomically: calls may come from any
+// thread, for any device).
+static int check_launch_regs(const void* kern, std::atomic<int>& cache, int expected) {
+  int regs = cache.load(std::memory_order_acquire);
+  if (regs < 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return RIB_ERR_CUDA;
+    regs = fa.numRegs;
+    cache.store(regs, std::memory_order_release);
+  }
+  return regs == expected ? RIB_OK : RIB_ERR_UNSUPPORTED;
+}
+
 static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int head_dim,
                            int window, int shift, const void* qp_bf16, const void* kp_bf16,
                            int rank, float scale, void* out, float* lse, const void* gate,
@@ -594,14 +611,9 @@ static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int 
   if ((rc = set_smem(kern, kFwdSmemBytes))) return rc;
   {
     // setmaxnreg split: only safe with the launch budget it was sized for
-    static int launch_regs[2] = {-1, -1};
-    int& lr = launch_regs[p.region_mask ? 1 : 0];
-    if (lr < 0) {
-      cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return RIB_ERR_CUDA;
-      lr = fa.numRegs;
-    }
-    if (lr != kFwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
+    static std::atomic<int> launch_regs[2] = {{-1}, {-1}};
+    if ((rc = check_launch_regs(reinterpret_cast<const void*>(kern), launch_regs[p.region_mask ? 1 : 0], kFwdLaunchRegs)))
+      return rc;
   }
   // one CTA per SM walks the work items (unit, pair of query tiles)
   int sms = 0;
@@ -893,14 +905,9 @@ static int attn_bwd_launch(const void* qkv, const void* out, const void* dout,
   {
     // The kernel moves registers between warpgroups with setmaxnreg; that is
     // only safe if the compiled launch budget is the one the split assumes.
-    static int launch_regs[2] = {-1, -1};
-    int& lr = launch_regs[p.region_mask ? 1 : 0];
-    if (lr < 0) {
-      cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return RIB_ERR_CUDA;
-      lr = fa.numRegs;
-    }
-    if (lr != kBwdLaunchRegs) return RIB_ERR_UNSUPPORTED;
+    static std::atomic<int> launch_regs[2] = {{-1}, {-1}};
+    if ((rc = check_launch_regs(reinterpret_cast<const void*>(kern), launch_regs[p.region_mask ? 1 : 0], kBwdLaunchRegs)))
+      return rc;
   }
   {
     TraceScope ts(K_BWD, st);
