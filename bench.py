@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="rib", choices=["rib", "reference"])
     ap.add_argument("--workload", default="w96train")
+    ap.add_argument("--bwd-kernel", default="auto", choices=["auto", "per_item", "persistent"],
+                    help="form of the attention backward kernel (default: by window size)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
@@ -299,6 +301,32 @@ def config_sweep(I, R, dev, rank, world, timed, steps, warmup, peak, pk):
         res[name] = line
         del layers, qkvs, stack
         torch.cuda.empty_cache()
+    # the tiny workload as stated, in fp32: its forward on the tf32 path
+    w = I.get_workload("tiny", seed=I.get_workload("tiny").seed + 7919 * rank)
+    inp = I.make_layer_inputs(w, 0, qkv_dtype=torch.float32)
+    mlp = R.PositionMLP.from_params(inp["freqs"], inp["mlp_q"], inp["mlp_k"], w.heads, w.rank,
+                                    device=dev)
+    M, sh = w.windows[0], w.shifts[0]
+    qkv32 = inp["qkv"].to(dev)
+    qp32, kp32, _, _ = R.rib_pos_tokens(mlp, M)
+    out32 = torch.empty((w.batch, w.height, w.width, w.heads, w.head_dim), device=dev)
+    lse32 = torch.empty((w.batch, w.heads, w.height, w.width), device=dev)
+
+    def fwd32():
+        R.rib_window_attn_fwd_tf32(qkv32, M, sh, qp32, kp32, out=out32, lse=lse32)
+
+    for _ in range(warmup):
+        fwd32()
+    ms32, kern32, _ = timed(fwd32, steps, trace=True)
+    ms32 /= steps
+    f32 = 160.0 * (M * M) ** 2 * w.units(0)
+    k32 = kern32.get("attn_fwd_tf32_kernel", (1, ms32 * steps))
+    res["tiny_fp32"] = {"layers": 1, "windows": [M], "shifts": [sh],
+                        "map": [w.batch, w.height, w.width], "heads": w.heads,
+                        "precision": "fp32 inputs, tf32 tensor cores (kind::tf32), fp32 out",
+                        "fwd_ms": ms32, "fwd_tflops": world * f32 / (ms32 * 1e-3) / 1e12,
+                        "fwd_tokens_per_s": world * w.tokens() / (ms32 * 1e-3),
+                        "fwd_kernel_ms": k32[1] / k32[0]}
     return res
 
 
@@ -363,7 +391,8 @@ def mask_line(w, ms_step, kern, f_fwd, f_bwd, peak):
     per = {k: v[1] / v[0] for k, v in kern.items()}
     line = {"training_step_ms": ms_step, "kernels_ms": per,
             "workload": f"{w.name} with the mask of shift {w.shifts[0]}"}
-    for k, f in (("attn_fwd_kernel", f_fwd), ("attn_bwd_kernel", f_bwd)):
+    for k, f in (("attn_fwd_kernel", f_fwd), ("attn_bwd_kernel", f_bwd),
+                 ("attn_bwd_persistent_kernel", f_bwd)):
         if k in per:
             line[k.replace("attn_", "").replace("_kernel", "") + "_frac"] = (
                 f / (per[k] * 1e-3) / 1e12 / peak)
@@ -484,6 +513,9 @@ def run_rib(args, w):
             raise SystemExit(f"{world} ranks but only {torch.cuda.device_count()} GPUs visible")
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     R.library()
+    from windowed_attention_implicit_b200 import _abi
+    R.rib_set_bwd_kernel({"auto": _abi.RIB_BWD_AUTO, "per_item": _abi.RIB_BWD_PER_ITEM,
+                          "persistent": _abi.RIB_BWD_PERSISTENT}[args.bwd_kernel])
 
     M, s = w.windows[0], w.shifts[0]
     # each rank trains on its own batch: seeds differ per rank (weak scaling)
@@ -701,7 +733,8 @@ def run_rib(args, w):
     per_kernel = {k: {"launches": n, "total_ms": t, "avg_ms": t / n,
                       "share": t / sum(x for _, x in kern.values())} for k, (n, t) in kern.items()}
     top = max(per_kernel, key=lambda k: per_kernel[k]["total_ms"])
-    kflops = {"attn_bwd_kernel": f_bwd, "attn_fwd_kernel": f_fwd}
+    kflops = {"attn_bwd_kernel": f_bwd, "attn_bwd_persistent_kernel": f_bwd,
+              "attn_fwd_kernel": f_fwd}
     both = {k: roofline_entry(k, f, per_kernel[k]["avg_ms"], pk, stored_traffic(k, w.name))
             for k, f in kflops.items() if k in per_kernel}
     roof = None

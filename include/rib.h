@@ -199,6 +199,33 @@ int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw,
                  void* gate, void* stream);
 
 /* ------------------------------------------------------------------------
+ * rib_window_attn_fwd_tf32 -- RIB window attention forward for fp32 inputs.
+ *
+ * The same computation as rib_window_attn_fwd (English summary §2.A steps
+ * 3-4 and the score equation: S = scale * [Qc,Qp][Kc,Kp]^T, P =
+ * softmax_rows(S), O = P V, lse = ln sum_k exp(S[:,k])), for features and
+ * position tokens kept in fp32: nothing is rounded to bf16.  The tcgen05
+ * tensor cores read the fp32 operands as tf32 (10 explicit mantissa bits)
+ * and accumulate in fp32; P is rounded to tf32 (to nearest) before the PV
+ * product and the softmax denominator is summed from the rounded P.
+ *
+ *   qkv      : fp32 [B][H][W][3][heads][head_dim]  (Qc, Kc, V)
+ *   qp, kp   : fp32 [heads][M][M][rank], e.g. the fp32 outputs of
+ *              rib_pos_tokens (ignored when rank == 0)
+ *   rank     : 0 or 16
+ *   scale    : softmax scale; <= 0 selects 1/sqrt(head_dim + rank)
+ *   out      : out, fp32 [B][H][W][heads][head_dim]
+ *   lse      : out, fp32 [B][heads][H][W] (natural log)
+ * Same shape support, errors and B == 0 behaviour as rib_window_attn_fwd;
+ * every pointer 16-byte aligned (RIB_ERR_ALIGN).  Device pointers, caller
+ * owned; asynchronous on `stream`.  No shift mask, no CLA gate.
+ * ------------------------------------------------------------------------ */
+int rib_window_attn_fwd_tf32(const float* qkv, int B, int H, int W, int heads,
+                             int head_dim, int window, int shift, const float* qp,
+                             const float* kp, int rank, float scale, float* out,
+                             float* lse, void* stream);
+
+/* ------------------------------------------------------------------------
  * rib_window_attn_fwd_cla -- rib_window_attn_fwd with the CLA gate applied
  * in the same kernel's epilogue (German summary, Methodik §B: O' = O * G).
  *
@@ -356,6 +383,24 @@ const char* rib_status_string(int status);
  * kernel since the previous call (RIB_OK if none) and clears it.  If `site`
  * is non-NULL it receives a code naming the wait that gave up. */
 int rib_last_status(int* site);
+
+/* Form of the attention backward kernel (rib_window_attn_bwd and
+ * rib_window_attn_bwd_masked).  Both compute the same gradients (the same
+ * arithmetic in the same order per key tile):
+ *   RIB_BWD_PER_ITEM    one CTA per (unit, key tile);
+ *   RIB_BWD_PERSISTENT  one CTA per SM walking the (unit, key tile) items,
+ *                       the next item's loads and MMAs overlapping the end
+ *                       of the current one;
+ *   RIB_BWD_AUTO        (default) the persistent form for windows up to
+ *                       64 x 64, where per-CTA set-up weighs on few query
+ *                       tiles, and the per-item form above.
+ * rib_set_bwd_kernel sets it process-wide (RIB_ERR_ARG for another value);
+ * rib_bwd_kernel_for returns the form a call with this window would use. */
+#define RIB_BWD_AUTO         0
+#define RIB_BWD_PER_ITEM     1
+#define RIB_BWD_PERSISTENT   2
+int rib_set_bwd_kernel(int which);
+int rib_bwd_kernel_for(int window);
 
 /* Time limit, in nanoseconds, of every bounded wait in kernels launched
  * after this call (process-wide; default 1e9 = 1 s; 0 restores it). */

@@ -156,11 +156,12 @@ def make_mlp(n_freq, hidden, heads, rank, seed, which, strong=False):
 
 
 def make_layer_inputs(w: Workload, layer: int = 0, strong: bool = False,
-                      with_dout: Optional[bool] = None):
-    """All host-side inputs of one layer of workload w (CPU tensors)."""
+                      with_dout: Optional[bool] = None, qkv_dtype=torch.bfloat16):
+    """All host-side inputs of one layer of workload w (CPU tensors).
+    qkv_dtype=torch.float32 keeps the features unrounded (the fp32 path)."""
     seed = w.seed + 1000 * layer
     mlp_seed = w.seed if w.shared_mlp else seed
-    qkv = make_qkv(w.batch, w.height, w.width, w.heads, w.head_dim, seed)
+    qkv = make_qkv(w.batch, w.height, w.width, w.heads, w.head_dim, seed, dtype=qkv_dtype)
     out = {
         "qkv": qkv,
         "freqs": default_freqs(w.n_freq),

@@ -8,6 +8,18 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+@pytest.fixture(params=["per_item", "persistent"])
+def bwd_kernel(request):
+    """Runs the test once with each form of the attention backward kernel
+    forced (process-wide), and restores the window-size dispatch after."""
+    import windowed_attention_implicit_b200 as R
+    from windowed_attention_implicit_b200 import _abi
+    which = {"per_item": _abi.RIB_BWD_PER_ITEM, "persistent": _abi.RIB_BWD_PERSISTENT}
+    R.rib_set_bwd_kernel(which[request.param])
+    yield request.param
+    R.rib_set_bwd_kernel(_abi.RIB_BWD_AUTO)
+
+
 def pytest_configure(config):
     config.addinivalue_line(
         "markers", "gpu: needs a CUDA device (B200, sm_100a) and the built library")

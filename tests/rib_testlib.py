@@ -20,6 +20,69 @@ MEAN_ABS = 2e-3
 POS_REL = 1e-5     # Qp/Kp fp32: max|d| / max|ref|
 
 
+def tf32_error_bounds(qkv, qp, kp, M, s, tau, row_block=512):
+    """First-order elementwise error bounds of the fp32 forward on the tf32
+    tensor cores against the exact result, from tf32's 10 explicit mantissa
+    bits.  Per unit, with augmented rows q_i = [Qc_i, Qp_i], k_j = [Kc_j, Kp_j]:
+
+      the MMA reads every operand as tf32: |relative error| <= 2^-10 each
+      (2^-10 whether it truncates or rounds), so a logit s_ij = tau q_i.k_j
+      is off by at most  e_ij = (2 * 2^-10 + 48 * 2^-24) tau sum_k |q_ik k_jk|
+      (the second term: fp32 accumulation of 48 products);
+      lse_i = ln sum_j exp(s_ij) moves by at most max_j e_ij;
+      P is perturbed by e_ij, by its rounding to tf32 (2^-11, to nearest) and
+      by the hardware exp2 (< 2^-20); V by 2^-10; to first order
+        |dO_ic| <= sum_j P_ij (e_ij + 2^-11 + 2^-20) |v_jc - O_ic|
+                   + (2^-10 + N 2^-24) sum_j P_ij |v_jc|.
+
+    Returns (out_bound [B][H][W][heads][d], lse_bound [B][heads][H][W]) at
+    the map's pixels, computed in fp64 from the same inputs as the oracle."""
+    x = O.window_partition(np.asarray(qkv, dtype=np.float64), M, s)
+    B, nW, N, _, heads, d = x.shape
+    qp = np.asarray(qp, dtype=np.float64).reshape(heads, N, -1)
+    kp = np.asarray(kp, dtype=np.float64).reshape(heads, N, -1)
+    r = qp.shape[-1]
+    ob = np.empty((B, nW, N, heads, d))
+    lb = np.empty((B, nW, N, heads))
+    e_log = 2.0 ** -9 + (d + r) * 2.0 ** -24
+    for b in range(B):
+        for w in range(nW):
+            for h in range(heads):
+                qa = np.concatenate([x[b, w, :, 0, h], qp[h]], 1)
+                ka = np.concatenate([x[b, w, :, 1, h], kp[h]], 1)
+                v = x[b, w, :, 2, h]
+                for r0 in range(0, N, row_block):
+                    r1 = min(N, r0 + row_block)
+                    e = e_log * tau * (np.abs(qa[r0:r1]) @ np.abs(ka).T)
+                    sc = tau * (qa[r0:r1] @ ka.T)
+                    pm = np.exp(sc - sc.max(1, keepdims=True))
+                    pm /= pm.sum(1, keepdims=True)
+                    o = pm @ v
+                    lb[b, w, r0:r1, h] = e.max(1)
+                    ep = pm * (e + 2.0 ** -11 + 2.0 ** -20)
+                    dev = np.abs(v[None, :, :] - o[:, None, :])       # [rows, N, d]
+                    ob[b, w, r0:r1, h] = (np.einsum("ij,ijc->ic", ep, dev) +
+                                          (2.0 ** -10 + N * 2.0 ** -24) * (pm @ np.abs(v)))
+    H, W = np.asarray(qkv).shape[1:3]
+    out_b = O.window_reverse(ob, M, s, H, W)
+    lse_b = O.window_reverse(lb, M, s, H, W).transpose(0, 3, 1, 2)
+    # second-order terms and the few ulps of the fp32 rescales: 5 % + 1e-6
+    return 1.05 * out_b + 1e-6, 1.05 * lse_b + 1e-6
+
+
+def check_within_bound(got, ref, bound, what):
+    """'' if |got - ref| <= bound elementwise, else a message; prints the
+    largest ratio of error to bound."""
+    err = np.abs(np.asarray(got, dtype=np.float64) - np.asarray(ref, dtype=np.float64))
+    ratio = float((err / bound).max()) if err.size else 0.0
+    msg = f"{what}: max |d| / bound = {ratio:.3f} (max |d| {err.max():.3e}, max bound {bound.max():.3e})"
+    print(msg)
+    RECORDS.append({"what": what + " (tf32 bound)", "max_abs": float(err.max()),
+                    "mean_abs": float(err.mean()), "max_ref": float(np.abs(ref).max()),
+                    "abs_within": ratio <= 1.0, "normalised_by": None, "within": ratio <= 1.0})
+    return "" if ratio <= 1.0 else msg
+
+
 def stats(got, ref):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

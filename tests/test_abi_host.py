@@ -281,3 +281,23 @@ def test_work_entry_points_run_inside_nvtx_ranges(monkeypatch):
     assert log == [("push", "rib_window_scatter"), "pop"]
     # the real library: the wrapped entry points keep their names
     assert R.library().rib_cla_bwd.__name__ == "rib_cla_bwd"
+
+
+def test_backward_form_dispatch_by_window_and_override():
+    """Windows up to 64 x 64 take the persistent backward, larger ones the
+    per-item kernel; a forced form applies to every window until reset."""
+    lib = R.library()
+    assert lib.rib_bwd_kernel_for(16) == _abi.RIB_BWD_PERSISTENT
+    assert lib.rib_bwd_kernel_for(64) == _abi.RIB_BWD_PERSISTENT
+    assert lib.rib_bwd_kernel_for(96) == _abi.RIB_BWD_PER_ITEM
+    assert lib.rib_bwd_kernel_for(256) == _abi.RIB_BWD_PER_ITEM
+    try:
+        R.rib_set_bwd_kernel(_abi.RIB_BWD_PER_ITEM)
+        assert R.rib_bwd_kernel_for(16) == _abi.RIB_BWD_PER_ITEM
+        R.rib_set_bwd_kernel(_abi.RIB_BWD_PERSISTENT)
+        assert R.rib_bwd_kernel_for(96) == _abi.RIB_BWD_PERSISTENT
+        assert lib.rib_set_bwd_kernel(7) == _abi.RIB_ERR_ARG
+        assert R.rib_bwd_kernel_for(96) == _abi.RIB_BWD_PERSISTENT   # unchanged by the refusal
+    finally:
+        R.rib_set_bwd_kernel(_abi.RIB_BWD_AUTO)
+    assert R.rib_bwd_kernel_for(32) == _abi.RIB_BWD_PERSISTENT

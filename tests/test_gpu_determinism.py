@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("name,B", [("w32", 2), ("w96train", 4)])
-def test_backward_repeatability(name, B):
+def test_backward_repeatability(name, B, bwd_kernel):
     w = I.get_workload(name)
     inp = I.make_layer_inputs(w, 0, strong=True)
     M, s = w.windows[0], w.shifts[0]

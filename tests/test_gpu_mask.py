@@ -25,7 +25,7 @@ def _ids(c):
 
 
 @pytest.mark.parametrize("case", MASK_CASES, ids=[_ids(c) for c in MASK_CASES])
-def test_masked_fwd_bwd_parity(case):
+def test_masked_fwd_bwd_parity(case, bwd_kernel):
     B, H, W, heads, M, s, rank = case
     c = Case(B, H, W, heads, M, s, rank=rank, seed=21)
     d = c.device()

@@ -134,7 +134,7 @@ def test_fwd_explicit_scale_and_default_agree():
 
 
 @pytest.mark.parametrize("case", FWD_CASES, ids=[_ids(c) for c in FWD_CASES])
-def test_bwd_parity(case):
+def test_bwd_parity(case, bwd_kernel):
     B, H, W, heads, M, s, rank, strong = case
     c = Case(B, H, W, heads, M, s, rank=rank, strong=strong, seed=13)
     d = c.device()
@@ -153,7 +153,7 @@ def test_bwd_parity(case):
     assert_all(checks)
 
 
-def test_bwd_mlp_grads_parity():
+def test_bwd_mlp_grads_parity(bwd_kernel):
     """Training step of the w32 shape at reduced batch: MLP weight grads from
     the kernel chain (pos tokens -> attention bwd -> MLP bwd) vs the oracle."""
     B, H, W, heads, M, s = 1, 64, 64, 6, 32, 16

@@ -16,7 +16,7 @@ from tests.rib_testlib import assert_all, bf16_round, check_close, to_np
 pytestmark = pytest.mark.gpu
 
 
-def test_cyclic_window_schedule_fwd_bwd():
+def test_cyclic_window_schedule_fwd_bwd(bwd_kernel):
     w = I.get_workload("cyclic", batch=1, heads=2)
     layers, inputs = [], []
     for l in range(w.layers):

@@ -25,9 +25,10 @@ from . import _abi
 __all__ = [
     "RibError", "PositionMLP", "PositionMLPGrad", "PosTokenCache", "rib_pos_tokens",
     "rib_pos_tokens_bwd", "rib_pos_tokens_bwd_workspace", "rib_pos_tokens_bwd_noalloc",
-    "rib_window_attn_fwd", "rib_window_attn_bwd", "rib_window_attn_bwd_workspace",
+    "rib_window_attn_fwd", "rib_window_attn_fwd_tf32", "rib_window_attn_bwd",
+    "rib_window_attn_bwd_workspace",
     "rib_window_gather", "rib_window_scatter", "rib_last_status", "rib_status_string",
-    "rib_set_wait_limit_ns", "rib_debug_wait_timeout", "rib_version", "library",
+    "rib_set_wait_limit_ns", "rib_set_bwd_kernel", "rib_bwd_kernel_for", "rib_debug_wait_timeout", "rib_version", "library",
     "rib_trace_enable", "rib_trace_collect", "rib_debug_exp2", "ClaGate", "rib_cla_gate",
     "rib_window_attn_fwd_cla", "rib_cla_bwd", "rib_cla_bwd_workspace",
 ]
@@ -336,6 +337,28 @@ def rib_window_attn_fwd(qkv: torch.Tensor, window: int, shift: int, qp_bf16=None
     return out, lse
 
 
+def rib_window_attn_fwd_tf32(qkv: torch.Tensor, window: int, shift: int, qp=None, kp=None,
+                             rank: int = 16, scale: float = 0.0, out=None, lse=None,
+                             stream=None):
+    """fp32 forward on the tf32 tensor cores: qkv fp32 [B][H][W][3][heads][d],
+    qp/kp fp32 [heads][M][M][rank]; returns out fp32 [B][H][W][heads][d] and
+    lse fp32 [B][heads][H][W]."""
+    B, H, W, three, heads, d = qkv.shape
+    if three != 3:
+        raise ValueError("qkv must be [B][H][W][3][heads][head_dim]")
+    out = torch.empty((B, H, W, heads, d), device=qkv.device, dtype=torch.float32) if out is None else out
+    lse = torch.empty((B, heads, H, W), device=qkv.device, dtype=torch.float32) if lse is None else lse
+    nt = heads * int(window) ** 2 * int(rank)
+    name = "rib_window_attn_fwd_tf32"
+    _sizes(name, qkv.device, out=(out, B * H * W * heads * d), lse=(lse, B * heads * H * W),
+           qp=(qp if rank > 0 else None, nt), kp=(kp if rank > 0 else None, nt))
+    _check(library().rib_window_attn_fwd_tf32(
+        _ptr(qkv, torch.float32, "qkv"), B, H, W, heads, d, int(window), int(shift),
+        _ptr(qp, torch.float32, "qp"), _ptr(kp, torch.float32, "kp"), int(rank), float(scale),
+        _ptr(out, torch.float32, "out"), _ptr(lse, torch.float32, "lse"), _stream(stream)), name)
+    return out, lse
+
+
 @dataclass
 class ClaGate:
     """Device fp32 weights of the convolutional local attention gate:
@@ -517,6 +540,17 @@ def rib_last_status() -> Tuple[int, int]:
 
 def rib_set_wait_limit_ns(limit_ns: int) -> None:
     _check(library().rib_set_wait_limit_ns(int(limit_ns)), "rib_set_wait_limit_ns")
+
+
+def rib_set_bwd_kernel(which: int) -> None:
+    """Form of the attention backward kernel, process-wide: _abi.RIB_BWD_AUTO
+    (by window size), RIB_BWD_PER_ITEM or RIB_BWD_PERSISTENT."""
+    _check(library().rib_set_bwd_kernel(int(which)), "rib_set_bwd_kernel")
+
+
+def rib_bwd_kernel_for(window: int) -> int:
+    """The backward form a call with this window size would use."""
+    return int(library().rib_bwd_kernel_for(int(window)))
 
 
 def rib_debug_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:

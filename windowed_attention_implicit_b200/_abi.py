@@ -16,6 +16,9 @@ RIB_ERR_CUDA = -5
 RIB_ERR_TIMEOUT = -6
 RIB_ERR_ALIGN = -7
 RIB_NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
+RIB_BWD_AUTO = 0
+RIB_BWD_PER_ITEM = 1
+RIB_BWD_PERSISTENT = 2
 
 _p = ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
@@ -54,6 +57,8 @@ _SIGS = {
                                         ctypes.c_float, _p, _p, _p]),
     "rib_window_attn_fwd_cla": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
                                      ctypes.c_float, _p, _p, _p, _p, _p]),
+    "rib_window_attn_fwd_tf32": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _i,
+                                      ctypes.c_float, _p, _p, _p]),
     "rib_cla_gate": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]),
     "rib_cla_bwd_workspace": (ctypes.c_size_t, [_i, _i, _i, _i]),
     "rib_cla_bwd": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
@@ -75,6 +80,8 @@ _SIGS = {
     "rib_status_string": (ctypes.c_char_p, [_i]),
     "rib_last_status": (_i, [ctypes.POINTER(_i)]),
     "rib_set_wait_limit_ns": (_i, [ctypes.c_ulonglong]),
+    "rib_set_bwd_kernel": (_i, [_i]),
+    "rib_bwd_kernel_for": (_i, [_i]),
     "rib_debug_wait_timeout": (_i, [ctypes.c_ulonglong, _p]),
     "rib_debug_exp2": (_i, [_p, _p, _i, _p]),
     "rib_version": (ctypes.c_char_p, []),

@@ -100,6 +100,7 @@ struct BwdParams {
   __nv_bfloat16* dqkv;
   float* dq_acc;     // [units][n_tiles][48][128]  (channel-major per tile)
   float* dkp_part;   // [units][n_tiles][128][16]
+  int n_items;       // persistent form only: work items (unit, key tile), units * n_tiles
   uint64_t wait_limit_ns;
 };
 

@@ -471,7 +471,11 @@ __device__ __forceinline__ void reg_fence_x32(uint32_t (&r)[32]) {
 // Shared-memory matrix descriptor of tcgen05.mma (sm_100 format):
 // start address, leading / stride byte offsets (all >> 4), version 1 at
 // bits 46-47, base offset 0, layout type at bits 61-63.
-enum : uint32_t { kLayoutNone = 0, kLayoutSW128 = 2, kLayoutSW64 = 4, kLayoutSW32 = 6 };
+// kLayoutSW128B32: 128-byte rows whose 32-byte granules are XORed with the
+// row index mod 4 (a 4-row atom); the layout an MN-major tf32 operand needs.
+enum : uint32_t {
+  kLayoutNone = 0, kLayoutSW128B32 = 1, kLayoutSW128 = 2, kLayoutSW64 = 4, kLayoutSW32 = 6
+};
 
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_bytes,
                                                uint32_t sbo_bytes, uint32_t layout) {
@@ -492,6 +496,52 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, 
          | (1u << 10)                              // B format: bf16
          | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of tcgen05.mma kind::tf32: fp32 operands in shared
+// or tensor memory read as tf32 (10 explicit mantissa bits), fp32 D.
+__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                                 // D format: f32
+         | (2u << 7)                               // A format: tf32
+         | (2u << 10)                              // B format: tf32
+         | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::tf32 (K = 8 per MMA),
+// issued by one elected lane of a converged warp.
+__device__ __forceinline__ void umma_tf32_ss_elect(uint32_t d_tmem, uint64_t a_desc,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::tf32 (A: 8 fp32 columns per MMA),
+// issued by one elected lane of a converged warp.
+__device__ __forceinline__ void umma_tf32_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// fp32 -> tf32 (round to nearest, ties away from zero), kept in an fp32
+// register with the 13 low mantissa bits zero.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -21,7 +21,9 @@
 #include "pos_tokens.cuh"
 #include "window_copy.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_tf32.cuh"
 #include "attn_bwd.cuh"
+#include "attn_bwd_persist.cuh"
 #include "cla.cuh"
 #include "cla_bwd.cuh"
 
@@ -31,6 +33,8 @@ namespace {
 // ---------------------------------------------------------------- helpers
 
 unsigned long long g_wait_limit_ns = 1000000000ull;  // 1 s
+// Backward kernel form: RIB_BWD_AUTO picks by window size (rib_bwd_kernel_for)
+std::atomic<int> g_bwd_kernel{RIB_BWD_AUTO};
 constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -104,6 +108,28 @@ int map_pos_padded(CUtensorMap* m, const void* base, int heads, int M) {
                   CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// fp32 qkv-like tensor [B][H][W][slots][32]: 128-byte rows, 128B swizzle
+// (the tf32 forward's K-major and MN-major operand tiles).
+// sw: CU_TENSOR_MAP_SWIZZLE_128B for K-major operand tiles,
+// CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B for the MN-major V tile.
+int map_tokens_f32(CUtensorMap* m, const void* base, int B, int H, int W, int slots,
+                   CUtensorMapSwizzle sw) {
+  const uint64_t dims[5] = {32, (uint64_t)slots, (uint64_t)W, (uint64_t)H, (uint64_t)B};
+  const uint64_t row = 128;
+  const uint64_t strides[4] = {row, row * slots, row * slots * W, row * slots * W * H};
+  const uint32_t box[5] = {32, 1, 8, 8, 1};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, base, dims, strides, box, sw);
+}
+
+// fp32 positional tokens [heads][M][M][16]: 64-byte rows, 64B swizzle.
+int map_pos_f32(CUtensorMap* m, const void* base, int heads, int M) {
+  const uint64_t dims[4] = {16, (uint64_t)M, (uint64_t)M, (uint64_t)heads};
+  const uint64_t strides[3] = {64, 64ull * M, 64ull * M * M};
+  const uint32_t box[4] = {16, 8, 8, 1};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 // per-pixel fp32 [B][heads][H][W], 8x8-pixel boxes.
 int map_pixel_f32(CUtensorMap* m, const void* base, int B, int heads, int H, int W) {
   const uint64_t dims[4] = {(uint64_t)W, (uint64_t)H, (uint64_t)heads, (uint64_t)B};
@@ -116,14 +142,15 @@ int map_pixel_f32(CUtensorMap* m, const void* base, int B, int heads, int H, int
 // ---------------------------------------------------------------- tracing
 enum KernelId {
   K_POS, K_FWD, K_BWD_PRE, K_BWD, K_DQ_FIN, K_POSGRAD, K_MLP_PART, K_MLP_RED, K_COPY, K_DEBUG,
-  K_CLA, K_CLA_DZ, K_CLA_DWPW, K_CLA_DX, K_CLA_RED, K_COUNT
+  K_CLA, K_CLA_DZ, K_CLA_DWPW, K_CLA_DX, K_CLA_RED, K_BWD_PERSIST, K_FWD_TF32, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "pos_tokens_kernel",   "attn_fwd_kernel",        "bwd_preprocess_kernel",
     "attn_bwd_kernel",     "dq_finalize_kernel",     "posgrad_reduce_kernel",
     "mlp_bwd_partial_kernel", "mlp_bwd_reduce_kernel", "window_copy_kernel",
     "debug_wait_kernel",   "cla_gate_kernel",        "cla_bwd_dz_kernel",
-    "cla_bwd_dwpw_kernel", "cla_bwd_dx_kernel",      "cla_bwd_reduce_kernel"};
+    "cla_bwd_dwpw_kernel", "cla_bwd_dx_kernel",      "cla_bwd_reduce_kernel",
+    "attn_bwd_persistent_kernel", "attn_fwd_tf32_kernel"};
 
 struct TraceRec {
   int id;
@@ -422,6 +449,23 @@ int rib_last_status(int* site) {
   return h[0];
 }
 
+int rib_set_bwd_kernel(int which) {
+  if (which != RIB_BWD_AUTO && which != RIB_BWD_PER_ITEM && which != RIB_BWD_PERSISTENT)
+    return RIB_ERR_ARG;
+  g_bwd_kernel.store(which);
+  return RIB_OK;
+}
+
+int rib_bwd_kernel_for(int window) {
+  const int which = g_bwd_kernel.load();
+  if (which != RIB_BWD_AUTO) return which;
+  // Up to 64 x 64 windows (32 query tiles per key tile) the per-CTA set-up
+  // and the pipeline's ramp and drain weigh on few tiles, and the persistent
+  // form, which overlaps them with the neighbouring item, is faster; at
+  // 96 x 96 windows the per-item kernel is.
+  return window <= 64 ? RIB_BWD_PERSISTENT : RIB_BWD_PER_ITEM;
+}
+
 int rib_set_wait_limit_ns(unsigned long long limit_ns) {
   g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs;
   return RIB_OK;
@@ -646,6 +690,45 @@ int rib_window_attn_fwd_cla(const void* qkv, int B, int H, int W, int heads, int
   if (!gate || !out_gated) return RIB_ERR_ARG;
   return attn_fwd_launch(qkv, B, H, W, heads, head_dim, window, shift, qp_bf16, kp_bf16, rank,
                          scale, out, lse, gate, out_gated, 0, stream);
+}
+
+int rib_window_attn_fwd_tf32(const float* qkv, int B, int H, int W, int heads, int head_dim,
+                             int window, int shift, const float* qp, const float* kp, int rank,
+                             float scale, float* out, float* lse, void* stream) {
+  AttnGeom g;
+  int rc = check_attn(B, H, W, heads, head_dim, window, shift, rank, &g);
+  if (rc) return rc;
+  if (B == 0) return RIB_OK;
+  if (!qkv || !out || !lse || (rank > 0 && (!qp || !kp))) return RIB_ERR_ARG;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(lse) ||
+      (rank > 0 && (!aligned16(qp) || !aligned16(kp))))
+    return RIB_ERR_ALIGN;
+  if (!std::isfinite(scale)) return RIB_ERR_ARG;
+  const float tau = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(head_dim + rank));
+  CUtensorMap tq, tv, tqp, tkp;
+  if ((rc = map_tokens_f32(&tq, qkv, B, H, W, 3 * heads, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  if ((rc = map_tokens_f32(&tv, qkv, B, H, W, 3 * heads, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)))
+    return rc;
+  if (rank > 0) {
+    if ((rc = map_pos_f32(&tqp, qp, heads, window))) return rc;
+    if ((rc = map_pos_f32(&tkp, kp, heads, window))) return rc;
+  } else {
+    tqp = tq;
+    tkp = tq;
+  }
+  TfParams p{};
+  p.B = B; p.H = H; p.W = W; p.heads = heads; p.M = window; p.s = shift; p.rank = rank;
+  p.nWx = g.nWx; p.nW = g.nW; p.tiles_x = g.tiles_x; p.n_tiles = g.n_tiles;
+  p.scale_log2 = tau * 1.4426950408889634f;
+  p.out = out;
+  p.lse = lse;
+  p.wait_limit_ns = g_wait_limit_ns;
+  if ((rc = set_smem(attn_fwd_tf32_kernel, kTfSmemBytes))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  TraceScope ts(K_FWD_TF32, st);
+  attn_fwd_tf32_kernel<<<dim3(g.n_tiles, g.units), kTfThreads, kTfSmemBytes, st>>>(tq, tv, tqp,
+                                                                                   tkp, p);
+  return launch_status();
 }
 
 int rib_cla_gate(const void* x, int B, int H, int W, int C, const float* w_dw, const float* b_dw,
@@ -899,17 +982,30 @@ static int attn_bwd_launch(const void* qkv, const void* out, const void* dout,
   p.dqkv = a.dqkv;
   p.dq_acc = a.dq_acc;
   p.dkp_part = reinterpret_cast<float*>(wsb + ws.dkp_part);
+  p.n_items = g.units * g.n_tiles;
   p.wait_limit_ns = g_wait_limit_ns;
-  auto* kern = p.region_mask ? attn_bwd_kernel<true> : attn_bwd_kernel<false>;
-  if ((rc = set_smem(kern, kBwdSmemBytes))) return rc;
-  {
-    // The kernel moves registers between warpgroups with setmaxnreg; that is
-    // only safe if the compiled launch budget is the one the split assumes.
-    static std::atomic<int> launch_regs[2] = {{-1}, {-1}};
-    if ((rc = check_launch_regs(reinterpret_cast<const void*>(kern), launch_regs[p.region_mask ? 1 : 0], kBwdLaunchRegs)))
+  // Both forms move registers between warpgroups with setmaxnreg, which is
+  // only safe if the compiled launch budget is the one the split assumes.
+  static std::atomic<int> launch_regs[4] = {{-1}, {-1}, {-1}, {-1}};
+  if (rib_bwd_kernel_for(window) == RIB_BWD_PERSISTENT) {
+    auto* kern = p.region_mask ? pbwd::attn_bwd_persistent_kernel<true>
+                               : pbwd::attn_bwd_persistent_kernel<false>;
+    if ((rc = set_smem(kern, pbwd::kPBwdSmemBytes))) return rc;
+    if ((rc = check_launch_regs(reinterpret_cast<const void*>(kern),
+                                launch_regs[2 + (p.region_mask ? 1 : 0)], kBwdLaunchRegs)))
       return rc;
-  }
-  {
+    // one CTA per SM walks the work items (unit, key tile)
+    int sms = 0;
+    if ((rc = device_sms(&sms))) return rc;
+    TraceScope ts(K_BWD_PERSIST, st);
+    kern<<<std::min(p.n_items, sms), kBwdThreads, pbwd::kPBwdSmemBytes, st>>>(tq, tdo, tqp, tkp,
+                                                                             tl, td, p);
+  } else {
+    auto* kern = p.region_mask ? attn_bwd_kernel<true> : attn_bwd_kernel<false>;
+    if ((rc = set_smem(kern, kBwdSmemBytes))) return rc;
+    if ((rc = check_launch_regs(reinterpret_cast<const void*>(kern),
+                                launch_regs[p.region_mask ? 1 : 0], kBwdLaunchRegs)))
+      return rc;
     TraceScope ts(K_BWD, st);
     kern<<<dim3(g.n_tiles, g.units), kBwdThreads, kBwdSmemBytes, st>>>(tq, tdo, tqp, tkp, tl,
                                                                        td, p);
