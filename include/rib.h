@@ -58,6 +58,7 @@ extern "C" {
 #define RIB_ERR_CUDA        -5  /* a CUDA runtime/driver call failed */
 #define RIB_ERR_TIMEOUT     -6  /* a kernel's bounded wait ran out (status word) */
 #define RIB_ERR_ALIGN       -7  /* a device pointer is not 16-byte aligned */
+#define RIB_ERR_BOUNDS      -8  /* debug build: a guarded access fell outside its buffer */
 
 /* Position-MLP weights (device, fp32, PyTorch Linear layout weight[out][in]).
  * d_in = 4*n_freq (features [sin(w x), cos(w x), sin(w y), cos(w y)]),
@@ -405,6 +406,30 @@ int rib_bwd_kernel_for(int window);
 /* Time limit, in nanoseconds, of every bounded wait in kernels launched
  * after this call (process-wide; default 1e9 = 1 s; 0 restores it). */
 int rib_set_wait_limit_ns(unsigned long long limit_ns);
+
+/* ------------------------------------------------------------------------
+ * Debug build.  librib_debug.so is this library compiled with RIB_DEBUG: every
+ * global-memory access of its kernels that does not go through a TMA tensor
+ * map first tests its element index against the extent of its buffer, as
+ * the call's shapes define it.  A refused access is skipped (nothing out of
+ * range is read or written); the first one records RIB_ERR_BOUNDS, reported
+ * by rib_last_status with the code of the guarded site, and its index and
+ * extent, reported by rib_debug_guard_info.  Results are otherwise those of
+ * the release library, at lower speed.  It stands in for a memory checker.
+ *
+ * rib_debug_build         1 in the debug build, 0 in the release build.
+ * rib_debug_guard_info    synchronises, writes {index, extent} of the first
+ *                         refused access since the last call (zeros if none,
+ *                         and always zeros in the release build), clears it.
+ * rib_debug_guard_selftest  launches one CTA that writes element `index` of
+ *                         a 32-float shared array whose first `extent`
+ *                         elements are in bounds, through a guard; index >=
+ *                         extent must be refused and recorded.  Release
+ *                         build: RIB_ERR_UNSUPPORTED, nothing launched.
+ * ------------------------------------------------------------------------ */
+int rib_debug_build(void);
+int rib_debug_guard_info(unsigned long long* index_extent);
+int rib_debug_guard_selftest(int index, int extent, void* stream);
 
 /* Test hook for the failure path: launches one CTA that waits on an
  * mbarrier nothing will arrive on, with the given limit, using the same

@@ -33,11 +33,26 @@ def test_library_exports_every_declared_symbol():
         assert name in _abi._SIGS, f"{name} has no ctypes signature"
 
 
+def test_debug_library_exports_the_same_symbols_and_says_so():
+    """librib_debug.so (the bounds-checked build) offers every declared entry
+    point too; each library reports which build it is (no GPU call)."""
+    import ctypes
+    from windowed_attention_implicit_b200 import build as B
+    if not os.path.exists(B.LIB_DEBUG):
+        B.build(debug=True)
+    dbg = ctypes.CDLL(B.LIB_DEBUG)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    assert dbg.rib_debug_build() == 1
+    assert R.library().rib_debug_build() == 0
+
+
 def test_status_strings():
     lib = R.library()
     for code, name in ((0, "RIB_OK"), (-1, "RIB_ERR_ARG"), (-2, "RIB_ERR_SHAPE"),
                        (-3, "RIB_ERR_UNSUPPORTED"), (-4, "RIB_ERR_WORKSPACE"),
-                       (-5, "RIB_ERR_CUDA"), (-6, "RIB_ERR_TIMEOUT"), (-7, "RIB_ERR_ALIGN")):
+                       (-5, "RIB_ERR_CUDA"), (-6, "RIB_ERR_TIMEOUT"), (-7, "RIB_ERR_ALIGN"),
+                       (-8, "RIB_ERR_BOUNDS")):
         assert lib.rib_status_string(code).decode() == name
     assert R.rib_version().startswith("rib-b200")
 

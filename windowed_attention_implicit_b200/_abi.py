@@ -5,7 +5,10 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librib.so")
+# RIB_DEBUG_LIBRARY=1 selects the bounds-checked debug build of the same
+# library (librib_debug.so); otherwise the release build is loaded.
+LIB_PATH = os.path.join(_HERE, "librib_debug.so" if os.environ.get("RIB_DEBUG_LIBRARY") == "1"
+                        else "librib.so")
 
 RIB_OK = 0
 RIB_ERR_ARG = -1
@@ -15,6 +18,7 @@ RIB_ERR_WORKSPACE = -4
 RIB_ERR_CUDA = -5
 RIB_ERR_TIMEOUT = -6
 RIB_ERR_ALIGN = -7
+RIB_ERR_BOUNDS = -8
 RIB_NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
 RIB_BWD_AUTO = 0
 RIB_BWD_PER_ITEM = 1
@@ -84,6 +88,9 @@ _SIGS = {
     "rib_bwd_kernel_for": (_i, [_i]),
     "rib_debug_wait_timeout": (_i, [ctypes.c_ulonglong, _p]),
     "rib_debug_exp2": (_i, [_p, _p, _i, _p]),
+    "rib_debug_build": (_i, []),
+    "rib_debug_guard_info": (_i, [ctypes.POINTER(ctypes.c_ulonglong)]),
+    "rib_debug_guard_selftest": (_i, [_i, _i, _p]),
     "rib_version": (ctypes.c_char_p, []),
     "rib_trace_enable": (_i, [_i]),
     "rib_trace_collect": (_i, [ctypes.c_void_p, _i, ctypes.POINTER(_i)]),
@@ -99,8 +106,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         return _lib
     if not os.path.exists(path):
         raise ImportError(
-            f"librib.so not found at {path}; build it with "
-            "`python -m windowed_attention_implicit_b200.build`")
+            f"{os.path.basename(path)} not found at {path}; build it with "
+            "`python -m windowed_attention_implicit_b200.build`"
+            f"{' --debug' if path.endswith('_debug.so') else ''}")
     lib = ctypes.CDLL(path)
     for name, (res, args) in _SIGS.items():
         fn = getattr(lib, name)

@@ -104,6 +104,12 @@ struct BwdParams {
   uint64_t wait_limit_ns;
 };
 
+// Units (batch entry, window, head) of a call: the extent of the per-unit
+// buffers, for the debug build's guards.
+__device__ __forceinline__ size_t bwd_units(const BwdParams& p) {
+  return static_cast<size_t>(p.B) * p.nW * p.heads;
+}
+
 struct __align__(1024) BwdSmem {
   uint8_t kc[8192];                // key tile, content, [128 rows][64 B], 64B swizzle
   uint8_t kp[8192];                // key tile, positional zero-padded to 32 ch (kc + 8 KB)
@@ -340,8 +346,9 @@ __device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdP
     named_bar_sync(kDrainBar, 128);
     if (!all_ok) break;
     if (leader) {
-      bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(unit) * p.n_tiles + it) * 48 * 128,
-                          sm.dq_stage, tile_bytes);
+      const size_t dq0 = (static_cast<size_t>(unit) * p.n_tiles + it) * 48 * 128;
+      if (rib_guard(dq0 + 48 * 128 - 1, bwd_units(p) * p.n_tiles * 48 * 128, G_BWD_DQ_ACC))
+        bulk_reduce_add_f32(p.dq_acc + dq0, sm.dq_stage, tile_bytes);
       tma_store_commit();
     }
   }
@@ -484,6 +491,7 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
   const int x = wrap_once(u.wx * p.M + jl + p.s, p.W);
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
   __nv_bfloat16* base = p.dqkv + pix * 3 * p.heads * 32;
+  const size_t n_dqkv = static_cast<size_t>(p.B) * p.H * p.W * 3 * p.heads * 32;
   uint32_t r[32];
   if (g == 0) {  // dV
     tmem_ld_x32(tmem + lane_off + kBColDV, r);
@@ -492,7 +500,9 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     uint4* dst = reinterpret_cast<uint4*>(base + (2 * p.heads + u.head) * 32);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(
+      if (rib_guard(pix * 3 * p.heads * 32 + (2 * p.heads + u.head) * 32 + 8 * q + 7, n_dqkv,
+                    G_BWD_DQKV))
+        dst[q] = make_uint4(
           pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1])),
           pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
           pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
@@ -502,12 +512,13 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
       tmem_ld_x16(tmem + lane_off + kBColDK + 32, r16);
       tmem_wait_ld();
       reg_fence_x16(r16);
-      float4* dk = reinterpret_cast<float4*>(
-          p.dkp_part + ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + key) * 16);
+      const size_t kp0 = ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + key) * 16;
+      float4* dk = reinterpret_cast<float4*>(p.dkp_part + kp0);
       const float t = p.scale;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        dk[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
+        if (rib_guard(kp0 + 4 * q + 3, bwd_units(p) * p.n_tiles * 128 * 16, G_BWD_DKP_PART))
+          dk[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
                             __uint_as_float(r16[4 * q + 2]) * t,
                             __uint_as_float(r16[4 * q + 3]) * t);
     }
@@ -519,7 +530,9 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     uint4* dst = reinterpret_cast<uint4*>(base + (p.heads + u.head) * 32);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(
+      if (rib_guard(pix * 3 * p.heads * 32 + (p.heads + u.head) * 32 + 8 * q + 7, n_dqkv,
+                    G_BWD_DQKV))
+        dst[q] = make_uint4(
           pack_bf16x2(__uint_as_float(r[8 * q + 0]) * t, __uint_as_float(r[8 * q + 1]) * t),
           pack_bf16x2(__uint_as_float(r[8 * q + 2]) * t, __uint_as_float(r[8 * q + 3]) * t),
           pack_bf16x2(__uint_as_float(r[8 * q + 4]) * t, __uint_as_float(r[8 * q + 5]) * t),
@@ -635,6 +648,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdAuxParams 
     const uint4* o4 = reinterpret_cast<const uint4*>(p.out + row);
     const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + row);
     float acc = 0.f;
+    if (!rib_guard(row + 31, n * 32, G_BWD_PRE_IN)) continue;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint4 a = o4[q], c = g4[q];
@@ -676,6 +690,10 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(const BwdAuxParams p) 
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
   uint4* dst = reinterpret_cast<uint4*>(p.dqkv + (pix * 3 * p.heads + u.head) * 32);
   const float t = p.scale;
+  if (!rib_guard((ut * 48 + 31) * 128 + row, p.dq_acc_floats, G_DQ_FIN_IN) ||
+      !rib_guard((pix * 3 * p.heads + u.head) * 32 + 31,
+                 static_cast<size_t>(p.B) * p.H * p.W * 3 * p.heads * 32, G_DQ_FIN_OUT))
+    return;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const float* c = src + 8 * q * 128;
@@ -702,6 +720,9 @@ __global__ void __launch_bounds__(256) posgrad_reduce_kernel(const BwdAuxParams 
   for (int bw = 0; bw < bw_units; ++bw) {
     const size_t unit = static_cast<size_t>(bw) * p.heads + h;
     const size_t ut = unit * p.n_tiles + tile;
+    if (!rib_guard((ut * 48 + 32 + r) * 128 + row, p.dq_acc_floats, G_POSGRAD_IN) ||
+        !rib_guard((ut * 128 + row) * 16 + r, p.dq_acc_floats / 48 * 16, G_POSGRAD_IN))
+      break;
     aq += p.dq_acc[(ut * 48 + 32 + r) * 128 + row];
     ak += p.dkp_part[(ut * 128 + row) * 16 + r];
   }

@@ -320,8 +320,10 @@ __device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdP
       named_bar_sync(kDrainBar, 128);
       if (!all_ok) break;
       if (leader) {
-        bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(unit) * p.n_tiles + it) * 48 * 128,
-                            sm.dq_stage, tile_bytes);
+        if (rib_guard((static_cast<size_t>(unit) * p.n_tiles + it + 1) * 48 * 128 - 1,
+                      bwd_units(p) * p.n_tiles * 48 * 128, G_BWD_DQ_ACC))
+          bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(unit) * p.n_tiles + it) * 48 * 128,
+                              sm.dq_stage, tile_bytes);
         tma_store_commit();
       }
     }
@@ -354,7 +356,10 @@ __device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdP
         uint4* dst = reinterpret_cast<uint4*>(base + ((a == 0 ? 2 : 1) * p.heads + u.head) * 32);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(
+          if (rib_guard(pix * 3 * p.heads * 32 + ((a == 0 ? 2 : 1) * p.heads + u.head) * 32 +
+                            8 * q + 7,
+                        static_cast<size_t>(p.B) * p.H * p.W * 3 * p.heads * 32, G_BWD_DQKV))
+            dst[q] = make_uint4(
               pack_bf16x2(__uint_as_float(r32[8 * q + 0]) * f, __uint_as_float(r32[8 * q + 1]) * f),
               pack_bf16x2(__uint_as_float(r32[8 * q + 2]) * f, __uint_as_float(r32[8 * q + 3]) * f),
               pack_bf16x2(__uint_as_float(r32[8 * q + 4]) * f, __uint_as_float(r32[8 * q + 5]) * f),
@@ -368,7 +373,9 @@ __device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdP
             p.dkp_part + ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + row) * 16);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          dkp[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
+          if (rib_guard(((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + row) * 16 + 4 * q + 3,
+                        bwd_units(p) * p.n_tiles * 128 * 16, G_BWD_DKP_PART))
+            dkp[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
                                __uint_as_float(r16[4 * q + 2]) * t,
                                __uint_as_float(r16[4 * q + 3]) * t);
       }

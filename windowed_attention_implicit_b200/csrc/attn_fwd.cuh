@@ -485,10 +485,15 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
   const int y = wrap_once(u.wy * p.M + i + p.s, p.H);
   const int x = wrap_once(u.wx * p.M + jl + p.s, p.W);
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
-  uint4* dst = reinterpret_cast<uint4*>(p.out + (pix * p.heads + u.head) * 32);
+  const size_t row0 = (pix * p.heads + u.head) * 32;   // first of the row's 32 channels
+  const size_t n_out = static_cast<size_t>(p.B) * p.H * p.W * p.heads * 32;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + row0);
+  if (rib_guard(row0 + 31, n_out, G_FWD_OUT)) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-  if (p.gate != nullptr) {
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  }
+  if (p.gate != nullptr && rib_guard(row0 + 31, n_out, G_FWD_GATE)) {
     // convolutional local attention: O' = O * G at the same pixel and
     // channels (German summary, Methodik §B); O itself is kept for the
     // backward.  The product is formed from the fp32 O, then rounded.
@@ -509,8 +514,9 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
       dg[q] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
     }
   }
-  p.lse[(static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x] =
-      (m_run + log2f(l_run)) * 0.69314718055994531f;
+  const size_t li_ = (static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x;
+  if (rib_guard(li_, static_cast<size_t>(p.B) * p.heads * p.H * p.W, G_FWD_LSE))
+    p.lse[li_] = (m_run + log2f(l_run)) * 0.69314718055994531f;
   return true;
 }
 

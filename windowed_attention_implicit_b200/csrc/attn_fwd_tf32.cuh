@@ -229,13 +229,18 @@ __device__ __forceinline__ void tf_softmax(TfSmem& sm, uint32_t tmem, const TfPa
   const int y = wrap_once(u.wy * p.M + i + p.s, p.H);
   const int x = wrap_once(u.wx * p.M + jl + p.s, p.W);
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
-  float4* dst = reinterpret_cast<float4*>(p.out + (pix * p.heads + u.head) * 32);
+  const size_t row0 = (pix * p.heads + u.head) * 32;
+  float4* dst = reinterpret_cast<float4*>(p.out + row0);
+  if (rib_guard(row0 + 31, static_cast<size_t>(p.B) * p.H * p.W * p.heads * 32, G_TF32_OUT)) {
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
-    dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
-                         __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv);
-  p.lse[(static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x] =
-      (m_run + log2f(l_run)) * 0.69314718055994531f;
+    for (int q = 0; q < 8; ++q)
+      dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                           __uint_as_float(o[4 * q + 2]) * inv,
+                           __uint_as_float(o[4 * q + 3]) * inv);
+  }
+  const size_t li_ = (static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x;
+  if (rib_guard(li_, static_cast<size_t>(p.B) * p.heads * p.H * p.W, G_TF32_LSE))
+    p.lse[li_] = (m_run + log2f(l_run)) * 0.69314718055994531f;
 }
 
 // grid (n_tiles, units), block kTfThreads, dynamic smem kTfSmemBytes.

@@ -277,9 +277,13 @@ __global__ void __launch_bounds__(kClaThreads, 1)
                               fmaf(0.5f, tanh_approx(0.5f * z1), 0.5f));
         }
         uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+        const size_t g0 = ((static_cast<size_t>(b) * p.H + i0 + (r >> 4)) * p.W + j0 + (r & 15)) *
+                              C + c0;
+        if (rib_guard(g0 + 31, static_cast<size_t>(p.B) * p.H * p.W * C, G_CLA_GATE)) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          d4[e] = make_uint4(gk[4 * e], gk[4 * e + 1], gk[4 * e + 2], gk[4 * e + 3]);
+          for (int e = 0; e < 4; ++e)
+            d4[e] = make_uint4(gk[4 * e], gk[4 * e + 1], gk[4 * e + 2], gk[4 * e + 3]);
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -62,6 +62,11 @@ __device__ __forceinline__ size_t cla_pix(const ClaBwdParams& p, int b, int i, i
   return (static_cast<size_t>(b) * p.H + i) * p.W + j;
 }
 
+// Elements of one [B][H][W][C] tensor: the extent the debug build's guards use.
+__device__ __forceinline__ size_t cla_elems(const ClaBwdParams& p) {
+  return static_cast<size_t>(p.B) * p.H * p.W * p.C;
+}
+
 // Element-wise part of the dz kernel: thread = (pixel slot, channel octet),
 // kDzBatch pixels' loads in flight at once.
 constexpr int kDzBatch = 2;
@@ -130,6 +135,10 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
         const int r = r0 + e * slots;
         if (r < 128) {
           const size_t off = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
+          if (!rib_guard(off + 7, cla_elems(p), G_CLA_IN)) {
+            dgv[e] = ov[e] = gv[e] = make_uint4(0, 0, 0, 0);
+            continue;
+          }
           dgv[e] = ldg_nc_v4(p.dout_g + off);
           ov[e] = ldg_nc_v4(p.out + off);
           gv[e] = ldg_nc_v4(p.gate + off);
@@ -156,8 +165,10 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
           acc[2 * h + 1] += z1;
         }
         const uint4 z4 = make_uint4(zv[0], zv[1], zv[2], zv[3]);
-        *reinterpret_cast<uint4*>(p.dout + off) = make_uint4(dov[0], dov[1], dov[2], dov[3]);
-        *reinterpret_cast<uint4*>(p.dz + off) = z4;
+        if (rib_guard(off + 7, cla_elems(p), G_CLA_OUT)) {
+          *reinterpret_cast<uint4*>(p.dout + off) = make_uint4(dov[0], dov[1], dov[2], dov[3]);
+          *reinterpret_cast<uint4*>(p.dz + off) = z4;
+        }
         *reinterpret_cast<uint4*>(sA + cla_kmajor_offset(r, 8 * k, C)) = z4;
       }
     }
@@ -187,6 +198,9 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
         tmem_wait_ld();
         reg_fence_x32(v);
         uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+        if (!rib_guard(cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + c0 + 31, cla_elems(p),
+                       G_CLA_OUT))
+          continue;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           d4[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
@@ -211,7 +225,9 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     float s = 0.f;
     for (int w = 0; w < slots; ++w) s += red[w * C + c];
-    p.part_dbpw[static_cast<size_t>(blockIdx.x) * C + c] = s;
+    if (rib_guard(static_cast<size_t>(blockIdx.x) * C + c, static_cast<size_t>(p.grid) * C,
+                  G_CLA_PART))
+      p.part_dbpw[static_cast<size_t>(blockIdx.x) * C + c] = s;
   }
   tc_fence_before();
   __syncthreads();
@@ -311,8 +327,9 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1)
       const int ko = it & 7, q = it >> 5, ch = q % chunks, k = ch * 8 + ko;
       const int r = (q / chunks) * 4 + ((it >> 3) & 3);
       if (k >= octets) continue;
-      const uint4 zv =
-          ldg_nc_v4(p.dz + cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k);
+      const size_t zoff = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
+      const uint4 zv = rib_guard(zoff + 7, cla_elems(p), G_CLA_IN) ? ldg_nc_v4(p.dz + zoff)
+                                                                   : make_uint4(0, 0, 0, 0);
       *reinterpret_cast<uint4*>(sA + cla_mnmajor_offset(r, 8 * k)) = zv;
     }
     ok = mbar_wait(halo_bar, halo_seen & 1, abort_flag, p.wait_limit_ns, SITE_CLA);
@@ -389,18 +406,20 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1)
     const uint32_t taddr = tmem + half * 256 + (static_cast<uint32_t>(q * 32) << 16);
     if (half == 0 || two) {
       float* dst = p.part_dwpw + (static_cast<size_t>(blockIdx.x) * C + o) * C;
-      for (int c0 = 0; c0 < C; c0 += 32) {
+      const bool in = o >= C || rib_guard((static_cast<size_t>(blockIdx.x) * C + o) * C + C - 1,
+                                          static_cast<size_t>(p.grid) * C * C, G_CLA_PART);
+      for (int c0 = 0; c0 < C; c0 += 32) {   // every lane: the TMEM loads are collective
         uint32_t v[32];
         tmem_ld_x32(taddr + c0, v);
         tmem_wait_ld();
         reg_fence_x32(v);
-        if (o < C && n_done > 0) {
+        if (o < C && n_done > 0 && in) {
           float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-        } else if (o < C) {
+        } else if (o < C && in) {
           for (int e = 0; e < 32; ++e) dst[c0 + e] = 0.f;
         }
       }
@@ -519,8 +538,9 @@ __global__ void __launch_bounds__(kClaDxThreads, 2)
               dx0 = fmaf(w0[tp], dw[2 - u][2 - v].x, dx0);
               dx1 = fmaf(w1[tp], dw[2 - u][2 - v].y, dx1);
             }
-          *reinterpret_cast<uint32_t*>(p.dx + cla_pix(p, b, i0 + ii, j0 + jc) * C + c) =
-              pack_bf16x2(dx0, dx1);
+          if (rib_guard(cla_pix(p, b, i0 + ii, j0 + jc) * C + c + 1, cla_elems(p), G_CLA_OUT))
+            *reinterpret_cast<uint32_t*>(p.dx + cla_pix(p, b, i0 + ii, j0 + jc) * C + c) =
+                pack_bf16x2(dx0, dx1);
           if (ii < 7) {
 #pragma unroll
             for (int v = 0; v < 3; ++v) {
@@ -554,7 +574,9 @@ __global__ void __launch_bounds__(kClaDxThreads, 2)
       if (g * 64 + cc >= C) continue;
       float sacc = 0.f;
       for (int w = 0; w < kClaDxThreads / 32; ++w) sacc += red[(w * 10 + tp) * 64 + cc];
-      p.part_dw[(static_cast<size_t>(blockIdx.x) * 10 + tp) * C + g * 64 + cc] = sacc;
+      if (rib_guard((static_cast<size_t>(blockIdx.x) * 10 + tp) * C + g * 64 + cc,
+                    static_cast<size_t>(p.grid_dx) * 10 * C, G_CLA_PART))
+        p.part_dw[(static_cast<size_t>(blockIdx.x) * 10 + tp) * C + g * 64 + cc] = sacc;
     }
     __syncthreads();   // red is read before the next group's first halo lands there
   }

@@ -130,6 +130,10 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   const float* b1 = p.b1[side];
   const float* gr = g + t * ldg;
   for (int jh = q; jh < p.hid; jh += nq) {
+    // (debug build) the weight row's last element lies in W1
+    if (!rib_guard(static_cast<size_t>(jh) * din + din - 1, static_cast<size_t>(p.hid) * din,
+                   G_POS_W))
+      continue;
     const float acc = dot4<true>(w1 + static_cast<size_t>(jh) * din, 1, gr, 1, din, __ldg(b1 + jh));
     h[t * ldh + jh] = gelu_erf(acc);
   }
@@ -140,9 +144,13 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_kernel(PosParams p) {
   const float* b2 = p.b2[side];
   const float* hr = h + t * ldh;
   for (int o = q; o < p.dout; o += nq) {
+    if (!rib_guard(static_cast<size_t>(o) * p.hid + p.hid - 1,
+                   static_cast<size_t>(p.dout) * p.hid, G_POS_W))
+      continue;
     const float acc = dot4<true>(w2 + static_cast<size_t>(o) * p.hid, 1, hr, 1, p.hid, __ldg(b2 + o));
     const int head = o / p.rank, r = o - head * p.rank;
     const size_t off = (static_cast<size_t>(head) * p.N + tok) * p.rank + r;
+    if (!rib_guard(off, static_cast<size_t>(p.dout) * p.N, G_POS_OUT)) continue;
     p.out32[side][off] = acc;
     if (p.out16[side]) p.out16[side][off] = __float2bfloat16_rn(acc);
   }
@@ -155,6 +163,10 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
   const int side = blockIdx.y;
   const int chunk = blockIdx.x;
   const int t0 = chunk * kPosTok;
+  // (debug build) this chunk's slice of the partials lies in the buffer
+  if (!rib_guard((static_cast<size_t>(side) * p.n_chunks + chunk + 1) * p.n_params - 1,
+                 2ull * p.n_chunks * p.n_params, G_MLP_PART))
+    return;
   const int din = 4 * p.F, hid = p.hid, dout = p.dout;
   const int ldg = pad1(din), ldh = pad1(hid), ldo = pad1(dout);
   constexpr int T = kPosTok;
@@ -167,8 +179,10 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
     const int o = idx / T, t = idx - o * T;
     const int tok = t0 + t;
     const int head = o / p.rank, r = o - head * p.rank;
-    go[t * ldo + o] =
-        tok < p.N ? p.dtok[side][(static_cast<size_t>(head) * p.N + tok) * p.rank + r] : 0.f;
+    const size_t gi = (static_cast<size_t>(head) * p.N + tok) * p.rank + r;
+    go[t * ldo + o] = tok < p.N && rib_guard(gi, static_cast<size_t>(dout) * p.N, G_MLP_IN)
+                          ? p.dtok[side][gi]
+                          : 0.f;
   }
   __syncthreads();
   const float* w1 = p.w1[side];
@@ -179,6 +193,11 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_partial_kernel(PosParams 
     const float* gr = g + t * ldg;
     const float* gor = go + t * ldo;
     for (int jh = q; jh < hid; jh += nq) {
+      if (!rib_guard(static_cast<size_t>(jh) * din + din - 1, static_cast<size_t>(hid) * din,
+                     G_POS_W) ||
+          !rib_guard(static_cast<size_t>(dout - 1) * hid + jh, static_cast<size_t>(dout) * hid,
+                     G_POS_W))
+        continue;
       const float acc = dot4<true>(w1 + static_cast<size_t>(jh) * din, 1, gr, 1, din, __ldg(b1 + jh));
       const float dh = dot4<true>(w2 + jh, hid, gor, 1, dout, 0.f);
       h[t * ldh + jh] = gelu_erf(acc);
@@ -233,6 +252,10 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_tiled_kernel(PosParams p)
   const int side = blockIdx.y;
   const int chunk = blockIdx.x;
   const int t0 = chunk * kPosTok;
+  // (debug build) this chunk's slice of the partials lies in the buffer
+  if (!rib_guard((static_cast<size_t>(side) * p.n_chunks + chunk + 1) * p.n_params - 1,
+                 2ull * p.n_chunks * p.n_params, G_MLP_PART))
+    return;
   const int din = 4 * p.F, hid = p.hid, dout = p.dout;
   const int ldg = pad4(din), ldh = pad4(hid), ldo = pad4(dout);
   constexpr int T = kPosTok;
@@ -245,8 +268,10 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_tiled_kernel(PosParams p)
     const int o = idx / T, t = idx - o * T;
     const int tok = t0 + t;
     const int head = o / p.rank, r = o - head * p.rank;
-    go[t * ldo + o] =
-        tok < p.N ? p.dtok[side][(static_cast<size_t>(head) * p.N + tok) * p.rank + r] : 0.f;
+    const size_t gi = (static_cast<size_t>(head) * p.N + tok) * p.rank + r;
+    go[t * ldo + o] = tok < p.N && rib_guard(gi, static_cast<size_t>(dout) * p.N, G_MLP_IN)
+                          ? p.dtok[side][gi]
+                          : 0.f;
   }
   __syncthreads();
   const float* w1 = p.w1[side];
@@ -256,6 +281,12 @@ __global__ void __launch_bounds__(kPosThreads) mlp_bwd_tiled_kernel(PosParams p)
   // hidden units jh0 .. jh0 + 7; then h = GELU(a), da = dh * GELU'(a)
   for (int tile = threadIdx.x; tile < 16 * (hid / 8); tile += blockDim.x) {
     const int tg = tile % 16, jh0 = (tile / 16) * 8;
+    // (debug build) the W1 rows and W2 columns this tile reads lie in W1, W2
+    if (!rib_guard(static_cast<size_t>(jh0 + 7) * din + din - 1, static_cast<size_t>(hid) * din,
+                   G_POS_W) ||
+        !rib_guard(static_cast<size_t>(dout - 1) * hid + jh0 + 7, static_cast<size_t>(dout) * hid,
+                   G_POS_W))
+      continue;
     float acc[4][8], dh[4][8];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -409,6 +440,9 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_tiled_kernel(PosParams
   // h = GELU(g W1^T + b1)
   for (int tile = threadIdx.x; tile < 16 * (hid / 8); tile += blockDim.x) {
     const int tg = tile % 16, jh0 = (tile / 16) * 8;
+    if (!rib_guard(static_cast<size_t>(jh0 + 7) * din + din - 1, static_cast<size_t>(hid) * din,
+                   G_POS_W))
+      continue;
     float acc[4][8];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -444,6 +478,9 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_tiled_kernel(PosParams
   // out = h W2^T + b2; 8 consecutive outputs lie in one head (rank % 8 == 0)
   for (int tile = threadIdx.x; tile < 16 * (dout / 8); tile += blockDim.x) {
     const int tg = tile % 16, o0 = (tile / 16) * 8;
+    if (!rib_guard(static_cast<size_t>(o0 + 7) * hid + hid - 1, static_cast<size_t>(dout) * hid,
+                   G_POS_W))
+      continue;
     float acc[4][8];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -474,6 +511,7 @@ __global__ void __launch_bounds__(kPosThreads) pos_tokens_tiled_kernel(PosParams
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = acc[j][i] + __ldg(b2 + o0 + i);
       const size_t off = (static_cast<size_t>(head) * p.N + tok) * p.rank + r0;
+      if (!rib_guard(off + 7, static_cast<size_t>(dout) * p.N, G_POS_OUT)) continue;
       float4* d32 = reinterpret_cast<float4*>(p.out32[side] + off);
       d32[0] = make_float4(v[0], v[1], v[2], v[3]);
       d32[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -496,6 +534,9 @@ __global__ void __launch_bounds__(256) mlp_bwd_reduce_kernel(PosParams p) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= p.n_params) return;
   const float* src = p.partial + static_cast<size_t>(side) * p.n_chunks * p.n_params + idx;
+  if (!rib_guard((static_cast<size_t>(side) * p.n_chunks + p.n_chunks - 1) * p.n_params + idx,
+                 2ull * p.n_chunks * p.n_params, G_MLP_PART))
+    return;
   float acc = 0.f;
   for (int c = 0; c < p.n_chunks; ++c) acc += src[static_cast<size_t>(c) * p.n_params];
   const int din = 4 * p.F;

@@ -27,6 +27,45 @@ __device__ __forceinline__ void record_error(int code, int site) {
   if (atomicCAS(&g_status[0], 0, code) == 0) atomicExch(&g_status[1], site);
 }
 
+// ---------------------------------------------------------------- debug guards
+// In the debug build (RIB_DEBUG, librib_debug.so) every global access that
+// does not go through a TMA tensor map is tested first: an element index at
+// or beyond its buffer's extent (derived from the call's shapes) records
+// RIB_ERR_BOUNDS with the site, the index and the extent, and the access is
+// skipped.  In the release build rib_guard is `true` and compiles away.
+constexpr int kErrBounds = -8;
+enum GuardSite : int {
+  G_FWD_OUT = 100, G_FWD_LSE, G_FWD_GATE, G_FWD_OUT_GATED,
+  G_TF32_OUT = 110, G_TF32_LSE,
+  G_BWD_DQKV = 120, G_BWD_DKP_PART, G_BWD_DQ_ACC, G_BWD_PRE_IN, G_BWD_PRE_OUT,
+  G_BWD_PRE_ZERO, G_DQ_FIN_IN, G_DQ_FIN_OUT, G_POSGRAD_IN, G_POSGRAD_OUT,
+  G_POS_W = 140, G_POS_OUT, G_MLP_IN, G_MLP_PART, G_MLP_OUT,
+  G_CLA_W = 150, G_CLA_GATE, G_CLA_IN, G_CLA_OUT, G_CLA_PART, G_CLA_RED,
+  G_SELFTEST = 190,
+};
+#ifdef RIB_DEBUG
+// [0] element index, [1] extent of the first access a guard refused
+__device__ unsigned long long g_guard_info[2];
+__device__ __noinline__ bool rib_guard_fail(unsigned long long idx, unsigned long long n,
+                                            int site) {
+  if (atomicCAS(&g_status[0], 0, kErrBounds) == 0) {
+    atomicExch(&g_status[1], site);
+    atomicExch(&g_guard_info[0], idx);
+    atomicExch(&g_guard_info[1], n);
+  }
+  return false;
+}
+__device__ __forceinline__ bool rib_guard(unsigned long long idx, unsigned long long n,
+                                          int site) {
+  return idx < n ? true : rib_guard_fail(idx, n, site);
+}
+#else
+__device__ __forceinline__ constexpr bool rib_guard(unsigned long long, unsigned long long,
+                                                    int) {
+  return true;
+}
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

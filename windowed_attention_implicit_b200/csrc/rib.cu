@@ -367,6 +367,22 @@ __global__ void debug_wait_kernel(unsigned long long limit_ns) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns, SITE_DEBUG);
 }
 
+#ifdef RIB_DEBUG
+// Test of the debug build's guards: element `idx` of a shared array of
+// `n` floats (n <= 32) is written only if the guard lets it through; an
+// index beyond the array is refused and recorded, and nothing is written.
+__global__ void debug_guard_kernel(int idx, int n, int* seen) {
+  __shared__ float buf[32];
+  if (threadIdx.x == 0) buf[0] = 0.f;
+  __syncthreads();
+  if (threadIdx.x == 0 && rib_guard(static_cast<unsigned long long>(idx),
+                                    static_cast<unsigned long long>(n), G_SELFTEST))
+    buf[idx & 31] = 1.f;
+  __syncthreads();
+  if (threadIdx.x == 0 && seen) *seen = buf[0] != 0.f ? 1 : 0;
+}
+#endif
+
 __global__ void debug_exp2_kernel(const float* x, float* y, int n_pairs) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n_pairs) return;
@@ -435,6 +451,7 @@ const char* rib_status_string(int s) {
     case RIB_ERR_CUDA: return "RIB_ERR_CUDA";
     case RIB_ERR_TIMEOUT: return "RIB_ERR_TIMEOUT";
     case RIB_ERR_ALIGN: return "RIB_ERR_ALIGN";
+    case RIB_ERR_BOUNDS: return "RIB_ERR_BOUNDS";
     default: return "RIB_ERR_UNKNOWN";
   }
 }
@@ -515,6 +532,41 @@ int rib_debug_exp2(const float* x, float* y, int n, void* stream) {
   const int pairs = n / 2;
   debug_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, pairs);
   return launch_status();
+}
+
+int rib_debug_build(void) {
+#ifdef RIB_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int rib_debug_guard_info(unsigned long long* index_extent) {
+  if (!index_extent) return RIB_ERR_ARG;
+  index_extent[0] = index_extent[1] = 0;
+#ifdef RIB_DEBUG
+  if (cudaDeviceSynchronize() != cudaSuccess) return RIB_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(index_extent, g_guard_info, 2 * sizeof(unsigned long long)) !=
+      cudaSuccess)
+    return RIB_ERR_CUDA;
+  const unsigned long long zero[2] = {0, 0};
+  if (cudaMemcpyToSymbol(g_guard_info, zero, sizeof(zero)) != cudaSuccess) return RIB_ERR_CUDA;
+#endif
+  return RIB_OK;
+}
+
+int rib_debug_guard_selftest(int index, int extent, void* stream) {
+#ifdef RIB_DEBUG
+  if (extent < 0 || extent > 32 || index < 0) return RIB_ERR_ARG;
+  debug_guard_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(index, extent, nullptr);
+  return launch_status();
+#else
+  (void)index;
+  (void)extent;
+  (void)stream;
+  return RIB_ERR_UNSUPPORTED;
+#endif
 }
 
 int rib_debug_wait_timeout(unsigned long long limit_ns, void* stream) {
