@@ -628,6 +628,7 @@ struct BwdAuxParams {
   __nv_bfloat16* dqkv;
   float* dqp;       // [heads][M][M][rank]
   float* dkp;
+  int pg_chunks;    // posgrad_reduce: warps sharing one group of outputs (1, 2, 4, 8, 16)
 };
 
 // One thread per (b, head, y, x): -D = -sum_c dO*O and -lse*log2(e), stored
@@ -702,32 +703,88 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(const BwdAuxParams p) 
   }
 }
 
-// One thread per (head, window-local token, r): fixed-order sums over the
-// B*nW units of that head.
-__global__ void __launch_bounds__(256) posgrad_reduce_kernel(const BwdAuxParams p) {
-  const int N = p.M * p.M;
-  const size_t n = static_cast<size_t>(p.heads) * N * p.rank;
-  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= n) return;
-  const int r = static_cast<int>(idx % p.rank);
-  const int tok = static_cast<int>((idx / p.rank) % N);
-  const int h = static_cast<int>(idx / (static_cast<size_t>(p.rank) * N));
-  const int i = tok / p.M, j = tok - i * p.M;
-  const int tile = (i >> 3) * p.tiles_x + (j >> 4);
-  const int row = ((j >> 3) & 1) * 64 + (i & 7) * 8 + (j & 7);
-  float aq = 0.f, ak = 0.f;
-  const int bw_units = p.B * p.nW;
-  for (int bw = 0; bw < bw_units; ++bw) {
-    const size_t unit = static_cast<size_t>(bw) * p.heads + h;
-    const size_t ut = unit * p.n_tiles + tile;
-    if (!rib_guard((ut * 48 + 32 + r) * 128 + row, p.dq_acc_floats, G_POSGRAD_IN) ||
-        !rib_guard((ut * 128 + row) * 16 + r, p.dq_acc_floats / 48 * 16, G_POSGRAD_IN))
-      break;
-    aq += p.dq_acc[(ut * 48 + 32 + r) * 128 + row];
-    ak += p.dkp_part[(ut * 128 + row) * 16 + r];
+// dQp[h][i][j][r] = tau * sum over the B*nW units of head h of the dQ
+// accumulator's positional channels, dKp likewise from the dKp partials
+// (one Qp/Kp set serves every window).  grid (heads*N*rank / kPgBlockOut, 2):
+// blockIdx.y 0 sums dQp, 1 sums dKp.  Outputs are taken in the layout their
+// source is read in (dQp: row fastest, matching the accumulator's
+// [unit][tile][channel][row]; dKp: rank fastest, matching the partials'
+// [unit][tile][row][rank]), 32 consecutive ones per warp, so each warp's
+// loads are 128-byte runs.  p.pg_chunks warps share a group of 32 outputs
+// and sum consecutive ranges of the units (eight accumulators taking the
+// units in turn, the remainder going to the first); the group's first warp
+// adds their sums in warp order.
+// The order is fixed: the result is deterministic.  Many units (small
+// windows) get 16 warps per group, few (large windows) one.  The grid is
+// sized to the SMs and the blocks loop over the passes.
+constexpr int kPgWarps = 16;
+constexpr int kPgBlockOut = 32 * kPgWarps;   // outputs per block pass with one warp per group
+__global__ void __launch_bounds__(32 * kPgWarps, 2) posgrad_reduce_kernel(const BwdAuxParams p) {
+  __shared__ float part[kPgWarps][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int chunks = p.pg_chunks, groups = kPgWarps / chunks, grp = w / chunks,
+            cw = w % chunks;
+  const bool kside = blockIdx.y == 1;
+  const int rank = p.rank;
+  const size_t n_out = static_cast<size_t>(p.heads) * p.n_tiles * rank * 128;
+  const size_t n_pass = (n_out + 32 * groups - 1) / (32 * groups);
+  const int total = p.B * p.nW;
+  const int per = (total + chunks - 1) / chunks;
+  const int b0 = cw * per, b1 = min(total, b0 + per);
+  const size_t unit_stride = static_cast<size_t>(p.heads) * p.n_tiles;
+  const size_t step = kside ? unit_stride * 128 * 16 : unit_stride * 48 * 128;
+  const size_t n_src = kside ? p.dq_acc_floats / 48 * 16 : p.dq_acc_floats;
+  // the blocks walk the passes (groups x 32 outputs each) in a grid-stride loop
+  for (size_t pass = blockIdx.x; pass < n_pass; pass += gridDim.x) {
+    const size_t o = (pass * groups + grp) * 32 + lane;
+    int h = 0, tile = 0, r = 0, row = 0;
+    if (o < n_out) {
+      size_t rem = o;
+      if (kside) {          // o = ((h * n_tiles + tile) * 128 + row) * rank + r
+        r = static_cast<int>(rem % rank);
+        rem /= rank;
+        row = static_cast<int>(rem % 128);
+        rem /= 128;
+      } else {              // o = ((h * n_tiles + tile) * rank + r) * 128 + row
+        row = static_cast<int>(rem % 128);
+        rem /= 128;
+        r = static_cast<int>(rem % rank);
+        rem /= rank;
+      }
+      tile = static_cast<int>(rem % p.n_tiles);
+      h = static_cast<int>(rem / p.n_tiles);
+    }
+    // element of unit (bw, h) that this output sums: base + bw * step
+    const size_t first = static_cast<size_t>(h) * p.n_tiles + tile;
+    const size_t base = kside ? (first * 128 + row) * 16 + r : (first * 48 + 32 + r) * 128 + row;
+    const float* src = (kside ? p.dkp_part : p.dq_acc) + base;
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (o < n_out && (b1 <= b0 || rib_guard(base + (b1 - 1) * step, n_src, G_POSGRAD_IN))) {
+      int bw = b0;
+      for (; bw + 7 < b1; bw += 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a[e] += src[(bw + e) * step];
+      }
+      for (; bw < b1; ++bw) a[0] += src[bw * step];
+    }
+    part[w][lane] = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+    __syncthreads();
+    if (cw == 0 && o < n_out) {
+      float sum = 0.f;
+      for (int c = 0; c < chunks; ++c) sum += part[w + c][lane];
+      int i0, j0, i, j;
+      tile_origin(tile, p.tiles_x, i0, j0);
+      tile_row_local(row, i0, j0, i, j);
+      const size_t dst = (static_cast<size_t>(h * p.M + i) * p.M + j) * rank + r;
+      if (rib_guard(dst, n_out, G_POSGRAD_OUT)) {
+        if (kside)
+          p.dkp[dst] = sum;
+        else
+          p.dqp[dst] = sum * p.scale;
+      }
+    }
+    __syncthreads();   // part is read before the next pass writes it
   }
-  p.dqp[idx] = aq * p.scale;
-  p.dkp[idx] = ak;
 }
 
 }  // namespace rib

@@ -1071,8 +1071,18 @@ static int attn_bwd_launch(const void* qkv, const void* out, const void* dout,
   }
   if (rank > 0) {
     const size_t n = (size_t)heads * g.N * rank;
+    // about 48 units or fewer per warp: 16 warps per output group for the
+    // 1152 units of 16 x 16 windows on a batch-8 192 x 192 map, one for 16
+    const int units_bw = B * g.nW;
+    a.pg_chunks = 1;
+    while (a.pg_chunks < kPgWarps && units_bw > 48 * a.pg_chunks) a.pg_chunks *= 2;
+    const size_t per_block = static_cast<size_t>(kPgBlockOut / a.pg_chunks);
+    int sms = 0;
+    if ((rc = device_sms(&sms))) return rc;
+    const size_t passes = (n + per_block - 1) / per_block;
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>(passes, 4ull * sms));
     TraceScope ts(K_POSGRAD, st);
-    posgrad_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(a);
+    posgrad_reduce_kernel<<<dim3(blocks, 2), 32 * kPgWarps, 0, st>>>(a);
     if ((rc = launch_status())) return rc;
   }
   if (do_mlp) {
