@@ -16,9 +16,10 @@
 //   cla_bwd_dz_kernel    dO, dz (to the workspace), db_pw partials, and
 //                        dy = dz W_pw on the tensor cores (tcgen05, dz tile
 //                        and W_pw^T in shared memory, accumulator in TMEM)
-//   cla_bwd_dwpw_kernel  dW_pw partials = sum over the CTA's tiles of
-//                        dz^T y, y recomputed from x; both operands MN-major
-//                        in shared memory, the C x C partial in TMEM
+//   cla_bwd_dwpw_kernel  dW_pw partials = sum over the CTA's 8 x 8-pixel
+//                        tiles of dz^T y, y recomputed from x; dz by TMA,
+//                        both operands MN-major with the 128-byte swizzle,
+//                        the C x C partial in TMEM
 //   cla_bwd_dx_kernel    dx, and dW_dw / db_dw partials (FMA pipe, two CTAs per SM,
 //                        x and dy halos staged by TMA)
 //   cla_bwd_reduce_kernel fixed-order sums of the partials
@@ -28,7 +29,7 @@
 
 namespace rib {
 
-constexpr int kClaBwdThreads = 512;   // dz and dW_pw kernels
+constexpr int kDzThreads = 384;   // dz kernel (12 warps: up to 168 registers a thread)
 constexpr int kClaDxThreads = 256;
 
 struct ClaBwdParams {
@@ -48,6 +49,7 @@ struct ClaBwdParams {
   float* part_dwpw;                // [grid][C][C]
   float* part_dw;                  // [grid_dx][10][C]  (9 taps, then the bias)
   int B, H, W, C, tiles_x, tiles_per_img, n_tiles, grid, grid_dx;
+  int tiles_x8, n_tiles8;          // 8 x 8-pixel tiles of the dW_pw kernel
   uint64_t wait_limit_ns;
 };
 
@@ -68,10 +70,12 @@ __device__ __forceinline__ size_t cla_elems(const ClaBwdParams& p) {
 }
 
 // Element-wise part of the dz kernel: thread = (pixel slot, channel octet),
-// kDzBatch pixels' loads in flight at once.
-constexpr int kDzBatch = 2;
+// kDzBatch pixels' loads in flight at once (three 16-byte loads a pixel:
+// 48 registers at 4).
+constexpr int kDzBatch = 4;
+// W_pw^T (2 C^2 bytes) | two dz tiles (256 C bytes each) | db_pw slots | barriers
 __host__ __device__ __forceinline__ size_t cla_dz_smem_bytes(int C) {
-  return 2ull * C * C + 256ull * C + 4ull * 8 * kClaBwdThreads + 64 + 1024;
+  return 2ull * C * C + 2ull * 256 * C + 4ull * 8 * kDzThreads + 64 + 1024;
 }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const __nv_bfloat16* ptr) {
@@ -79,20 +83,24 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const __nv_bfloat16* ptr) {
 }
 
 // -------------------------------------------------------------- dz and dy
-// grid p.grid, block kClaBwdThreads, dynamic smem cla_dz_smem_bytes(C).
-__global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const ClaBwdParams p) {
+// grid p.grid, block kDzThreads, dynamic smem cla_dz_smem_bytes(C).
+// The dz tile and the dy accumulator are double-buffered: tile n's MMAs run
+// while the threads do tile n + 1's element-wise part, and its dy is read
+// from TMEM after that.
+__global__ void __launch_bounds__(kDzThreads, 1) cla_bwd_dz_kernel(const ClaBwdParams p) {
   extern __shared__ uint8_t dz_raw[];
   uint8_t* base = dz_raw + ((1024u - (smem_u32(dz_raw) & 1023u)) & 1023u);
   const int C = p.C;
   uint8_t* sB = base;                                   // W_pw^T bf16 [N = c][K = o]
-  uint8_t* sA = base + 2ull * C * C;                    // dz bf16 [M = 128 pixels][K = o]
-  float* red = reinterpret_cast<float*>(sA + 256ull * C);   // [slot][C] db_pw partials
-  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 8 * kClaBwdThreads);
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
+  uint8_t* sA0 = base + 2ull * C * C;                   // dz bf16 [M = 128 pixels][K = o], x2
+  float* red = reinterpret_cast<float*>(sA0 + 2ull * 256 * C);   // [slot][C] db_pw partials
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 8 * kDzThreads);   // [2]
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -106,7 +114,7 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   }
   fence_proxy_async_smem();
   if (warp == 0) {
-    tmem_alloc(tbase, 256);
+    tmem_alloc(tbase, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -114,21 +122,53 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   tc_fence_after();
   const uint32_t tmem = *tbase;
   const uint32_t idesc = make_idesc_bf16(128, C, false, false);
-  const uint64_t adesc = make_sdesc(smem_u32(sA), 128, 16 * C, kLayoutNone);
   const uint64_t bdesc = make_sdesc(smem_u32(sB), 128, 16 * C, kLayoutNone);
   // element-wise part: thread = (pixel slot sl, channel octet k); slots
   // take pixels sl, sl + slots, ...; consecutive threads read consecutive
   // 16-byte octets of one pixel
-  const int octets = C / 8, slots = kClaBwdThreads / octets;
+  const int octets = C / 8, slots = kDzThreads / octets;
   const int sl = threadIdx.x / octets, k = threadIdx.x % octets;
   const bool act = sl < slots;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // db_pw, channels 8k..8k+7
-  bool ok = true;
-  int phase = 0;
-  for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x) {
+  const int G = gridDim.x;
+  const int my_tiles = (p.n_tiles - static_cast<int>(blockIdx.x) + G - 1) / G;
+  // dy of tile n (accumulator n % 2) to the workspace: warp w reads TMEM
+  // lanes 32 (w % 4).. (pixels), columns 32 (w / 4) + 128 i
+  auto drain_dy = [&](int n) -> bool {
+    bool ok = mbar_wait(&bar[n & 1], (n >> 1) & 1, abort_flag, p.wait_limit_ns, SITE_CLA);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (!ok) return false;
     int b, i0, j0;
-    cla_tile(p, t, b, i0, j0);
-    for (int r0 = sl; act && r0 < 128; r0 += kDzBatch * slots) {
+    cla_tile(p, static_cast<int>(blockIdx.x) + n * G, b, i0, j0);
+    const int q = warp & 3, slot = warp >> 2;
+    const int r = q * 32 + lane;
+    const size_t pix = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15));
+    __nv_bfloat16* dst = p.dy + pix * C;
+    const uint32_t taddr = tmem + (n & 1) * 256 + (static_cast<uint32_t>(q * 32) << 16);
+    for (int c0 = 32 * slot; c0 < C; c0 += 32 * (kDzThreads / 128)) {
+      uint32_t v[32];
+      tmem_ld_x32(taddr + c0, v);
+      tmem_wait_ld();
+      reg_fence_x32(v);
+      if (!rib_guard(pix * C + c0 + 31, cla_elems(p), G_CLA_OUT)) continue;
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        d4[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                           pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                           pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                           pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+    }
+    return true;
+  };
+  bool ok = true;
+  int n_mma = 0;
+  for (int n = 0; n < my_tiles; ++n) {
+    int b, i0, j0;
+    cla_tile(p, static_cast<int>(blockIdx.x) + n * G, b, i0, j0);
+    uint8_t* sA = sA0 + (n & 1) * 256ull * C;   // last read by tile n - 2's MMAs, drained
+    for (int r0 = sl; ok && act && r0 < 128; r0 += kDzBatch * slots) {
       uint4 dgv[kDzBatch], ov[kDzBatch], gv[kDzBatch];
 #pragma unroll
       for (int e = 0; e < kDzBatch; ++e) {
@@ -174,48 +214,32 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // ---- dy = dz W_pw  (M = 128 pixels, N = C, K = C)
-    if (warp == 0) {
-      for (int ks = 0; ks < C / 16; ++ks)
-        umma_ss_elect(tmem, adesc + ks * 16, bdesc + ks * 16, idesc, ks > 0 ? 1u : 0u);
-      umma_commit_elect(bar);
-    }
-    ok = mbar_wait(bar, phase, abort_flag, p.wait_limit_ns, SITE_CLA);
-    phase ^= 1;
     ok = __syncthreads_and(ok);
     tc_fence_after();
-    if (ok) {
-      // warp w reads TMEM lanes 32 (w % 4).. (pixels), columns 32 (w / 4) + 32 k (warps / 4)
-      const int q = warp & 3, slot = warp >> 2;
-      const int r = q * 32 + lane;
-      __nv_bfloat16* dst = p.dy + cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 32 * slot; c0 < C; c0 += 32 * (kClaBwdThreads / 128)) {
-        uint32_t v[32];
-        tmem_ld_x32(taddr + c0, v);
-        tmem_wait_ld();
-        reg_fence_x32(v);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-        if (!rib_guard(cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + c0 + 31, cla_elems(p),
-                       G_CLA_OUT))
-          continue;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          d4[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                             pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                             pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                             pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-      }
+    if (!ok) break;
+    // ---- dy = dz W_pw  (M = 128 pixels, N = C, K = C) into accumulator n % 2
+    if (warp == 0) {
+      const uint64_t adesc = make_sdesc(smem_u32(sA), 128, 16 * C, kLayoutNone);
+      for (int ks = 0; ks < C / 16; ++ks)
+        umma_ss_elect(tmem + (n & 1) * 256, adesc + ks * 16, bdesc + ks * 16, idesc,
+                      ks > 0 ? 1u : 0u);
+      umma_commit_elect(&bar[n & 1]);
     }
+    ++n_mma;
+    // tile n - 1's dy, whose MMAs ran during this tile's element-wise part
+    if (n >= 1) ok = drain_dy(n - 1);
     tc_fence_before();
-    __syncthreads();   // accumulator read before the next tile's MMAs
+    ok = __syncthreads_and(ok);   // accumulator (n - 1) % 2 and dz tile (n - 1) % 2 are free
     tc_fence_after();
+    if (!ok) break;
   }
-  if (!ok) {
+  if (ok && n_mma > 0) ok = drain_dy(n_mma - 1);
+  ok = __syncthreads_and(ok);
+  if (!ok && warp == 0 && n_mma > 0) {
+    // the last tile's MMAs (and every earlier one) land before the CTA exits
     volatile int no_abort = 0;
-    mbar_wait(bar, phase ^ 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
+    mbar_wait(&bar[(n_mma - 1) & 1], ((n_mma - 1) >> 1) & 1, &no_abort, 200ull * 1000ull * 1000ull,
+              SITE_CLA);
   }
   // db_pw partial of this CTA: the slots' sums, added in slot order
   // (thread (sl, k) holds channels 8k..8k+7 at red[sl * C + 8k + e] = red[8 tid + e])
@@ -233,195 +257,293 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1) cla_bwd_dz_kernel(const Cla
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 // -------------------------------------------------------------- dW_pw
-// Byte offset of element (k = pixel r, mn = channel) in an MN-major
-// no-swizzle operand of K = 128 pixels: core matrices of 8 pixels x 16 bytes
-// (8 channels), K-adjacent ones 128 bytes apart (LBO), MN-adjacent ones
-// 2048 bytes apart (SBO).
-__device__ __forceinline__ uint32_t cla_mnmajor_offset(int r, int mn) {
-  return static_cast<uint32_t>((mn >> 3) * 2048 + (r >> 3) * 128 + (r & 7) * 16 + (mn & 7) * 2);
-}
+// dW_pw = sum over pixels of dz^T y on tiles of 8 x 8 pixels (K = 64 per
+// tile).  A tile stored as 64 rows (pixels) of 128 bytes (64 channels) with
+// the 128-byte swizzle is, per 64-channel chunk, exactly one canonical
+// MN-major atom column of a K = 64 operand: dz^T (M = output channel) and
+// y^T (N = input channel) both take that form, 8 KB per chunk, chunks
+// kDwpwAtom bytes apart (LBO), 8-pixel row groups 1024 bytes apart (SBO).
+// Warp-specialised, 4 C/64 + 1 warps:
+//   y warps (4 per chunk)  recompute y = b_dw + DW3x3(x) from the tile's x
+//       halo: a thread keeps the 9 taps of one channel octet in registers
+//       and walks 4 vertically adjacent pixels of one column (6 halo rows
+//       read once each), writing y into one of two y buffers;
+//   the last warp           issues the TMA loads (dz, one 64 x 8 x 8 box per
+//       chunk with the 128-byte swizzle, into a 3-buffer ring; the x halo,
+//       one 64 x 10 x 10 box per chunk, into one of two slots) and, through
+//       an elected lane, the MMAs D_m (+)= dz^T[o in 128 m ..] y over the
+//       tile's four K = 16 steps (M blocks m = 0, 1 when C > 128), which
+//       accumulate in TMEM over all of the CTA's tiles.
+// The MMAs of tile n run while the y warps compute tile n + 1.  M block 1
+// of a C = 160 or 192 map reads one atom past dz's chunks (the next buffer
+// in shared memory): those are accumulator rows o >= C, never read.
+constexpr int kDwpwPix = 64;
+constexpr uint32_t kDwpwAtom = kDwpwPix * 128;                      // 8 KB
+constexpr uint32_t kDwpwHaloBytes = 10u * 10u * 64u * 2u;           // one chunk's halo
+constexpr uint32_t kDwpwHaloSlot = (kDwpwHaloBytes + 1023u) & ~1023u;
+constexpr int kDwpwA = 3, kDwpwB = 2, kDwpwH = 2;                   // ring depths (tiles)
+constexpr int kDwpwMaxChunks = 3;                                   // C <= 192
+constexpr int kDwpwThreads = 32 * (4 * kDwpwMaxChunks + 1);         // 416
 
-// A: dz^T [M = 256 output channels, padded][K = 128 pixels]; B: y^T [N = C][K];
-// the tile's x halo (10 x 18 pixels, one TMA box per 64 channels); weights
-// of the depth-wise convolution [9][C] and its bias [C].
-constexpr uint32_t kDwpwHaloChunk = (kClaHaloBytes + 1023u) & ~1023u;
+struct DwpwLayout {
+  uint32_t a, b, halo, bars, total;   // byte offsets from a 1024-aligned base
+};
+__host__ __device__ __forceinline__ DwpwLayout cla_dwpw_layout(int C) {
+  const uint32_t chunks = static_cast<uint32_t>((C + 63) / 64);
+  const uint32_t chunk_bytes = chunks * kDwpwAtom;
+  DwpwLayout L;
+  L.a = 0;                                    // kDwpwA dz tiles
+  L.b = L.a + kDwpwA * chunk_bytes;           // kDwpwB y tiles (after dz: the atom past the
+  L.halo = L.b + kDwpwB * chunk_bytes;        //   last dz tile stays inside the allocation)
+  L.bars = L.halo + kDwpwH * chunks * kDwpwHaloSlot;
+  L.total = L.bars + 256u;
+  return L;
+}
 __host__ __device__ __forceinline__ size_t cla_dwpw_smem_bytes(int C) {
-  return 256ull * 256 + 256ull * C + kDwpwHaloChunk * ((C + 63) / 64) + 40ull * C + 64 + 1024;
+  return static_cast<size_t>(cla_dwpw_layout(C).total) + 1024;
 }
 
-// grid p.grid, block kClaBwdThreads, dynamic smem cla_dwpw_smem_bytes(C).
-// tm_x: x [B][H][W][C] as a 4D map with boxes of 64 channels x 18 x 10.
-__global__ void __launch_bounds__(kClaBwdThreads, 1)
-    cla_bwd_dwpw_kernel(const __grid_constant__ CUtensorMap tm_x, const ClaBwdParams p) {
+// grid p.grid, block kDwpwThreads, dynamic smem cla_dwpw_smem_bytes(C); C <= 192.
+// tm_x: x [B][H][W][C], boxes of 64 channels x 10 x 10 (no swizzle);
+// tm_dz: dz [B][H][W][C], boxes of 64 channels x 8 x 8, 128-byte swizzle.
+// p.n_tiles8 tiles of 8 x 8 pixels, p.tiles_x8 per image row.
+__global__ void __launch_bounds__(kDwpwThreads, 1)
+    cla_bwd_dwpw_kernel(const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_dz, const ClaBwdParams p) {
   extern __shared__ uint8_t dw_raw[];
   uint8_t* base = dw_raw + ((1024u - (smem_u32(dw_raw) & 1023u)) & 1023u);
-  const int C = p.C, octets = C / 8;
-  uint8_t* sA = base;                          // dz^T, 64 KB
-  uint8_t* sB = base + 256 * 256;              // y^T, 256 C bytes
-  const int chunks = (C + 63) / 64;
-  uint8_t* sH = sB + 256ull * C;               // halo [chunk][10 rows][18 cols][64 ch]
-  float* sWdw = reinterpret_cast<float*>(sH + static_cast<size_t>(kDwpwHaloChunk) * chunks);
-  float* sBdw = sWdw + 9 * C;                  // ([tap][C] weights before it)
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sBdw + C);
-  uint64_t* halo_bar = bar + 1;
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
+  const int C = p.C, octets = C / 8, chunks = (C + 63) / 64;
+  const DwpwLayout L = cla_dwpw_layout(C);
+  const uint32_t chunk_bytes = static_cast<uint32_t>(chunks) * kDwpwAtom;
+  uint64_t* dz_full = reinterpret_cast<uint64_t*>(base + L.bars);   // [kDwpwA]
+  uint64_t* a_free = dz_full + kDwpwA;                               // [kDwpwA]
+  uint64_t* b_free = a_free + kDwpwA;                                // [kDwpwB]
+  uint64_t* y_full = b_free + kDwpwB;                                // [kDwpwB]
+  uint64_t* h_full = y_full + kDwpwB;                                // [kDwpwH]
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(h_full + kDwpwH);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int y_warps = 4 * chunks, mma_warp = kDwpwThreads / 32 - 1;
+  const int G = gridDim.x;
+  const int my_tiles = (p.n_tiles8 - static_cast<int>(blockIdx.x) + G - 1) / G;
+  const int blocks = C > 128 ? 2 : 1;
+  const uint32_t tcols = blocks == 2 ? 512u : 256u;
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    mbar_init(halo_bar, 1);
+    for (int i = 0; i < kDwpwA; ++i) {
+      mbar_init(&dz_full[i], 1);
+      mbar_init(&a_free[i], 1);
+    }
+    for (int i = 0; i < kDwpwB; ++i) {
+      mbar_init(&b_free[i], 1);
+      mbar_init(&y_full[i], 32 * y_warps);
+    }
+    for (int i = 0; i < kDwpwH; ++i) mbar_init(&h_full[i], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  // thread 0 loads the halo of each of the CTA's tiles; halos issued / waited for
-  int halo_issued = 0, halo_seen = 0;
-  auto load_halo = [&](int t) {
-    int b, i0, j0;
-    cla_tile(p, t, b, i0, j0);
-    mbar_arrive_expect_tx(halo_bar, kClaHaloBytes * chunks);
-    for (int g = 0; g < chunks; ++g)
-      tma_load_4d(sH + g * kDwpwHaloChunk, &tm_x, halo_bar, 64 * g, j0 - 1, i0 - 1, b);
-    ++halo_issued;
-  };
-  for (int i = threadIdx.x; i < C; i += blockDim.x) {
-    sBdw[i] = p.b_dw[i];
-#pragma unroll
-    for (int tp = 0; tp < 9; ++tp) sWdw[tp * C + i] = p.w_dw[i * 9 + tp];
-  }
-  // rows C..255 of dz^T are padding: zero them once (they only feed
-  // accumulator rows that are never read, but stay finite)
-  for (int i = threadIdx.x * 16; i < 256 * 256; i += blockDim.x * 16)
-    *reinterpret_cast<uint4*>(sA + i) = make_uint4(0, 0, 0, 0);
-  fence_proxy_async_smem();
   if (warp == 0) {
-    tmem_alloc(tbase, 512);
+    tmem_alloc(tbase, tcols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tbase;
-  const uint32_t idesc = make_idesc_bf16(128, C, true, true);
-  const uint64_t adesc = make_sdesc(smem_u32(sA), 128, 2048, kLayoutNone);
-  const uint64_t bdesc = make_sdesc(smem_u32(sB), 128, 2048, kLayoutNone);
-  const bool two = C > 128;
-  // (after the barrier initialisation above is visible to the async proxy)
-  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < p.n_tiles) load_halo(blockIdx.x);
+  auto tile_origin8 = [&](int n, int& b, int& i0, int& j0) {
+    const int t = static_cast<int>(blockIdx.x) + n * G;
+    const int per_img = p.n_tiles8 / p.B;
+    b = t / per_img;
+    const int tt = t % per_img;
+    i0 = (tt / p.tiles_x8) * 8;
+    j0 = (tt % p.tiles_x8) * 8;
+  };
   bool ok = true;
-  int phase = 0, n_done = 0;
-  for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x, ++n_done) {
-    int b, i0, j0;
-    cla_tile(p, t, b, i0, j0);
-    // items: (pixel r, channel octet k = 8 ch + ko); a warp takes 4
-    // neighbouring pixels x 8 octets of one 64-channel chunk, so its global
-    // reads are 128-byte runs and its halo reads 512 contiguous bytes
-    const int n_items = chunks * 1024;
-    // dz^T: 8 output channels of pixel r
-#pragma unroll 2
-    for (int it = threadIdx.x; it < n_items; it += blockDim.x) {
-      const int ko = it & 7, q = it >> 5, ch = q % chunks, k = ch * 8 + ko;
-      const int r = (q / chunks) * 4 + ((it >> 3) & 3);
-      if (k >= octets) continue;
-      const size_t zoff = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
-      const uint4 zv = rib_guard(zoff + 7, cla_elems(p), G_CLA_IN) ? ldg_nc_v4(p.dz + zoff)
-                                                                   : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(sA + cla_mnmajor_offset(r, 8 * k)) = zv;
+  if (warp == mma_warp) {
+    // ------------------------------------------------ TMA loads and MMAs
+    int dz_issued = 0, h_issued = 0, dz_seen = 0, n_mma = 0;
+    auto issue_dz = [&](int n) {   // lane 0
+      int b, i0, j0;
+      tile_origin8(n, b, i0, j0);
+      uint64_t* bar = &dz_full[n % kDwpwA];
+      mbar_arrive_expect_tx(bar, kDwpwAtom * chunks);
+      for (int g = 0; g < chunks; ++g)
+        tma_load_4d(base + L.a + (n % kDwpwA) * chunk_bytes + g * kDwpwAtom, &tm_dz, bar, 64 * g,
+                    j0, i0, b);
+      ++dz_issued;
+    };
+    auto issue_halo = [&](int n) {   // lane 0
+      int b, i0, j0;
+      tile_origin8(n, b, i0, j0);
+      uint64_t* bar = &h_full[n % kDwpwH];
+      mbar_arrive_expect_tx(bar, kDwpwHaloBytes * chunks);
+      for (int g = 0; g < chunks; ++g)
+        tma_load_4d(base + L.halo + ((n % kDwpwH) * chunks + g) * kDwpwHaloSlot, &tm_x, bar,
+                    64 * g, j0 - 1, i0 - 1, b);
+      ++h_issued;
+    };
+    if (lane == 0) {
+      for (int n = 0; n < 2 && n < my_tiles; ++n) {
+        issue_dz(n);
+        issue_halo(n);
+      }
     }
-    ok = mbar_wait(halo_bar, halo_seen & 1, abort_flag, p.wait_limit_ns, SITE_CLA);
-    ++halo_seen;
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      break;
+    const uint32_t idesc = make_idesc_bf16(128, C, true, true);
+    for (int n = 0; ok && n < my_tiles; ++n) {
+      ok = mbar_wait(&y_full[n % kDwpwB], (n / kDwpwB) & 1, abort_flag, p.wait_limit_ns,
+                     SITE_CLA) &&
+           mbar_wait(&dz_full[n % kDwpwA], (n / kDwpwA) & 1, abort_flag, p.wait_limit_ns,
+                     SITE_CLA);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++dz_seen;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(base + L.a + (n % kDwpwA) * chunk_bytes);
+      const uint64_t bdesc =
+          make_sdesc(smem_u32(base + L.b + (n % kDwpwB) * chunk_bytes), kDwpwAtom, 1024,
+                     kLayoutSW128);
+      for (int m = 0; m < blocks; ++m) {
+        const uint64_t adesc = make_sdesc(a0 + 2 * m * kDwpwAtom, kDwpwAtom, 1024, kLayoutSW128);
+        for (int ks = 0; ks < 4; ++ks)
+          umma_ss_elect(tmem + 256 * m, adesc + ks * (2048 >> 4), bdesc + ks * (2048 >> 4), idesc,
+                        (n > 0 || ks > 0) ? 1u : 0u);
+      }
+      umma_commit_elect(&a_free[n % kDwpwA]);
+      umma_commit_elect(&b_free[n % kDwpwB]);
+      ++n_mma;
+      // the y warps are done with halo slot n % 2: tile n + 2's halo goes there
+      if (lane == 0 && n + kDwpwH < my_tiles) issue_halo(n + kDwpwH);
+      // dz of tile n + 2 goes to the buffer the MMAs of tile n - 1 read
+      if (n + 2 < my_tiles) {
+        if (n >= 1)
+          ok = mbar_wait(&a_free[(n + 2) % kDwpwA], ((n - 1) / kDwpwA) & 1, abort_flag,
+                         p.wait_limit_ns, SITE_CLA);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && lane == 0) issue_dz(n + 2);
+      }
     }
-    // y^T: the depth-wise convolution of x from the halo (zero outside the
-    // map: the TMA fills out-of-range pixels with zeros)
-#pragma unroll 2
-    for (int it = threadIdx.x; it < n_items; it += blockDim.x) {
-      const int ko = it & 7, q = it >> 5, ch = q % chunks, k = ch * 8 + ko;
-      const int r = (q / chunks) * 4 + ((it >> 3) & 3);
-      if (k >= octets) continue;
-      const int i = r >> 4, j = r & 15;   // tile-local; halo row i + u, column j + v
-      const uint8_t* h = sH + ch * kDwpwHaloChunk + ko * 16;
-      float a[8];
+    // The accumulator is read once the last tile's MMAs (and so every
+    // earlier one) are done.  After an error, every TMA load and MMA still
+    // in flight lands before the CTA exits.
+    volatile int no_abort = 0;
+    const uint64_t drain = 200ull * 1000ull * 1000ull;
+    bool w = true;
+    if (n_mma > 0)
+      w = mbar_wait(&a_free[(n_mma - 1) % kDwpwA], ((n_mma - 1) / kDwpwA) & 1,
+                    ok ? abort_flag : &no_abort, ok ? p.wait_limit_ns : drain, SITE_CLA);
+    if (!ok) {
+      *abort_flag = 1;
+      for (int n = dz_seen; n < dz_issued; ++n)
+        mbar_wait(&dz_full[n % kDwpwA], (n / kDwpwA) & 1, &no_abort, drain, SITE_CLA);
+      // halo loads are issued for tiles the y warps have consumed, or for the
+      // next two: wait for those not yet seen complete
+      for (int n = max(0, h_issued - kDwpwH); n < h_issued; ++n)
+        mbar_wait(&h_full[n % kDwpwH], (n / kDwpwH) & 1, &no_abort, drain, SITE_CLA);
+    }
+    w = __all_sync(0xffffffffu, w);
+    if (!w && lane == 0) *abort_flag = 1;
+  } else if (warp < y_warps) {
+    // ------------------------------------------------ y = b_dw + DW3x3(x)
+    // thread: chunk g = warp / 4, octet ko of it, column j and rows 4 h ..
+    // 4 h + 3 of the tile; a warp covers 4 neighbouring columns x 8 octets,
+    // so its halo reads and y stores are 512-byte runs
+    const int g = warp >> 2, ko = lane & 7;
+    const int pg = ((warp & 3) << 2) | (lane >> 3);   // 0..15
+    const int j = pg & 7, h = pg >> 3;
+    const int k = 8 * g + ko;                         // channel octet
+    const bool act = k < octets;
+    uint64_t wp[9][4];                                // taps (u, v) of channels 8k .. 8k+7
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a[e] = sBdw[8 * k + e];
+    for (int e = 0; e < 4; ++e) {
+      const int c = 8 * k + 2 * e;
 #pragma unroll
-      for (int u = 0; u < 3; ++u)
+      for (int tp = 0; tp < 9; ++tp)
+        wp[tp][e] = act ? pk2(p.w_dw[c * 9 + tp], p.w_dw[(c + 1) * 9 + tp]) : 0ull;
+    }
+    for (int n = 0; ok && n < my_tiles; ++n) {
+      ok = mbar_wait(&h_full[n % kDwpwH], (n / kDwpwH) & 1, abort_flag, p.wait_limit_ns,
+                     SITE_CLA);
+      if (ok && n >= kDwpwB)   // y buffer n % 2 was last read by the MMAs of tile n - 2
+        ok = mbar_wait(&b_free[n % kDwpwB], ((n - kDwpwB) / kDwpwB) & 1, abort_flag,
+                       p.wait_limit_ns, SITE_CLA);
+      if (!ok) break;
+      uint8_t* sB = base + L.b + (n % kDwpwB) * chunk_bytes + g * kDwpwAtom;
+      const uint8_t* hs = base + L.halo + ((n % kDwpwH) * chunks + g) * kDwpwHaloSlot + ko * 16;
+      uint64_t acc[4][4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {   // b_dw (re-read per tile: fewer live registers)
+        const float2 bd = act ? __ldg(reinterpret_cast<const float2*>(p.b_dw + 8 * k + 2 * e))
+                              : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc[m][e] = pk2(bd.x, bd.y);
+      }
+      // halo row ri (map row 4h + ri - 1 of the tile) feeds pixel m with tap
+      // row u = ri - m; for each pixel the taps arrive in (u, v) order.  Each
+      // halo vector is converted once and used by up to three pixels.
+#pragma unroll
+      for (int ri = 0; ri < 6; ++ri)
 #pragma unroll
         for (int v = 0; v < 3; ++v) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(h + ((i + u) * 18 + (j + v)) * 128);
+          const uint4 xv = *reinterpret_cast<const uint4*>(hs + ((4 * h + ri) * 10 + j + v) * 128);
           const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-          const float* w = sWdw + (u * 3 + v) * C + 8 * k;
+          uint64_t xf[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
-            a[2 * e] = fmaf(w[2 * e], xf.x, a[2 * e]);
-            a[2 * e + 1] = fmaf(w[2 * e + 1], xf.y, a[2 * e + 1]);
+          for (int e = 0; e < 4; ++e)
+            xf[e] = pk2(__uint_as_float(xw[e] << 16), __uint_as_float(xw[e] & 0xffff0000u));
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int u = ri - m;
+            if (u < 0 || u > 2) continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[m][e] = ffma2(wp[u * 3 + v][e], xf[e], acc[m][e]);
           }
         }
-      *reinterpret_cast<uint4*>(sB + cla_mnmajor_offset(r, 8 * k)) =
-          make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                     pack_bf16x2(a[6], a[7]));
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // the halo is read: fetch the next tile's while this one's MMAs run
-    if (threadIdx.x == 0 && t + static_cast<int>(gridDim.x) < p.n_tiles)
-      load_halo(t + gridDim.x);
-    // D0 (+)= dz^T[o 0..127] y, D1 (+)= dz^T[o 128..255] y: 8 K-steps of 16 pixels
-    if (warp == 0) {
-      const uint32_t acc = n_done > 0 ? 1u : 0u;
-      for (int ks = 0; ks < 8; ++ks) {
-        umma_ss_elect(tmem, adesc + ks * 16, bdesc + ks * 16, idesc, (acc | ks) ? 1u : 0u);
-        if (two)
-          umma_ss_elect(tmem + 256, adesc + (16 * 2048 >> 4) + ks * 16, bdesc + ks * 16, idesc,
-                        (acc | ks) ? 1u : 0u);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = (4 * h + m) * 8 + j;
+        const uint4 yv = act ? make_uint4(pack_bf16x2(lo2(acc[m][0]), hi2(acc[m][0])),
+                                          pack_bf16x2(lo2(acc[m][1]), hi2(acc[m][1])),
+                                          pack_bf16x2(lo2(acc[m][2]), hi2(acc[m][2])),
+                                          pack_bf16x2(lo2(acc[m][3]), hi2(acc[m][3])))
+                             : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sB + r * 128 + ((ko ^ (r & 7)) << 4)) = yv;
       }
-      umma_commit_elect(bar);
+      fence_proxy_async_smem();
+      mbar_arrive(&y_full[n % kDwpwB]);
     }
-    // the operands are rewritten for the next tile once the MMAs are done
-    ok = mbar_wait(bar, phase, abort_flag, p.wait_limit_ns, SITE_CLA);
-    phase ^= 1;
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
   }
-  if (!ok) {
-    volatile int no_abort = 0;
-    mbar_wait(bar, phase ^ 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
-    // a halo still in flight lands before the CTA exits
-    if (threadIdx.x == 0 && halo_issued > halo_seen)
-      mbar_wait(halo_bar, (halo_issued - 1) & 1, &no_abort, 200ull * 1000ull * 1000ull, SITE_CLA);
-  }
-  // the CTA's partial dW_pw: rows o from TMEM lanes, C columns each
-  if (ok && warp < 8) {
-    const int q = warp & 3, half = warp >> 2;
-    const int o = half * 128 + q * 32 + lane;
-    const uint32_t taddr = tmem + half * 256 + (static_cast<uint32_t>(q * 32) << 16);
-    if (half == 0 || two) {
-      float* dst = p.part_dwpw + (static_cast<size_t>(blockIdx.x) * C + o) * C;
-      const bool in = o >= C || rib_guard((static_cast<size_t>(blockIdx.x) * C + o) * C + C - 1,
-                                          static_cast<size_t>(p.grid) * C * C, G_CLA_PART);
-      for (int c0 = 0; c0 < C; c0 += 32) {   // every lane: the TMEM loads are collective
-        uint32_t v[32];
+  __syncthreads();
+  ok = *abort_flag == 0;
+  tc_fence_after();
+  // the CTA's partial dW_pw: warp w < 8 reads TMEM lanes 32 (w % 4).. of
+  // block w / 4 (rows o), all C columns
+  if (warp < 4 * blocks) {
+    const int q = warp & 3, blk = warp >> 2;
+    const int o = blk * 128 + q * 32 + lane;
+    const uint32_t taddr = tmem + blk * 256 + (static_cast<uint32_t>(q * 32) << 16);
+    float* dst = p.part_dwpw + (static_cast<size_t>(blockIdx.x) * C + o) * C;
+    const bool in = o >= C || rib_guard((static_cast<size_t>(blockIdx.x) * C + o) * C + C - 1,
+                                        static_cast<size_t>(p.grid) * C * C, G_CLA_PART);
+    for (int c0 = 0; ok && c0 < C; c0 += 32) {   // every lane: the TMEM loads are collective
+      uint32_t v[32];
+      if (my_tiles > 0) {
         tmem_ld_x32(taddr + c0, v);
         tmem_wait_ld();
         reg_fence_x32(v);
-        if (o < C && n_done > 0 && in) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c0);
+      } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-        } else if (o < C && in) {
-          for (int e = 0; e < 32; ++e) dst[c0 + e] = 0.f;
-        }
+        for (int e = 0; e < 32; ++e) v[e] = 0u;   // no tiles: an empty sum
+      }
+      if (o < C && in) {
+        float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
       }
     }
   }
@@ -429,7 +551,7 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, tcols);
   }
 }
 
@@ -442,8 +564,9 @@ __global__ void __launch_bounds__(kClaBwdThreads, 1)
 // zero padding is the TMA's out-of-range fill), and a warp walks down a
 // tile column with the 3 x 3 neighbourhoods of x and dy in registers,
 // reading only the new row of each per pixel.
+constexpr uint32_t kClaHaloSlot = (kClaHaloBytes + 1023u) & ~1023u;   // one 10 x 18 halo box
 __host__ __device__ __forceinline__ size_t cla_dx_smem_bytes() {
-  return 4ull * kDwpwHaloChunk + 64 + 1024;
+  return 4ull * kClaHaloSlot + 64 + 1024;
 }
 
 __device__ __forceinline__ float2 cla_lds2(const uint8_t* ptr) {
@@ -456,7 +579,7 @@ __global__ void __launch_bounds__(kClaDxThreads, 2)
                       const __grid_constant__ CUtensorMap tm_dy, const ClaBwdParams p) {
   extern __shared__ uint8_t dx_raw[];
   uint8_t* base = dx_raw + ((1024u - (smem_u32(dx_raw) & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + 4 * kDwpwHaloChunk);   // [2] stages
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + 4 * kClaHaloSlot);   // [2] stages
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.C;
@@ -470,8 +593,8 @@ __global__ void __launch_bounds__(kClaDxThreads, 2)
   const int G = gridDim.x;
   const int my_tiles = (p.n_tiles - static_cast<int>(blockIdx.x) + G - 1) / G;
   // stage s: x halo at base + s * chunk, dy halo at base + (2 + s) * chunk
-  auto hx = [&](int st) { return base + st * kDwpwHaloChunk; };
-  auto hdy = [&](int st) { return base + (2 + st) * kDwpwHaloChunk; };
+  auto hx = [&](int st) { return base + st * kClaHaloSlot; };
+  auto hdy = [&](int st) { return base + (2 + st) * kClaHaloSlot; };
   int issued = 0, consumed = 0;   // halo loads (thread 0 issues; all threads consume)
   auto issue = [&](int g, int k) {
     int b, i0, j0;
@@ -589,25 +712,58 @@ __global__ void __launch_bounds__(kClaDxThreads, 2)
 }
 
 // -------------------------------------------------------------- reduction
-// Fixed-order sums over the CTAs' partials; one thread per gradient element
-// (C*C of dW_pw, then C of db_pw, 9C of dW_dw, C of db_dw).
-__global__ void __launch_bounds__(256) cla_bwd_reduce_kernel(const ClaBwdParams p) {
-  const int C = p.C;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  const int n_pw = C * C;
-  if (idx >= n_pw + 11 * C) return;
-  float s = 0.f;
+// Fixed-order sums over the CTAs' partials of the C*C dW_pw, C db_pw and
+// 10C dW_dw / db_dw gradient elements.  A block takes 32 consecutive
+// elements (lane = element, so every warp's loads are 128-byte runs); warp
+// w sums the partials of CTAs [w per, (w + 1) per) with four accumulators
+// taking the CTAs in turn, and warp 0 adds the kClaRedWarps warp sums in warp
+// order, so the result is the same on every run.
+constexpr int kClaRedWarps = 16;
+__global__ void __launch_bounds__(32 * kClaRedWarps) cla_bwd_reduce_kernel(const ClaBwdParams p) {
+  __shared__ float part[kClaRedWarps][32];
+  const int C = p.C, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int n_pw = C * C, n_all = n_pw + 11 * C;
+  const int idx = blockIdx.x * 32 + lane;
+  // element idx: its partials are src[k * stride], k < count
+  const float* src = nullptr;
+  size_t stride = 0;
+  int count = 0;
   if (idx < n_pw) {
-    for (int k = 0; k < p.grid; ++k) s += p.part_dwpw[static_cast<size_t>(k) * n_pw + idx];
+    src = p.part_dwpw + idx;
+    stride = static_cast<size_t>(n_pw);
+    count = p.grid;
+  } else if (idx < n_pw + C) {
+    src = p.part_dbpw + (idx - n_pw);
+    stride = static_cast<size_t>(C);
+    count = p.grid;
+  } else if (idx < n_all) {
+    src = p.part_dw + (idx - n_pw - C);   // [k][10][C]: element (tap, c) at k * 10C + tap * C + c
+    stride = 10ull * C;
+    count = p.grid_dx;
+  }
+  const int per = (count + kClaRedWarps - 1) / kClaRedWarps;
+  const int k0 = min(count, w * per), k1 = min(count, k0 + per);
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  if (src) {
+    int k = k0;
+    for (; k + 3 < k1; k += 4) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] += src[(k + e) * stride];
+    }
+    for (; k < k1; ++k) a[0] += src[k * stride];
+  }
+  part[w][lane] = (a[0] + a[1]) + (a[2] + a[3]);
+  __syncthreads();
+  if (w != 0 || !src) return;
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kClaRedWarps; ++i) s += part[i][lane];
+  if (idx < n_pw) {
     p.dw_pw[idx] = s;
   } else if (idx < n_pw + C) {
-    const int o = idx - n_pw;
-    for (int k = 0; k < p.grid; ++k) s += p.part_dbpw[static_cast<size_t>(k) * C + o];
-    p.db_pw[o] = s;
+    p.db_pw[idx - n_pw] = s;
   } else {
-    const int e = idx - n_pw - C;           // 0 .. 10C-1: tap-major [10][C]
-    const int tp = e / C, c = e % C;
-    for (int k = 0; k < p.grid_dx; ++k) s += p.part_dw[(static_cast<size_t>(k) * 10 + tp) * C + c];
+    const int e = idx - n_pw - C, tp = e / C, c = e % C;
     if (tp < 9) p.dw_dw[c * 9 + tp] = s;
     else p.db_dw[c] = s;
   }

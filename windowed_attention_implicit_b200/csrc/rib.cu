@@ -398,7 +398,9 @@ struct ClaBwdLayout {
 
 int cla_check(int B, int H, int W, int C) {
   if (B < 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
-  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u) return RIB_ERR_UNSUPPORTED;
+  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u || cla_dz_smem_bytes(C) > 227u * 1024u ||
+      cla_dwpw_smem_bytes(C) > 227u * 1024u)
+    return RIB_ERR_UNSUPPORTED;
   if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
   if ((long long)B * H * W * C > (1ll << 40) || B > (1 << 20)) return RIB_ERR_UNSUPPORTED;
   if ((long long)B * (H / 8) * (W / 16) > (1ll << 30)) return RIB_ERR_UNSUPPORTED;
@@ -879,6 +881,8 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   p.tiles_x = W / 16;
   p.tiles_per_img = (H / 8) * (W / 16);
   p.n_tiles = L.n_tiles;
+  p.tiles_x8 = W / 8;
+  p.n_tiles8 = B * (H / 8) * (W / 8);
   p.grid = L.grid;
   p.grid_dx = L.grid_dx;
   p.wait_limit_ns = g_wait_limit_ns;
@@ -903,6 +907,21 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
                   CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   }
+  // x again with 10 x 10 boxes (the halo of an 8 x 8 tile), and dz
+  // (workspace) with 8 x 8 boxes in the 128-byte swizzle, for the dW_pw kernel
+  CUtensorMap tm_x10, tm_dz;
+  {
+    const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {2ull * C, 2ull * C * W, 2ull * C * W * H};
+    const uint32_t box10[4] = {64, 10, 10, 1};
+    rc = make_map(&tm_x10, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, dims, strides, box10,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+    const uint32_t box8[4] = {64, 8, 8, 1};
+    rc = make_map(&tm_dz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.dz, dims, strides, box8,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+  }
   const size_t smem_dz = cla_dz_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
   const size_t smem_dx = cla_dx_smem_bytes();
   if ((rc = set_smem(cla_bwd_dz_kernel, smem_dz))) return rc;
@@ -910,12 +929,12 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
   if ((rc = set_smem(cla_bwd_dx_kernel, smem_dx))) return rc;
   {
     TraceScope ts(K_CLA_DZ, st);
-    cla_bwd_dz_kernel<<<L.grid, kClaBwdThreads, smem_dz, st>>>(p);
+    cla_bwd_dz_kernel<<<L.grid, kDzThreads, smem_dz, st>>>(p);
     if ((rc = launch_status())) return rc;
   }
   {
     TraceScope ts(K_CLA_DWPW, st);
-    cla_bwd_dwpw_kernel<<<L.grid, kClaBwdThreads, smem_dw, st>>>(tm_x, p);
+    cla_bwd_dwpw_kernel<<<L.grid, kDwpwThreads, smem_dw, st>>>(tm_x10, tm_dz, p);
     if ((rc = launch_status())) return rc;
   }
   {
@@ -924,7 +943,7 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
     if ((rc = launch_status())) return rc;
   }
   TraceScope ts(K_CLA_RED, st);
-  cla_bwd_reduce_kernel<<<(C * C + 11 * C + 255) / 256, 256, 0, st>>>(p);
+  cla_bwd_reduce_kernel<<<(C * C + 11 * C + 31) / 32, 32 * kClaRedWarps, 0, st>>>(p);
   return launch_status();
 }
 
