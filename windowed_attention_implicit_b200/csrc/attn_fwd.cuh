@@ -15,21 +15,21 @@
 // Persistent CTAs, one per SM, each walking work items = one unit (batch,
 // window, head) x two 128-query tiles (A, B); every barrier phase is counted
 // across items, so the next item's loads and score MMAs overlap the end of
-// the current one.  640 threads (5 warpgroups):
-//   warps 0-7    softmax group A: warp w owns TMEM lanes 32(w%4).. (query
-//                rows) and key columns 64((w/4)%2).. of each score tile; the
-//                two warps sharing a row exchange partial row maxima
-//   warps 8-15   softmax group B, the same for the second query tile
-//   warp  16     TMA producer: each item's Q tiles (two buffers, by item
+// the current one.  384 threads (3 warpgroups):
+//   warps 0-3    softmax group A: warp w owns TMEM lanes 32 w.. (query rows)
+//                and all 128 key columns of each score tile, one thread per
+//                query row, so the row maximum needs no exchange
+//   warps 4-7    softmax group B, the same for the second query tile
+//   warp  8      TMA producer: each item's Q tiles (two buffers, by item
 //                parity), then its K/V/Kp tiles through a 3-stage
 //                shared-memory ring; boxes at rolled map coordinates
-//   warp  17     TMEM allocator; issues the score MMAs
-//   warp  18     issues the PV MMAs of query tile A
-//   warp  19     issues the PV MMAs of query tile B
-// Four softmax warps per SM sub-partition hide the latency of the
-// exponential chains; the softmax warpgroups take 112 registers (with 104
-// the polynomial exponentials spill) and the service warpgroup 32
-// (setmaxnreg).
+//   warp  9      TMEM allocator; issues the score MMAs
+//   warp  10     issues the PV MMAs of query tile A
+//   warp  11     issues the PV MMAs of query tile B
+// Each SM sub-partition runs one softmax warp of each query tile; a thread's
+// 128 independent columns keep the exponential pipes fed.  The softmax
+// warpgroups take 208 registers (the 128 scores of a row stay in registers)
+// and the service warpgroup 56 (setmaxnreg).
 //
 // One thread issues at most one tcgen05.mma every ~43 cycles (an elected
 // lane of a converged warp; ~90 from a divergent branch), while the tensor
@@ -64,11 +64,11 @@
 namespace rib {
 
 constexpr int kFwdStages = 3;
-constexpr int kFwdThreads = 640;
-constexpr int kFwdLaunchRegs = 96;      // what the host checks ptxas gave (65536 / 640)
-constexpr int kFwdSoftmaxRegs = 112;    // warpgroups 0-3
-constexpr int kFwdServiceRegs = 32;     // warpgroup 4
-static_assert(4 * 128 * kFwdSoftmaxRegs + 128 * kFwdServiceRegs <= kFwdThreads * kFwdLaunchRegs,
+constexpr int kFwdThreads = 384;
+constexpr int kFwdLaunchRegs = 168;     // what the host checks ptxas gave (65536 / 384)
+constexpr int kFwdSoftmaxRegs = 208;    // warpgroups 0-1
+constexpr int kFwdServiceRegs = 56;     // warpgroup 2
+static_assert(2 * 128 * kFwdSoftmaxRegs + 128 * kFwdServiceRegs <= kFwdThreads * kFwdLaunchRegs,
               "register split exceeds the launch budget");
 constexpr uint32_t kFwdTmemCols = 512;
 constexpr int kRegions = 3;
@@ -113,9 +113,7 @@ struct __align__(1024) FwdSmem {
   uint64_t s_full[kRegions], r_free[kRegions];
   uint64_t p_full[2][2];          // [tile X][key tile parity]
   int pv_count[2];                // PV steps of tile X known complete
-  uint64_t pair_bar[2][4];        // the two warps sharing 32 rows of a tile
   uint64_t drain;
-  float red_max[2][2][2][128];    // [tile parity][group][column half][row] partial maxima
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -136,7 +134,7 @@ __device__ __forceinline__ void fwd_item(const FwdParams& p, int it, UnitCoord& 
   tile0 = 2 * (it % pairs);
 }
 
-// Warp 16, lane 0: Q of each item into the buffer of its parity (once the
+// Warp 8, lane 0: Q of each item into the buffer of its parity (once the
 // score MMAs of the item two back have read it), then its K/V/Kp tiles
 // through the ring.
 __device__ __forceinline__ void fwd_producer(FwdSmem& sm, const CUtensorMap* tq,
@@ -202,7 +200,7 @@ __device__ __forceinline__ void fwd_producer(FwdSmem& sm, const CUtensorMap* tq,
   }
 }
 
-// Warp 17: S(K) = Q_X K_J^T into region K % 3 for the score tiles
+// Warp 9: S(K) = Q_X K_J^T into region K % 3 for the score tiles
 // K = 2 J + X of every item, in order, each once the region has been freed
 // by the PV MMA of score tile K - 3.  After an item's last score tile the
 // commit to q_free releases its Q buffer.
@@ -247,7 +245,7 @@ __device__ __forceinline__ void fwd_mma_scores(FwdSmem& sm, uint32_t tmem, const
   mbar_wait(&sm.drain, 0, &no_abort, kFwdDrainNs, SITE_FWD_DRAIN);
 }
 
-// Warps 18 (X = 0) and 19 (X = 1), all lanes, one elected lane issuing:
+// Warps 10 (X = 0) and 11 (X = 1), all lanes, one elected lane issuing:
 // [O|L]_X (+)= P(K) [V_J | 1] for K = 2 J + X once group X has written P(K);
 // the first key tile of an item overwrites [O|L]_X, once the epilogue of the
 // previous item has read it (o_free).  The commits free the region and
@@ -319,12 +317,12 @@ __device__ __forceinline__ bool wait_pv_count(FwdSmem& sm, int X, int need, cons
 }
 
 // One work item (the CTA's li-th) of a softmax warp: tile X of the item's
-// pair, 32 rows (quarter wq), key columns 64 h .. 64 h + 63.  Returns false
-// on abort.
+// pair, 32 rows (quarter wq), all 128 key columns of each score tile (one
+// thread = one query row).  Returns false on abort.
 template <bool kMask>
 __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, const FwdParams& p,
-                                                 const UnitCoord& u, int tile0, int X, int h,
-                                                 int wq, int li) {
+                                                 const UnitCoord& u, int tile0, int X, int wq,
+                                                 int li) {
   volatile int* ab = &sm.abort_flag;
   const uint64_t lim = p.wait_limit_ns;
   const int lane = threadIdx.x & 31;
@@ -335,8 +333,8 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
   const uint64_t sl2 = pk2(sl, sl);
   const int n = p.n_tiles;
   // region mask: bands of this row's query token.  A warp's 32 rows are a
-  // 4 x 8 block of the window and its 64 key columns an 8 x 8 block, so the
-  // mask is one warp-uniform decision per key tile (kv).
+  // 4 x 8 block of the window and each half (64 columns) of a key tile an
+  // 8 x 8 block, so the mask is one warp-uniform decision per key-tile half.
   const bool mask_on = kMask && (u.wy == p.nW / p.nWx - 1 || u.wx == p.nWx - 1);
   int qbr = 0, qbc = 0;
   if (mask_on) {
@@ -351,53 +349,46 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
   for (int j = 0; j < n; ++j) {
     const int J = li * n + j;   // key tile counted across items
     const int k = 2 * J + X, r = k % kRegions;
-    bool kv = true;
+    bool kv0 = true, kv1 = true;
     if (mask_on) {
       int ki0, kj0;
       tile_origin(j, p.tiles_x, ki0, kj0);
-      kv = region_band(u.wy * p.M + ki0, p.H, p.M, p.s) == qbr &&
-           region_band(u.wx * p.M + kj0 + 8 * h, p.W, p.M, p.s) == qbc;
+      const bool rows_ok = region_band(u.wy * p.M + ki0, p.H, p.M, p.s) == qbr;
+      kv0 = rows_ok && region_band(u.wx * p.M + kj0, p.W, p.M, p.s) == qbc;
+      kv1 = rows_ok && region_band(u.wx * p.M + kj0 + 8, p.W, p.M, p.s) == qbc;
     }
-    const uint32_t tS = tl + r * 128 + 64 * h;  // this warp's 64 score columns
-    const uint32_t tP = tl + r * 128 + 32 * h;  // its 64 bf16 P values, packed in pairs
+    const uint32_t tS = tl + r * 128;  // the row's 128 score columns
+    const uint32_t tP = tl + r * 128;  // its 128 bf16 P values, packed in pairs
     if (!(ok = warp_wait(&sm.s_full[r], (k / kRegions) & 1, ab, lim, SITE_FWD_SOFTMAX,
                          kFwdSleepNs)))
       break;
     tc_fence_after();
-    uint32_t s[2][32];
-    tmem_ld_x32(tS, s[0]);
-    tmem_ld_x32(tS + 32, s[1]);
-    tmem_wait_ld();
-    reg_fence_x32(s[0]);
-    reg_fence_x32(s[1]);
-
-    // row maximum: this warp's 64 columns, then the partner warp's.  The
-    // exchange also orders both warps' score loads before either overwrites
-    // the region with P.
-    // four independent chains of 16 keep the reduction's latency short
-    float m4[4];
+    uint32_t s[4][32];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 4; ++q) tmem_ld_x32(tS + 32 * q, s[q]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) reg_fence_x32(s[q]);
+
+    // row maximum over the 128 columns: eight independent chains of 16
+    float m8[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
       const uint32_t* v = &s[q >> 1][(q & 1) * 16];
       float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
 #pragma unroll
       for (int e = 3; e + 1 < 16; e += 2)
         m = fmax3(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-      m4[q] = fmaxf(m, __uint_as_float(v[15]));
+      m8[q] = fmaxf(m, __uint_as_float(v[15]));
     }
-    float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-    if (!kv) mx = -INFINITY;   // a masked key block adds nothing to the row maximum
-    sm.red_max[J & 1][X][h][row] = mx;
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.pair_bar[X][wq]);
-    if (!(ok = warp_wait(&sm.pair_bar[X][wq], J & 1, ab, lim, SITE_FWD_SOFTMAX, kFwdSleepNs)))
-      break;
-    tc_fence_after();
-    mx = fmaxf(mx, sm.red_max[J & 1][X][h ^ 1][row]);
+    float mh0 = fmaxf(fmax3(m8[0], m8[1], m8[2]), m8[3]);
+    float mh1 = fmaxf(fmax3(m8[4], m8[5], m8[6]), m8[7]);
+    if (!kv0) mh0 = -INFINITY;   // a masked key block adds nothing to the row maximum
+    if (!kv1) mh1 = -INFINITY;
+    const float mx = fmaxf(mh0, mh1);
 
-    // (a key tile masked for both halves of a row leaves mx = -inf: the
-    // running maximum then stays at a finite floor, so no -inf - -inf arises)
+    // (a key tile masked for the whole row leaves mx = -inf: the running
+    // maximum then stays at a finite floor, so no -inf - -inf arises)
     const float m_tile = mask_on ? fmaxf(mx * sl, -1e30f) : mx * sl;
     float m_new = m_run, alpha = 1.f;
     bool resc = false;
@@ -410,7 +401,7 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
     }
     const uint64_t neg2 = pk2(-m_new, -m_new);
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < 4; ++c) {
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -427,7 +418,7 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
         }
         pk[e] = pack_bf16x2(p0, p1);
       }
-      if (kv) {
+      if (c < 2 ? kv0 : kv1) {
         tmem_st_x16(tP + c * 16, pk);
       } else {
         // a masked block: P = 0 exactly (its own store, so that the
@@ -436,10 +427,9 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
         tmem_st_x16(tP + c * 16, z16);
       }
     }
-    // the column-half-0 warp of each row pair rescales [O|L] (both halves
-    // took the same decision from the same row maximum), once every PV step
-    // accumulated so far has completed
-    if (h == 0 && __any_sync(0xffffffffu, resc)) {
+    // rescale [O|L] of this warp's rows once every PV step accumulated so
+    // far has completed
+    if (__any_sync(0xffffffffu, resc)) {
       if (!(ok = wait_pv_count(sm, X, J, p))) break;
       uint32_t o[32], l[16];
       tmem_ld_x32(tO, o);
@@ -461,7 +451,6 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
     m_run = m_new;
   }
   if (!ok) return false;
-  if (h != 0) return true;
   if (!wait_pv_count(sm, X, (li + 1) * n, p)) return false;
   uint32_t o[32], l[16];
   tmem_ld_x32(tO, o);
@@ -520,16 +509,16 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
   return true;
 }
 
-// Warps 0-15: the softmax of every work item of the CTA in turn.
+// Warps 0-7: the softmax of every work item of the CTA in turn.
 template <bool kMask>
 __device__ __forceinline__ void fwd_softmax(FwdSmem& sm, uint32_t tmem, const FwdParams& p, int X,
-                                            int h, int wq) {
+                                            int wq) {
   int li = 0;
   for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++li) {
     UnitCoord u;
     int tile0;
     fwd_item(p, it, u, tile0);
-    if (!fwd_softmax_item<kMask>(sm, tmem, p, u, tile0, X, h, wq, li)) return;
+    if (!fwd_softmax_item<kMask>(sm, tmem, p, u, tile0, X, wq, li)) return;
   }
 }
 
@@ -560,10 +549,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&sm.r_free[r], 1);
     }
     for (int X = 0; X < 2; ++X) {
-      mbar_init(&sm.p_full[X][0], 8);
-      mbar_init(&sm.p_full[X][1], 8);
+      mbar_init(&sm.p_full[X][0], 4);
+      mbar_init(&sm.p_full[X][1], 4);
       sm.pv_count[X] = 0;
-      for (int q = 0; q < 4; ++q) mbar_init(&sm.pair_bar[X][q], 2);
     }
     mbar_init(&sm.drain, 3);   // one commit from each MMA-issuing thread
     sm.abort_flag = 0;
@@ -576,14 +564,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_proxy_async_smem();
   }
-  if (warp == 16 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_qkv);
     if (p.rank > 0) {
       tma_prefetch_desc(&tm_qp);
       tma_prefetch_desc(&tm_kp);
     }
   }
-  if (warp == 17) {
+  if (warp == 9) {
     tmem_alloc(&sm.tmem_base, kFwdTmemCols);
     tmem_relinquish();
   }
@@ -591,22 +579,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp < 16) {
+  if (warp < 8) {
     regs_inc<kFwdSoftmaxRegs>();
-    fwd_softmax<kMask>(sm, tmem, p, warp >> 3, (warp >> 2) & 1, warp & 3);
+    fwd_softmax<kMask>(sm, tmem, p, warp >> 2, warp & 3);
   } else {
     regs_dec<kFwdServiceRegs>();
-    if (warp == 16) {
+    if (warp == 8) {
       if (lane == 0) fwd_producer(sm, &tm_qkv, &tm_qp, &tm_kp, p);
-    } else if (warp == 17) {
+    } else if (warp == 9) {
       fwd_mma_scores(sm, tmem, p);
     } else {
-      fwd_mma_pv(sm, tmem, p, warp - 18);  // warps 18, 19
+      fwd_mma_pv(sm, tmem, p, warp - 10);  // warps 10, 11
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 17) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kFwdTmemCols);
   }
