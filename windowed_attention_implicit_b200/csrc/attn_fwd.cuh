@@ -77,7 +77,7 @@ constexpr int kOCols = 48;
 static_assert(kRegions * 128 + 2 * kOCols <= kFwdTmemCols, "forward TMEM layout exceeds 512 columns");
 // Of every 16 element pairs, how many exponentials run on the FMA pipe.
 #ifndef RIB_FWD_POLY_PAIRS
-#define RIB_FWD_POLY_PAIRS 4
+#define RIB_FWD_POLY_PAIRS 5
 #endif
 constexpr int kPolyPairs = RIB_FWD_POLY_PAIRS;
 constexpr uint64_t kFwdDrainNs = 200ull * 1000ull * 1000ull;
