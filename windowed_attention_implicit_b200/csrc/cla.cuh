@@ -125,11 +125,25 @@ __global__ void __launch_bounds__(kClaThreads, 1)
     bb.abort_flag = 0;
     fence_mbarrier_init();
   }
-  // W_pw -> bf16 B operand (row n = output channel, k = input channel)
-  for (int i = threadIdx.x; i < C * C / 2; i += blockDim.x) {
-    const int n = (2 * i) / C, k = (2 * i) % C;
-    const float2 w = *reinterpret_cast<const float2*>(p.w_pw + static_cast<size_t>(n) * C + k);
-    *reinterpret_cast<uint32_t*>(sW + cla_kmajor_offset(n, k, C)) = pack_bf16x2(w.x, w.y);
+  // W_pw -> bf16 B operand (row n = output channel, k = input channel).
+  // Pair i is W_pw[2i], W_pw[2i + 1]; eight pairs' loads are issued before
+  // any store, so the fill costs a few memory latencies, not one per pair.
+  const int n_pairs = C * C / 2;
+  for (int i0 = threadIdx.x; i0 < n_pairs; i0 += 8 * blockDim.x) {
+    float2 w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * static_cast<int>(blockDim.x);
+      w[e] = i < n_pairs ? __ldg(reinterpret_cast<const float2*>(p.w_pw) + i)
+                         : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * static_cast<int>(blockDim.x);
+      if (i >= n_pairs) break;
+      const int n = (2 * i) / C, k = (2 * i) % C;
+      *reinterpret_cast<uint32_t*>(sW + cla_kmajor_offset(n, k, C)) = pack_bf16x2(w[e].x, w[e].y);
+    }
   }
   float* sBias = reinterpret_cast<float*>(base + L.bias);
   float* sWdw = sBias + C;       // [tap][channel]: a warp reads 64 consecutive channels

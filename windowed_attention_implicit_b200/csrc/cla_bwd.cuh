@@ -13,9 +13,11 @@
 // Kernels, in launch order (persistent grids, tiles of
 // 8 x 16 pixels; sums over pixels go through per-CTA partials and a
 // fixed-order reduction, so the weight gradients are deterministic):
-//   cla_bwd_dz_kernel    dO, dz (to the workspace), db_pw partials, and
-//                        dy = dz W_pw on the tensor cores (tcgen05, dz tile
-//                        and W_pw^T in shared memory, accumulator in TMEM)
+//   cla_bwd_dz_kernel    dO, dz (to the workspace), db_pw partials: a plain
+//                        element-wise stream
+//   cla_bwd_dy_kernel    dy = dz W_pw on the tensor cores (tcgen05; dz tiles
+//                        by TMA through a 3-stage ring, W_pw^T resident in
+//                        shared memory, two TMEM accumulators)
 //   cla_bwd_dwpw_kernel  dW_pw partials = sum over the CTA's 8 x 8-pixel
 //                        tiles of dz^T y, y recomputed from x; dz by TMA,
 //                        both operands MN-major with the 128-byte swizzle,
@@ -29,7 +31,7 @@
 
 namespace rib {
 
-constexpr int kDzThreads = 384;   // dz kernel (12 warps: up to 168 registers a thread)
+constexpr int kDzEwThreads = 512;   // element-wise dz kernel
 constexpr int kClaDxThreads = 256;
 
 struct ClaBwdParams {
@@ -69,177 +71,74 @@ __device__ __forceinline__ size_t cla_elems(const ClaBwdParams& p) {
   return static_cast<size_t>(p.B) * p.H * p.W * p.C;
 }
 
-// Element-wise part of the dz kernel: thread = (pixel slot, channel octet),
-// kDzBatch pixels' loads in flight at once (three 16-byte loads a pixel:
-// 48 registers at 4).
+// Element-wise dz kernel: thread = (pixel slot, channel octet), kDzBatch
+// pixels' loads in flight at once (three 16-byte loads a pixel: 48
+// registers at 4).
 constexpr int kDzBatch = 4;
-// W_pw^T (2 C^2 bytes) | two dz tiles (256 C bytes each) | db_pw slots | barriers
-__host__ __device__ __forceinline__ size_t cla_dz_smem_bytes(int C) {
-  return 2ull * C * C + 2ull * 256 * C + 4ull * 8 * kDzThreads + 64 + 1024;
-}
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const __nv_bfloat16* ptr) {
   return __ldg(reinterpret_cast<const uint4*>(ptr));
 }
 
-// -------------------------------------------------------------- dz and dy
-// grid p.grid, block kDzThreads, dynamic smem cla_dz_smem_bytes(C).
-// The dz tile and the dy accumulator are double-buffered: tile n's MMAs run
-// while the threads do tile n + 1's element-wise part, and its dy is read
-// from TMEM after that.
-__global__ void __launch_bounds__(kDzThreads, 1) cla_bwd_dz_kernel(const ClaBwdParams p) {
-  extern __shared__ uint8_t dz_raw[];
-  uint8_t* base = dz_raw + ((1024u - (smem_u32(dz_raw) & 1023u)) & 1023u);
+// -------------------------------------------------------------- dO, dz
+// Element-wise: dO = dO' G, dz = dO' O G (1 - G), and the per-CTA db_pw
+// partials.  Thread = (pixel slot sl, channel octet k): the octet stays the
+// thread's for the whole grid-stride walk over the pixels (pixel
+// (n gridDim + blockIdx) slots + sl), so its eight db_pw sums run in a fixed
+// order; consecutive threads read consecutive 16-byte octets of one pixel,
+// and kDzBatch pixels' loads are in flight before any is used.  A plain
+// stream: no shared-memory tile, no tensor-core step (dy is the next
+// kernel's).
+// grid p.grid, block kDzEwThreads.
+__global__ void __launch_bounds__(kDzEwThreads) cla_bwd_dz_kernel(const ClaBwdParams p) {
+  __shared__ float red[8 * kDzEwThreads];   // [slot][C] db_pw partials
   const int C = p.C;
-  uint8_t* sB = base;                                   // W_pw^T bf16 [N = c][K = o]
-  uint8_t* sA0 = base + 2ull * C * C;                   // dz bf16 [M = 128 pixels][K = o], x2
-  float* red = reinterpret_cast<float*>(sA0 + 2ull * 256 * C);   // [slot][C] db_pw partials
-  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 8 * kDzThreads);   // [2]
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    *abort_flag = 0;
-    fence_mbarrier_init();
-  }
-  // B(n = c, k = o) = W_pw[o][c]: dy[p][c] = sum_o dz[p][o] W_pw[o][c]
-  for (int i = threadIdx.x; i < C * C / 2; i += blockDim.x) {
-    const int o = (2 * i) / C, c = (2 * i) % C;
-    const float2 w = *reinterpret_cast<const float2*>(p.w_pw + static_cast<size_t>(o) * C + c);
-    *reinterpret_cast<__nv_bfloat16*>(sB + cla_kmajor_offset(c, o, C)) = __float2bfloat16_rn(w.x);
-    *reinterpret_cast<__nv_bfloat16*>(sB + cla_kmajor_offset(c + 1, o, C)) =
-        __float2bfloat16_rn(w.y);
-  }
-  fence_proxy_async_smem();
-  if (warp == 0) {
-    tmem_alloc(tbase, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tbase;
-  const uint32_t idesc = make_idesc_bf16(128, C, false, false);
-  const uint64_t bdesc = make_sdesc(smem_u32(sB), 128, 16 * C, kLayoutNone);
-  // element-wise part: thread = (pixel slot sl, channel octet k); slots
-  // take pixels sl, sl + slots, ...; consecutive threads read consecutive
-  // 16-byte octets of one pixel
-  const int octets = C / 8, slots = kDzThreads / octets;
+  const int octets = C / 8, slots = kDzEwThreads / octets;
   const int sl = threadIdx.x / octets, k = threadIdx.x % octets;
   const bool act = sl < slots;
+  const size_t n_pix = static_cast<size_t>(p.B) * p.H * p.W;
+  const size_t step = static_cast<size_t>(gridDim.x) * slots;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // db_pw, channels 8k..8k+7
-  const int G = gridDim.x;
-  const int my_tiles = (p.n_tiles - static_cast<int>(blockIdx.x) + G - 1) / G;
-  // dy of tile n (accumulator n % 2) to the workspace: warp w reads TMEM
-  // lanes 32 (w % 4).. (pixels), columns 32 (w / 4) + 128 i
-  auto drain_dy = [&](int n) -> bool {
-    bool ok = mbar_wait(&bar[n & 1], (n >> 1) & 1, abort_flag, p.wait_limit_ns, SITE_CLA);
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    if (!ok) return false;
-    int b, i0, j0;
-    cla_tile(p, static_cast<int>(blockIdx.x) + n * G, b, i0, j0);
-    const int q = warp & 3, slot = warp >> 2;
-    const int r = q * 32 + lane;
-    const size_t pix = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15));
-    __nv_bfloat16* dst = p.dy + pix * C;
-    const uint32_t taddr = tmem + (n & 1) * 256 + (static_cast<uint32_t>(q * 32) << 16);
-    for (int c0 = 32 * slot; c0 < C; c0 += 32 * (kDzThreads / 128)) {
-      uint32_t v[32];
-      tmem_ld_x32(taddr + c0, v);
-      tmem_wait_ld();
-      reg_fence_x32(v);
-      if (!rib_guard(pix * C + c0 + 31, cla_elems(p), G_CLA_OUT)) continue;
-      uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+  for (size_t p0 = static_cast<size_t>(blockIdx.x) * slots + sl; act && p0 < n_pix;
+       p0 += kDzBatch * step) {
+    uint4 dgv[kDzBatch], ov[kDzBatch], gv[kDzBatch];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        d4[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                           pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                           pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                           pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-    }
-    return true;
-  };
-  bool ok = true;
-  int n_mma = 0;
-  for (int n = 0; n < my_tiles; ++n) {
-    int b, i0, j0;
-    cla_tile(p, static_cast<int>(blockIdx.x) + n * G, b, i0, j0);
-    uint8_t* sA = sA0 + (n & 1) * 256ull * C;   // last read by tile n - 2's MMAs, drained
-    for (int r0 = sl; ok && act && r0 < 128; r0 += kDzBatch * slots) {
-      uint4 dgv[kDzBatch], ov[kDzBatch], gv[kDzBatch];
-#pragma unroll
-      for (int e = 0; e < kDzBatch; ++e) {
-        const int r = r0 + e * slots;
-        if (r < 128) {
-          const size_t off = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
-          if (!rib_guard(off + 7, cla_elems(p), G_CLA_IN)) {
-            dgv[e] = ov[e] = gv[e] = make_uint4(0, 0, 0, 0);
-            continue;
-          }
-          dgv[e] = ldg_nc_v4(p.dout_g + off);
-          ov[e] = ldg_nc_v4(p.out + off);
-          gv[e] = ldg_nc_v4(p.gate + off);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < kDzBatch; ++e) {
-        const int r = r0 + e * slots;
-        if (r >= 128) continue;
-        const size_t off = cla_pix(p, b, i0 + (r >> 4), j0 + (r & 15)) * C + 8 * k;
-        const uint32_t dw[4] = {dgv[e].x, dgv[e].y, dgv[e].z, dgv[e].w};
-        const uint32_t ow[4] = {ov[e].x, ov[e].y, ov[e].z, ov[e].w};
-        const uint32_t gw[4] = {gv[e].x, gv[e].y, gv[e].z, gv[e].w};
-        uint32_t dov[4], zv[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float2 dg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw[h]));
-          const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[h]));
-          const float2 gt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[h]));
-          const float z0 = dg.x * o.x * gt.x * (1.f - gt.x), z1 = dg.y * o.y * gt.y * (1.f - gt.y);
-          dov[h] = pack_bf16x2(dg.x * gt.x, dg.y * gt.y);
-          zv[h] = pack_bf16x2(z0, z1);
-          acc[2 * h] += z0;
-          acc[2 * h + 1] += z1;
-        }
-        const uint4 z4 = make_uint4(zv[0], zv[1], zv[2], zv[3]);
-        if (rib_guard(off + 7, cla_elems(p), G_CLA_OUT)) {
-          *reinterpret_cast<uint4*>(p.dout + off) = make_uint4(dov[0], dov[1], dov[2], dov[3]);
-          *reinterpret_cast<uint4*>(p.dz + off) = z4;
-        }
-        *reinterpret_cast<uint4*>(sA + cla_kmajor_offset(r, 8 * k, C)) = z4;
+    for (int e = 0; e < kDzBatch; ++e) {
+      const size_t pix = p0 + e * step;
+      const size_t off = pix * C + 8 * k;
+      if (pix < n_pix && rib_guard(off + 7, cla_elems(p), G_CLA_IN)) {
+        dgv[e] = ldg_nc_v4(p.dout_g + off);
+        ov[e] = ldg_nc_v4(p.out + off);
+        gv[e] = ldg_nc_v4(p.gate + off);
+      } else {
+        dgv[e] = ov[e] = gv[e] = make_uint4(0, 0, 0, 0);
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-    if (!ok) break;
-    // ---- dy = dz W_pw  (M = 128 pixels, N = C, K = C) into accumulator n % 2
-    if (warp == 0) {
-      const uint64_t adesc = make_sdesc(smem_u32(sA), 128, 16 * C, kLayoutNone);
-      for (int ks = 0; ks < C / 16; ++ks)
-        umma_ss_elect(tmem + (n & 1) * 256, adesc + ks * 16, bdesc + ks * 16, idesc,
-                      ks > 0 ? 1u : 0u);
-      umma_commit_elect(&bar[n & 1]);
+#pragma unroll
+    for (int e = 0; e < kDzBatch; ++e) {
+      const size_t pix = p0 + e * step;
+      if (pix >= n_pix) continue;
+      const size_t off = pix * C + 8 * k;
+      const uint32_t dw[4] = {dgv[e].x, dgv[e].y, dgv[e].z, dgv[e].w};
+      const uint32_t ow[4] = {ov[e].x, ov[e].y, ov[e].z, ov[e].w};
+      const uint32_t gw[4] = {gv[e].x, gv[e].y, gv[e].z, gv[e].w};
+      uint32_t dov[4], zv[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 dg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw[h]));
+        const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[h]));
+        const float2 gt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[h]));
+        const float z0 = dg.x * o.x * gt.x * (1.f - gt.x), z1 = dg.y * o.y * gt.y * (1.f - gt.y);
+        dov[h] = pack_bf16x2(dg.x * gt.x, dg.y * gt.y);
+        zv[h] = pack_bf16x2(z0, z1);
+        acc[2 * h] += z0;
+        acc[2 * h + 1] += z1;
+      }
+      if (rib_guard(off + 7, cla_elems(p), G_CLA_OUT)) {
+        *reinterpret_cast<uint4*>(p.dout + off) = make_uint4(dov[0], dov[1], dov[2], dov[3]);
+        *reinterpret_cast<uint4*>(p.dz + off) = make_uint4(zv[0], zv[1], zv[2], zv[3]);
+      }
     }
-    ++n_mma;
-    // tile n - 1's dy, whose MMAs ran during this tile's element-wise part
-    if (n >= 1) ok = drain_dy(n - 1);
-    tc_fence_before();
-    ok = __syncthreads_and(ok);   // accumulator (n - 1) % 2 and dz tile (n - 1) % 2 are free
-    tc_fence_after();
-    if (!ok) break;
-  }
-  if (ok && n_mma > 0) ok = drain_dy(n_mma - 1);
-  ok = __syncthreads_and(ok);
-  if (!ok && warp == 0 && n_mma > 0) {
-    // the last tile's MMAs (and every earlier one) land before the CTA exits
-    volatile int no_abort = 0;
-    mbar_wait(&bar[(n_mma - 1) & 1], ((n_mma - 1) >> 1) & 1, &no_abort, 200ull * 1000ull * 1000ull,
-              SITE_CLA);
   }
   // db_pw partial of this CTA: the slots' sums, added in slot order
   // (thread (sl, k) holds channels 8k..8k+7 at red[sl * C + 8k + e] = red[8 tid + e])
@@ -253,9 +152,230 @@ __global__ void __launch_bounds__(kDzThreads, 1) cla_bwd_dz_kernel(const ClaBwdP
                   G_CLA_PART))
       p.part_dbpw[static_cast<size_t>(blockIdx.x) * C + c] = s;
   }
+}
+
+// -------------------------------------------------------------- dy
+// dy = dz W_pw on tiles of 8 x 16 pixels (M = 128 pixels, N = C, K = C),
+// warp-specialised and pipelined:
+//   warp 8 (lane 0)  TMA: the dz tile, one 64-channel x 16 x 8 box per
+//                    chunk with the 128-byte swizzle (rows = pixels, the
+//                    canonical K-major A layout), into a kDyStages ring
+//   warp 9           MMAs through an elected lane: C / 16 K-steps into one
+//                    of two TMEM accumulators, B = W_pw^T resident in shared
+//                    memory, K-major with the 128-byte swizzle (64-channel
+//                    chunks of C rows; with no swizzle the tensor core's
+//                    shared-memory reads conflict and the MMAs run far
+//                    slower)
+//   warps 0-7        epilogue: TMEM lanes (pixels) -> bf16 -> a staging tile
+//                    in shared memory (the same swizzled layout) -> one TMA
+//                    store per 64-channel chunk, so dy leaves as whole
+//                    16-pixel rows (6 KB runs); warp w takes lane quarter
+//                    w % 4 and every other 32-column chunk from 32 (w / 4)
+//                    and frees the accumulator once its TMEM loads are done
+// Tile n's MMAs run while the epilogue drains tile n - 1 and the TMA loads
+// tile n + 1 and on.
+constexpr int kDyThreads = 320;
+constexpr int kDyStages = 2;
+constexpr uint32_t kDyChunk = 128u * 128u;   // one 64-channel chunk of a 128-pixel tile
+__host__ __device__ __forceinline__ size_t cla_dy_smem_bytes(int C) {
+  const size_t chunks = (C + 63) / 64;
+  return 128ull * C * chunks + (kDyStages + 1) * chunks * kDyChunk + 256 + 1024;
+}
+
+// grid p.grid, block kDyThreads, dynamic smem cla_dy_smem_bytes(C).
+// tm_dz: dz [B][H][W][C] (workspace), boxes of 64 channels x 16 x 8, 128-byte
+// swizzle; tm_dy: dy (workspace), the same boxes.
+constexpr int kDyEpiBar = 1;   // named barrier of the eight epilogue warps
+__global__ void __launch_bounds__(kDyThreads, 1)
+    cla_bwd_dy_kernel(const __grid_constant__ CUtensorMap tm_dz,
+                      const __grid_constant__ CUtensorMap tm_dy, const ClaBwdParams p) {
+  extern __shared__ uint8_t dy_raw[];
+  uint8_t* base = dy_raw + ((1024u - (smem_u32(dy_raw) & 1023u)) & 1023u);
+  const int C = p.C, chunks = (C + 63) / 64;
+  const uint32_t stage_bytes = static_cast<uint32_t>(chunks) * kDyChunk;
+  uint8_t* sA0 = base;                                              // dz stages (1024-aligned)
+  uint8_t* sY = base + kDyStages * stage_bytes;                     // dy staging tile
+  uint8_t* sB = sY + stage_bytes;                                   // W_pw^T [N = c][K = o]
+  const uint32_t b_chunk = static_cast<uint32_t>(C) * 128u;        // one 64-channel K chunk of B
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + static_cast<size_t>(b_chunk) * chunks);
+  uint64_t* empty = full + kDyStages;                               // [kDyStages]
+  uint64_t* acc_full = empty + kDyStages;                           // [2]
+  uint64_t* acc_free = acc_full + 2;                                // [2]
+  uint64_t* drain = acc_free + 2;
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
+  volatile int* epi_ok = abort_flag + 1;   // [8]: each epilogue warp's status, per tile
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int my_tiles = (p.n_tiles - static_cast<int>(blockIdx.x) + G - 1) / G;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDyStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_free[i], 8);   // the eight epilogue warps
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  // B(n = c, k = o) = W_pw[o][c]: dy[p][c] = sum_o dz[p][o] W_pw[o][c].
+  // Element (c, o) sits in K chunk o / 64, row c, 16-byte granule
+  // ((o % 64) / 8) ^ (c % 8) of the row's 128 bytes.
+  // Pair i is W_pw[2i], W_pw[2i + 1]; eight pairs' loads are issued before
+  // any store, so the fill costs a few memory latencies, not one per pair.
+  const int n_pairs = C * C / 2;
+  for (int i0 = threadIdx.x; i0 < n_pairs; i0 += 8 * blockDim.x) {
+    float2 wv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * static_cast<int>(blockDim.x);
+      wv[e] = i < n_pairs ? __ldg(reinterpret_cast<const float2*>(p.w_pw) + i)
+                          : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * static_cast<int>(blockDim.x);
+      if (i >= n_pairs) break;
+      const int o = (2 * i) / C, c = (2 * i) % C;
+      const uint32_t ko = static_cast<uint32_t>(o & 63) * 2;   // byte in the unswizzled row
+      const uint32_t g = static_cast<uint32_t>(o >> 6) * b_chunk;
+      *reinterpret_cast<__nv_bfloat16*>(sB + g + c * 128 + (ko ^ ((c & 7) << 4))) =
+          __float2bfloat16_rn(wv[e].x);
+      *reinterpret_cast<__nv_bfloat16*>(sB + g + (c + 1) * 128 + (ko ^ (((c + 1) & 7) << 4))) =
+          __float2bfloat16_rn(wv[e].y);
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 9) {
+    tmem_alloc(tbase, 512);
+    tmem_relinquish();
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  tc_fence_after();
+  const uint32_t tmem = *tbase;
+  const uint64_t lim = p.wait_limit_ns;
+  if (warp == 8) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      for (int n = 0; ok && n < my_tiles; ++n) {
+        const int s = n % kDyStages;
+        if (n >= kDyStages &&
+            !(ok = mbar_wait(&empty[s], ((n - kDyStages) / kDyStages) & 1, abort_flag, lim,
+                             SITE_CLA)))
+          break;
+        int b, i0, j0;
+        cla_tile(p, static_cast<int>(blockIdx.x) + n * G, b, i0, j0);
+        mbar_arrive_expect_tx(&full[s], stage_bytes);
+        for (int g = 0; g < chunks; ++g)
+          tma_load_4d(sA0 + s * stage_bytes + g * kDyChunk, &tm_dz, &full[s], 64 * g, j0, i0, b);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // the loads still in flight land before the CTA exits
+        volatile int no_abort = 0;
+        for (int n = max(0, issued - kDyStages); n < issued; ++n)
+          mbar_wait(&full[n % kDyStages], (n / kDyStages) & 1, &no_abort, 200000000ull, SITE_CLA);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------ MMA issue
+    const uint32_t idesc = make_idesc_bf16(128, C, false, false);
+    const uint32_t b0 = smem_u32(sB);
+    bool ok = true;
+    for (int n = 0; ok && n < my_tiles; ++n) {
+      const int s = n % kDyStages, a = n & 1;
+      ok = warp_wait(&full[s], (n / kDyStages) & 1, abort_flag, lim, SITE_CLA) &&
+           (n < 2 || warp_wait(&acc_free[a], ((n - 2) >> 1) & 1, abort_flag, lim, SITE_CLA));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sA0 + s * stage_bytes);
+      for (int ks = 0; ks < C / 16; ++ks) {
+        // K-step ks: channels 16 ks.. = chunk ks / 4, 32 (ks % 4) bytes into
+        // its rows, for both operands
+        const uint64_t adesc =
+            make_sdesc(a0 + (ks >> 2) * kDyChunk, 16, 1024, kLayoutSW128) + (ks & 3) * 2;
+        const uint64_t bdesc =
+            make_sdesc(b0 + (ks >> 2) * b_chunk, 16, 1024, kLayoutSW128) + (ks & 3) * 2;
+        umma_ss_elect(tmem + a * 256, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+      }
+      umma_commit_elect(&empty[s]);
+      umma_commit_elect(&acc_full[a]);
+    }
+    // every MMA issued above completes before the tensor memory is freed
+    umma_commit_elect(drain);
+    volatile int no_abort = 0;
+    mbar_wait(drain, 0, &no_abort, 200000000ull, SITE_CLA);
+  } else {
+    // ------------------------------------------------ epilogue (warps 0-7)
+    const int q = warp & 3, h = warp >> 2;
+    const int r = q * 32 + lane;   // tile row = pixel (i0 + r / 16, j0 + r % 16)
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const bool leader = warp == 0 && lane == 0;
+    for (int n = 0; n < my_tiles; ++n) {
+      const int a = n & 1;
+      const bool got = warp_wait(&acc_full[a], (n >> 1) & 1, abort_flag, lim, SITE_CLA);
+      // this warp's chunks: columns 32 h + 64 j, j < 3 (C <= 192)
+      uint32_t v[3][32];
+      if (got) {
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+          if (32 * h + 64 * j < C) tmem_ld_x32(tmem + a * 256 + lane_off + 32 * h + 64 * j, v[j]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_free[a]);   // the accumulator is in registers
+      }
+      // the staging tile is free once the previous tile's stores have read it
+      if (lane == 0) epi_ok[warp] = got ? 1 : 0;
+      if (leader) tma_store_wait_read_all();
+      named_bar_sync(kDyEpiBar, 256);
+      // one decision for all eight warps, from flags written before the barrier
+      const bool all_ok = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3] && epi_ok[4] &&
+                          epi_ok[5] && epi_ok[6] && epi_ok[7];
+      if (!all_ok) break;
+      {
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int c0 = 32 * h + 64 * j;
+          if (c0 >= C) continue;
+          reg_fence_x32(v[j]);
+          // row r of chunk c0 / 64: 16-byte granules (c0 % 64) / 8 + t, XOR r % 8
+          uint8_t* row = sY + (c0 >> 6) * kDyChunk + r * 128;
+          const int g0 = (c0 & 63) >> 3;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t* w = &v[j][8 * t];
+            *reinterpret_cast<uint4*>(row + (((g0 + t) ^ (r & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                           pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                           pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                           pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7])));
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(kDyEpiBar, 256);
+      if (leader) {
+        int b, i0, j0;
+        cla_tile(p, static_cast<int>(blockIdx.x) + n * G, b, i0, j0);
+        for (int g = 0; g < chunks; ++g)
+          tma_store_4d(&tm_dy, sY + g * kDyChunk, 64 * g, j0, i0, b);
+        tma_store_commit();
+      }
+    }
+    // the stores are complete before the kernel's work is considered done
+    if (leader) tma_store_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -142,7 +142,7 @@ int map_pixel_f32(CUtensorMap* m, const void* base, int B, int heads, int H, int
 // ---------------------------------------------------------------- tracing
 enum KernelId {
   K_POS, K_FWD, K_BWD_PRE, K_BWD, K_DQ_FIN, K_POSGRAD, K_MLP_PART, K_MLP_RED, K_COPY, K_DEBUG,
-  K_CLA, K_CLA_DZ, K_CLA_DWPW, K_CLA_DX, K_CLA_RED, K_BWD_PERSIST, K_FWD_TF32, K_COUNT
+  K_CLA, K_CLA_DZ, K_CLA_DWPW, K_CLA_DX, K_CLA_RED, K_BWD_PERSIST, K_FWD_TF32, K_CLA_DY, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "pos_tokens_kernel",   "attn_fwd_kernel",        "bwd_preprocess_kernel",
@@ -150,7 +150,7 @@ const char* const kKernelNames[K_COUNT] = {
     "mlp_bwd_partial_kernel", "mlp_bwd_reduce_kernel", "window_copy_kernel",
     "debug_wait_kernel",   "cla_gate_kernel",        "cla_bwd_dz_kernel",
     "cla_bwd_dwpw_kernel", "cla_bwd_dx_kernel",      "cla_bwd_reduce_kernel",
-    "attn_bwd_persistent_kernel", "attn_fwd_tf32_kernel"};
+    "attn_bwd_persistent_kernel", "attn_fwd_tf32_kernel", "cla_bwd_dy_kernel"};
 
 struct TraceRec {
   int id;
@@ -398,7 +398,7 @@ struct ClaBwdLayout {
 
 int cla_check(int B, int H, int W, int C) {
   if (B < 0 || H <= 0 || W <= 0 || C <= 0) return RIB_ERR_ARG;
-  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u || cla_dz_smem_bytes(C) > 227u * 1024u ||
+  if (C % 32 != 0 || cla_smem_bytes(C) > 227u * 1024u || cla_dy_smem_bytes(C) > 227u * 1024u ||
       cla_dwpw_smem_bytes(C) > 227u * 1024u)
     return RIB_ERR_UNSUPPORTED;
   if (H % 8 != 0 || W % 16 != 0) return RIB_ERR_SHAPE;
@@ -908,8 +908,9 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
     if (rc) return rc;
   }
   // x again with 10 x 10 boxes (the halo of an 8 x 8 tile), and dz
-  // (workspace) with 8 x 8 boxes in the 128-byte swizzle, for the dW_pw kernel
-  CUtensorMap tm_x10, tm_dz;
+  // (workspace) with 8 x 8 boxes in the 128-byte swizzle, for the dW_pw
+  // kernel; dz and dy with 16 x 8 boxes (a 128-pixel tile), for the dy kernel
+  CUtensorMap tm_x10, tm_dz, tm_dz16, tm_dy16;
   {
     const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)H, (uint64_t)B};
     const uint64_t strides[3] = {2ull * C, 2ull * C * W, 2ull * C * W * H};
@@ -921,15 +922,27 @@ int rib_cla_bwd(const void* x, int B, int H, int W, int C, const float* w_dw, co
     rc = make_map(&tm_dz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.dz, dims, strides, box8,
                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
+    const uint32_t box16[4] = {64, 16, 8, 1};
+    rc = make_map(&tm_dz16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.dz, dims, strides, box16,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    rc = make_map(&tm_dy16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.dy, dims, strides, box16,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
   }
-  const size_t smem_dz = cla_dz_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
+  const size_t smem_dy = cla_dy_smem_bytes(C), smem_dw = cla_dwpw_smem_bytes(C);
   const size_t smem_dx = cla_dx_smem_bytes();
-  if ((rc = set_smem(cla_bwd_dz_kernel, smem_dz))) return rc;
+  if ((rc = set_smem(cla_bwd_dy_kernel, smem_dy))) return rc;
   if ((rc = set_smem(cla_bwd_dwpw_kernel, smem_dw))) return rc;
   if ((rc = set_smem(cla_bwd_dx_kernel, smem_dx))) return rc;
   {
     TraceScope ts(K_CLA_DZ, st);
-    cla_bwd_dz_kernel<<<L.grid, kDzThreads, smem_dz, st>>>(p);
+    cla_bwd_dz_kernel<<<L.grid, kDzEwThreads, 0, st>>>(p);
+    if ((rc = launch_status())) return rc;
+  }
+  {
+    TraceScope ts(K_CLA_DY, st);
+    cla_bwd_dy_kernel<<<L.grid, kDyThreads, smem_dy, st>>>(tm_dz16, tm_dy16, p);
     if ((rc = launch_status())) return rc;
   }
   {
