@@ -54,3 +54,29 @@ def test_backward_repeatability(name, B, bwd_kernel):
         same = torch.equal(g["dqkv"][:, :, :, 0], g0["dqkv"][:, :, :, 0])
         print(f"{name}: dQc bit-identical across calls: {same}")
     assert_all(checks)
+
+
+def test_backward_dqkv_at_16_byte_offset():
+    """dqkv at an address 16- but not 32-byte aligned (the smallest the ABI
+    accepts): the dQ write takes its 16-byte store path and the gradients
+    match the call with an aligned dqkv (dKc, dV bit-identical; dQc within
+    the call-to-call bound of its reduction order)."""
+    w = I.get_workload("w32")
+    inp = I.make_layer_inputs(w, 0, strong=True)
+    M, s = w.windows[0], w.shifts[0]
+    qkv, dout = inp["qkv"][:1].cuda(), inp["dout"][:1].cuda()
+    mlp = R.PositionMLP.from_params(inp["freqs"], inp["mlp_q"], inp["mlp_k"], w.heads, w.rank)
+    _, _, q16, k16 = R.rib_pos_tokens(mlp, M)
+    out, lse = R.rib_window_attn_fwd(qkv, M, s, q16, k16)
+    g0 = R.rib_window_attn_bwd(qkv, out, dout, lse, M, s, q16, k16)
+    buf = torch.empty(qkv.numel() + 64, dtype=torch.bfloat16, device="cuda")
+    off = 8 if buf.data_ptr() % 32 == 0 else 24   # 16 bytes past a 32-byte boundary
+    dq = buf[off:off + qkv.numel()].view(qkv.shape)
+    assert dq.data_ptr() % 32 == 16
+    g1 = R.rib_window_attn_bwd(qkv, out, dout, lse, M, s, q16, k16, dqkv=dq,
+                               dqp=torch.empty_like(g0["dqp"]), dkp=torch.empty_like(g0["dkp"]))
+    torch.cuda.synchronize()
+    assert R.rib_last_status()[0] == 0
+    assert torch.equal(g1["dqkv"][:, :, :, 1:], g0["dqkv"][:, :, :, 1:]), "dKc / dV"
+    assert_all([check_close(to_np(g1["dqkv"][:, :, :, 0]), to_np(g0["dqkv"][:, :, :, 0]),
+                            "dQc, 16-byte-offset dqkv against aligned")])

@@ -626,6 +626,7 @@ struct BwdAuxParams {
   const float* dkp_part;
   size_t dq_acc_floats;
   __nv_bfloat16* dqkv;
+  int dq_v8;        // dqkv is 32-byte aligned: dq_finalize writes whole 32-byte sectors
   float* dqp;       // [heads][M][M][rank]
   float* dkp;
   int pg_chunks;    // posgrad_reduce: warps sharing one group of outputs (1, 2, 4, 8, 16)
@@ -695,11 +696,17 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(const BwdAuxParams p) 
       !rib_guard((pix * 3 * p.heads + u.head) * 32 + 31,
                  static_cast<size_t>(p.B) * p.H * p.W * 3 * p.heads * 32, G_DQ_FIN_OUT))
     return;
+  uint32_t w[16];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float* c = src + 8 * q * 128;
-    dst[q] = make_uint4(pack_bf16x2(c[0] * t, c[128] * t), pack_bf16x2(c[256] * t, c[384] * t),
-                        pack_bf16x2(c[512] * t, c[640] * t), pack_bf16x2(c[768] * t, c[896] * t));
+  for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(src[2 * e * 128] * t, src[(2 * e + 1) * 128] * t);
+  if (p.dq_v8) {
+    // two 32-byte stores: each a whole sector of the row's 64 bytes (16-byte
+    // stores from 32 different rows would half-fill a sector each)
+    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st_global_v8(dst + 2, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
 }
 

@@ -1033,6 +1033,7 @@ static int attn_bwd_launch(const void* qkv, const void* out, const void* dout,
   a.dkp_part = reinterpret_cast<const float*>(wsb + ws.dkp_part);
   a.dq_acc_floats = (size_t)B * H * W * heads * 48;
   a.dqkv = static_cast<__nv_bfloat16*>(dqkv);
+  a.dq_v8 = (reinterpret_cast<uintptr_t>(dqkv) & 31u) == 0 ? 1 : 0;
   a.dqp = dqp;
   a.dkp = dkp;
 
