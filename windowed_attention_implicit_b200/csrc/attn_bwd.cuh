@@ -98,6 +98,7 @@ struct BwdParams {
   float scale;       // tau
   float scale_log2;  // tau * log2(e)
   __nv_bfloat16* dqkv;
+  int dqkv_v8;       // dqkv is 32-byte aligned: rows go out as whole 32-byte sectors
   float* dq_acc;     // [units][n_tiles][48][128]  (channel-major per tile)
   float* dkp_part;   // [units][n_tiles][128][16]
   int n_items;       // persistent form only: work items (unit, key tile), units * n_tiles
@@ -145,6 +146,22 @@ constexpr uint32_t kIdescBQ = make_idesc_bf16(128, 48, true, true);      // dQ_a
 // every 2048 B.
 __device__ __forceinline__ uint32_t ds_offset(int k, int q) {
   return static_cast<uint32_t>((q >> 3) * 2048 + (k >> 3) * 128 + (k & 7) * 16 + (q & 7) * 2);
+}
+
+// One thread's 64-byte row (a key's 32 bf16 gradient channels, or its 16
+// fp32 dKp partials): with v8 (a 32-byte aligned row) two whole 32-byte
+// sectors, else four 16-byte stores.  A warp's 32 rows lie far apart, so a
+// 16-byte store per lane half-fills 32 sectors at once.
+__device__ __forceinline__ void store_row64(void* dst, const uint32_t (&w)[16], bool v8) {
+  if (v8) {
+    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st_global_v8(static_cast<uint8_t*>(dst) + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14],
+                 w[15]);
+  } else {
+    uint4* d = static_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
 }
 
 __device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
@@ -497,46 +514,37 @@ __device__ __forceinline__ void bwd_compute(BwdSmem& sm, uint32_t tmem, const Bw
     tmem_ld_x32(tmem + lane_off + kBColDV, r);
     tmem_wait_ld();
     reg_fence_x32(r);
-    uint4* dst = reinterpret_cast<uint4*>(base + (2 * p.heads + u.head) * 32);
+    uint32_t w[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (rib_guard(pix * 3 * p.heads * 32 + (2 * p.heads + u.head) * 32 + 8 * q + 7, n_dqkv,
-                    G_BWD_DQKV))
-        dst[q] = make_uint4(
-          pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1])),
-          pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-          pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-          pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+    for (int e = 0; e < 16; ++e)
+      w[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+    if (rib_guard(pix * 3 * p.heads * 32 + (2 * p.heads + u.head) * 32 + 31, n_dqkv, G_BWD_DQKV))
+      store_row64(base + (2 * p.heads + u.head) * 32, w, p.dqkv_v8 != 0);
     if (pos) {
       uint32_t r16[16];
       tmem_ld_x16(tmem + lane_off + kBColDK + 32, r16);
       tmem_wait_ld();
       reg_fence_x16(r16);
       const size_t kp0 = ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + key) * 16;
-      float4* dk = reinterpret_cast<float4*>(p.dkp_part + kp0);
       const float t = p.scale;
+      uint32_t w16[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (rib_guard(kp0 + 4 * q + 3, bwd_units(p) * p.n_tiles * 128 * 16, G_BWD_DKP_PART))
-          dk[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
-                            __uint_as_float(r16[4 * q + 2]) * t,
-                            __uint_as_float(r16[4 * q + 3]) * t);
+      for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(__uint_as_float(r16[e]) * t);
+      // the workspace partials are 256-byte aligned: always whole sectors
+      if (rib_guard(kp0 + 15, bwd_units(p) * p.n_tiles * 128 * 16, G_BWD_DKP_PART))
+        store_row64(p.dkp_part + kp0, w16, true);
     }
   } else {  // dKc
     tmem_ld_x32(tmem + lane_off + kBColDK, r);
     tmem_wait_ld();
     reg_fence_x32(r);
     const float t = p.scale;
-    uint4* dst = reinterpret_cast<uint4*>(base + (p.heads + u.head) * 32);
+    uint32_t w[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (rib_guard(pix * 3 * p.heads * 32 + (p.heads + u.head) * 32 + 8 * q + 7, n_dqkv,
-                    G_BWD_DQKV))
-        dst[q] = make_uint4(
-          pack_bf16x2(__uint_as_float(r[8 * q + 0]) * t, __uint_as_float(r[8 * q + 1]) * t),
-          pack_bf16x2(__uint_as_float(r[8 * q + 2]) * t, __uint_as_float(r[8 * q + 3]) * t),
-          pack_bf16x2(__uint_as_float(r[8 * q + 4]) * t, __uint_as_float(r[8 * q + 5]) * t),
-          pack_bf16x2(__uint_as_float(r[8 * q + 6]) * t, __uint_as_float(r[8 * q + 7]) * t));
+    for (int e = 0; e < 16; ++e)
+      w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * t, __uint_as_float(r[2 * e + 1]) * t);
+    if (rib_guard(pix * 3 * p.heads * 32 + (p.heads + u.head) * 32 + 31, n_dqkv, G_BWD_DQKV))
+      store_row64(base + (p.heads + u.head) * 32, w, p.dqkv_v8 != 0);
   }
 }
 

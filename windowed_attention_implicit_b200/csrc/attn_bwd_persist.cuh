@@ -353,31 +353,25 @@ __device__ __forceinline__ void bwd_drain(BwdSmem& sm, uint32_t tmem, const BwdP
         tmem_wait_ld();
         reg_fence_x32(r32);
         const float f = a == 0 ? 1.f : t;
-        uint4* dst = reinterpret_cast<uint4*>(base + ((a == 0 ? 2 : 1) * p.heads + u.head) * 32);
+        uint32_t w[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (rib_guard(pix * 3 * p.heads * 32 + ((a == 0 ? 2 : 1) * p.heads + u.head) * 32 +
-                            8 * q + 7,
-                        static_cast<size_t>(p.B) * p.H * p.W * 3 * p.heads * 32, G_BWD_DQKV))
-            dst[q] = make_uint4(
-              pack_bf16x2(__uint_as_float(r32[8 * q + 0]) * f, __uint_as_float(r32[8 * q + 1]) * f),
-              pack_bf16x2(__uint_as_float(r32[8 * q + 2]) * f, __uint_as_float(r32[8 * q + 3]) * f),
-              pack_bf16x2(__uint_as_float(r32[8 * q + 4]) * f, __uint_as_float(r32[8 * q + 5]) * f),
-              pack_bf16x2(__uint_as_float(r32[8 * q + 6]) * f, __uint_as_float(r32[8 * q + 7]) * f));
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(r32[2 * e]) * f, __uint_as_float(r32[2 * e + 1]) * f);
+        if (rib_guard(pix * 3 * p.heads * 32 + ((a == 0 ? 2 : 1) * p.heads + u.head) * 32 + 31,
+                      static_cast<size_t>(p.B) * p.H * p.W * 3 * p.heads * 32, G_BWD_DQKV))
+          store_row64(base + ((a == 0 ? 2 : 1) * p.heads + u.head) * 32, w, p.dqkv_v8 != 0);
       }
       if (pos) {
         tmem_ld_x16(tmem + lane_off + kBColDK + 32, r16);
         tmem_wait_ld();
         reg_fence_x16(r16);
-        float4* dkp = reinterpret_cast<float4*>(
-            p.dkp_part + ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + row) * 16);
+        const size_t kp0 = ((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + row) * 16;
+        uint32_t w16[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (rib_guard(((static_cast<size_t>(unit) * p.n_tiles + kt) * 128 + row) * 16 + 4 * q + 3,
-                        bwd_units(p) * p.n_tiles * 128 * 16, G_BWD_DKP_PART))
-            dkp[q] = make_float4(__uint_as_float(r16[4 * q]) * t, __uint_as_float(r16[4 * q + 1]) * t,
-                               __uint_as_float(r16[4 * q + 2]) * t,
-                               __uint_as_float(r16[4 * q + 3]) * t);
+        for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(__uint_as_float(r16[e]) * t);
+        // the workspace partials are 256-byte aligned: always whole sectors
+        if (rib_guard(kp0 + 15, bwd_units(p) * p.n_tiles * 128 * 16, G_BWD_DKP_PART))
+          store_row64(p.dkp_part + kp0, w16, true);
       }
       // every read of the accumulators is complete: the next item may overwrite them
       tc_fence_before();

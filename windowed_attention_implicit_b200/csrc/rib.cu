@@ -1065,6 +1065,7 @@ static int attn_bwd_launch(const void* qkv, const void* out, const void* dout,
   p.scale = tau;
   p.scale_log2 = tau * 1.4426950408889634f;
   p.dqkv = a.dqkv;
+  p.dqkv_v8 = a.dq_v8;
   p.dq_acc = a.dq_acc;
   p.dkp_part = reinterpret_cast<float*>(wsb + ws.dkp_part);
   p.n_items = g.units * g.n_tiles;
