@@ -80,3 +80,41 @@ def test_backward_dqkv_at_16_byte_offset():
     assert torch.equal(g1["dqkv"][:, :, :, 1:], g0["dqkv"][:, :, :, 1:]), "dKc / dV"
     assert_all([check_close(to_np(g1["dqkv"][:, :, :, 0]), to_np(g0["dqkv"][:, :, :, 0]),
                             "dQc, 16-byte-offset dqkv against aligned")])
+
+
+def _offset_like(t):
+    """A tensor shaped like t whose data starts 16 bytes past a 32-byte boundary."""
+    n = t.numel()
+    buf = torch.empty(n + 64, dtype=t.dtype, device=t.device)
+    step = 16 // t.element_size()
+    off = step if buf.data_ptr() % 32 == 0 else 3 * step
+    v = buf[off:off + n].view(t.shape)
+    assert v.data_ptr() % 32 == 16
+    return v
+
+
+def test_forward_outputs_at_16_byte_offset():
+    """out and out_gated 16- but not 32-byte aligned: the epilogue takes its
+    16-byte store path; the results are bit-identical to aligned outputs."""
+    w = I.get_workload("w32")
+    inp = I.make_layer_inputs(w, 0, strong=True)
+    M, s = w.windows[0], w.shifts[0]
+    qkv = inp["qkv"][:1].cuda()
+    mlp = R.PositionMLP.from_params(inp["freqs"], inp["mlp_q"], inp["mlp_k"], w.heads, w.rank)
+    _, _, q16, k16 = R.rib_pos_tokens(mlp, M)
+    o0, l0 = R.rib_window_attn_fwd(qkv, M, s, q16, k16)
+    o1 = _offset_like(o0)
+    R.rib_window_attn_fwd(qkv, M, s, q16, k16, out=o1, lse=torch.empty_like(l0))
+    C = w.heads * w.head_dim
+    p = I.make_cla(C, 3)
+    cla = R.ClaGate.from_params(p.w_dw, p.b_dw, p.w_pw, p.b_pw)
+    x = I.make_features(1, w.height, w.width, C, 3).cuda()
+    gate = R.rib_cla_gate(x, cla)
+    _, og0, _ = R.rib_window_attn_fwd_cla(qkv, M, s, gate, q16, k16)
+    og1 = _offset_like(og0)
+    R.rib_window_attn_fwd_cla(qkv, M, s, gate, q16, k16, out=torch.empty_like(o0),
+                              out_gated=og1, lse=torch.empty_like(l0))
+    torch.cuda.synchronize()
+    assert R.rib_last_status()[0] == 0
+    assert torch.equal(o1, o0), "O at a 16-byte offset"
+    assert torch.equal(og1, og0), "O * G at a 16-byte offset"

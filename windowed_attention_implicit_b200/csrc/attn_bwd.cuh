@@ -148,22 +148,6 @@ __device__ __forceinline__ uint32_t ds_offset(int k, int q) {
   return static_cast<uint32_t>((q >> 3) * 2048 + (k >> 3) * 128 + (k & 7) * 16 + (q & 7) * 2);
 }
 
-// One thread's 64-byte row (a key's 32 bf16 gradient channels, or its 16
-// fp32 dKp partials): with v8 (a 32-byte aligned row) two whole 32-byte
-// sectors, else four 16-byte stores.  A warp's 32 rows lie far apart, so a
-// 16-byte store per lane half-fills 32 sectors at once.
-__device__ __forceinline__ void store_row64(void* dst, const uint32_t (&w)[16], bool v8) {
-  if (v8) {
-    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
-    st_global_v8(static_cast<uint8_t*>(dst) + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14],
-                 w[15]);
-  } else {
-    uint4* d = static_cast<uint4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-  }
-}
-
 __device__ __forceinline__ void bwd_producer(BwdSmem& sm, const CUtensorMap* tq,
                                              const CUtensorMap* tdo, const CUtensorMap* tqp,
                                              const CUtensorMap* tkp, const CUtensorMap* tlse2,

@@ -96,6 +96,7 @@ struct FwdParams {
   float* lse;
   const __nv_bfloat16* gate;   // CLA gate G [B][H][W][heads*32], or null
   __nv_bfloat16* out_gated;    // O * G, written when gate is set
+  int out_v8, gated_v8;        // out / out_gated 32-byte aligned: rows as whole sectors
   uint64_t wait_limit_ns;
 };
 
@@ -476,32 +477,26 @@ __device__ __forceinline__ bool fwd_softmax_item(FwdSmem& sm, uint32_t tmem, con
   const size_t pix = (static_cast<size_t>(u.b) * p.H + y) * p.W + x;
   const size_t row0 = (pix * p.heads + u.head) * 32;   // first of the row's 32 channels
   const size_t n_out = static_cast<size_t>(p.B) * p.H * p.W * p.heads * 32;
-  uint4* dst = reinterpret_cast<uint4*>(p.out + row0);
-  if (rib_guard(row0 + 31, n_out, G_FWD_OUT)) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-  }
+  if (rib_guard(row0 + 31, n_out, G_FWD_OUT)) store_row64(p.out + row0, pk, p.out_v8 != 0);
   if (p.gate != nullptr && rib_guard(row0 + 31, n_out, G_FWD_GATE)) {
     // convolutional local attention: O' = O * G at the same pixel and
     // channels (German summary, Methodik §B); O itself is kept for the
     // backward.  The product is formed from the fp32 O, then rounded.
     const uint4* g4 = reinterpret_cast<const uint4*>(p.gate + (pix * p.heads + u.head) * 32);
-    uint4* dg = reinterpret_cast<uint4*>(p.out_gated + (pix * p.heads + u.head) * 32);
+    uint32_t r16[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint4 gv = g4[q];
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-      uint32_t r4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[e]));
         const int c = 8 * q + 2 * e;
-        r4[e] = pack_bf16x2(__uint_as_float(o[c]) * inv * gf.x,
-                            __uint_as_float(o[c + 1]) * inv * gf.y);
+        r16[4 * q + e] = pack_bf16x2(__uint_as_float(o[c]) * inv * gf.x,
+                                     __uint_as_float(o[c + 1]) * inv * gf.y);
       }
-      dg[q] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
     }
+    store_row64(p.out_gated + (pix * p.heads + u.head) * 32, r16, p.gated_v8 != 0);
   }
   const size_t li_ = (static_cast<size_t>(u.b * p.heads + u.head) * p.H + y) * p.W + x;
   if (rib_guard(li_, static_cast<size_t>(p.B) * p.heads * p.H * p.W, G_FWD_LSE))

@@ -603,6 +603,22 @@ __device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a0, uint32_t a1
                : "memory");
 }
 
+// One thread's 64-byte row (32 bf16 channels of a token, or 16 fp32
+// values): with v8 (a 32-byte aligned row) two whole 32-byte sectors, else
+// four 16-byte stores.  When a warp's 32 rows lie far apart, a 16-byte
+// store per lane half-fills 32 sectors at once.
+__device__ __forceinline__ void store_row64(void* dst, const uint32_t (&w)[16], bool v8) {
+  if (v8) {
+    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st_global_v8(static_cast<uint8_t*>(dst) + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14],
+                 w[15]);
+  } else {
+    uint4* d = static_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a),
                "f"(b), "f"(c), "f"(d)

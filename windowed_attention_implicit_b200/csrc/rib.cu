@@ -704,6 +704,8 @@ static int attn_fwd_launch(const void* qkv, int B, int H, int W, int heads, int 
   p.lse = lse;
   p.gate = static_cast<const __nv_bfloat16*>(gate);
   p.out_gated = static_cast<__nv_bfloat16*>(out_gated);
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
+  p.gated_v8 = (reinterpret_cast<uintptr_t>(out_gated) & 31u) == 0 ? 1 : 0;
   p.wait_limit_ns = g_wait_limit_ns;
   auto* kern = p.region_mask ? attn_fwd_kernel<true> : attn_fwd_kernel<false>;
   if ((rc = set_smem(kern, kFwdSmemBytes))) return rc;
