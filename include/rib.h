@@ -27,7 +27,15 @@
  *   - Layouts are row-major, innermost index last.  bf16 = IEEE bfloat16
  *     stored as 16-bit words; conversion is round-to-nearest-even.
  *   - Device buffers must be 16-byte aligned (TMA); violations return
- *     RIB_ERR_ALIGN.
+ *     RIB_ERR_ALIGN.  Outputs that are also 32-byte aligned are written in
+ *     whole 32-byte sectors (faster; the values are the same).
+ *   - The work entry points make no synchronous CUDA call and allocate
+ *     nothing, so a sequence of them may be captured into a CUDA graph on
+ *     `stream` and replayed (the kernel parameters, tensor maps included,
+ *     are fixed at capture: replays read and write the same buffers).  Only
+ *     the status and debug queries (rib_last_status, rib_debug_guard_info)
+ *     synchronise the device; rib_pos_tokens_bwd_noalloc's first call on a
+ *     device must precede any capture.
  *
  * Notation: B batch, H x W feature map, M window side, N = M*M tokens per
  * window, nW = (H/M)(W/M) windows, h heads, d = 32 content head dim,
