@@ -209,25 +209,38 @@ def peaks():
             "source": "fallback"}
 
 
-def kernel_source_hash():
-    """Hash of the kernel sources, to tell whether stored ncu counters still
-    describe the kernels being timed."""
+# The source files a kernel is built from: its own header, the headers it
+# includes and the host file that launches it (grid, shared memory, tensor
+# maps).  A kernel not listed depends on every source.
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("attn_fwd.cuh", "geom.cuh", "ptx.cuh", "rib.cu"),
+    "attn_bwd_kernel": ("attn_bwd.cuh", "geom.cuh", "ptx.cuh", "rib.cu"),
+    "cla_gate_kernel": ("cla.cuh", "ptx.cuh", "rib.cu"),
+}
+
+
+def kernel_source_hash(kernel=None):
+    """Hash of the sources of `kernel` (all kernel sources when it is None or
+    not listed), to tell whether stored ncu counters still describe the
+    kernel being timed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "windowed_attention_implicit_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    names = KERNEL_SOURCES.get(kernel)
+    if names is None:
+        names = [f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh"))]
+    for f in sorted(names):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def stored_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it still
-    matches the current kernel sources; else None."""
+    matches the current sources of the kernel; else None."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("source_hash") != kernel_source_hash():
+    if d.get("source_hash") != kernel_source_hash(kernel):
         return None
     return d.get("dram_bytes_per_launch")
 

@@ -128,6 +128,35 @@ def test_stored_traffic_follows_the_kernel_sources(monkeypatch, tmp_path):
     assert bench.stored_traffic("k", "w") is None
 
 
+def test_stored_traffic_of_a_listed_kernel_follows_its_own_sources(monkeypatch, tmp_path):
+    csrc = tmp_path / "windowed_attention_implicit_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "a.cuh").write_text("// kernel a v1\n")
+    (csrc / "common.cuh").write_text("// shared v1\n")
+    (csrc / "b.cuh").write_text("// kernel b v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", {"ka": ("a.cuh", "common.cuh")})
+    h = bench.kernel_source_hash("ka")
+    assert h != bench.kernel_source_hash()          # a subset of the sources
+    rec = {"kernel": "ka", "workload": "w", "source_hash": h, "dram_bytes_per_launch": 99}
+    (tmp_path / "profiles" / "ka_w.traffic.json").write_text(json.dumps(rec))
+    assert bench.stored_traffic("ka", "w") == 99
+    (csrc / "b.cuh").write_text("// kernel b v2\n")   # another kernel's source
+    assert bench.stored_traffic("ka", "w") == 99
+    (csrc / "common.cuh").write_text("// shared v2\n")  # one of its own
+    assert bench.stored_traffic("ka", "w") is None
+
+
+def test_committed_traffic_records_match_the_current_sources():
+    """Every committed record was taken from the sources now in the tree
+    (a stale record is nulled by the bench; this keeps the committed ones
+    current)."""
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.traffic.json"))):
+        d = json.load(open(p))
+        assert d["source_hash"] == bench.kernel_source_hash(d["kernel"]), os.path.basename(p)
+
+
 def test_committed_traffic_records_are_well_formed():
     recs = sorted(glob.glob(os.path.join(ROOT, "profiles", "*.traffic.json")))
     assert recs

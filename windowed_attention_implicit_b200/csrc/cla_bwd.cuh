@@ -16,7 +16,7 @@
 //   cla_bwd_dz_kernel    dO, dz (to the workspace), db_pw partials: a plain
 //                        element-wise stream
 //   cla_bwd_dy_kernel    dy = dz W_pw on the tensor cores (tcgen05; dz tiles
-//                        by TMA through a 3-stage ring, W_pw^T resident in
+//                        by TMA through a 2-stage ring, W_pw^T resident in
 //                        shared memory, two TMEM accumulators)
 //   cla_bwd_dwpw_kernel  dW_pw partials = sum over the CTA's 8 x 8-pixel
 //                        tiles of dz^T y, y recomputed from x; dz by TMA,
