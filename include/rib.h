@@ -27,8 +27,9 @@
  *   - Layouts are row-major, innermost index last.  bf16 = IEEE bfloat16
  *     stored as 16-bit words; conversion is round-to-nearest-even.
  *   - Device buffers must be 16-byte aligned (TMA); violations return
- *     RIB_ERR_ALIGN.  Outputs that are also 32-byte aligned are written in
- *     whole 32-byte sectors (faster; the values are the same).
+ *     RIB_ERR_ALIGN.  The attention outputs (out, out_gated, dqkv) are
+ *     written in whole 32-byte sectors when they are also 32-byte aligned
+ *     (faster; the values are the same either way).
  *   - The work entry points make no synchronous CUDA call and allocate
  *     nothing, so a sequence of them may be captured into a CUDA graph on
  *     `stream` and replayed (the kernel parameters, tensor maps included,
