@@ -311,21 +311,25 @@ def config_sweep(I, R, dev, rank, world, timed, steps, warmup, peak, pk):
             # entry points only enqueue on the current stream, so the whole
             # step (every layer's position tokens, forward and backward) is
             # one graph launch, without the per-call host and launch costs
-            side = torch.cuda.Stream()
-            side.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(side):
-                train_step()
-            torch.cuda.current_stream().wait_stream(side)
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                train_step()
-            for _ in range(warmup):
-                graph.replay()
-            ms_g, _, _ = timed(graph.replay, steps)
-            ms_g /= steps
-            line.update({"step_graph_ms": ms_g,
-                         "step_graph_tflops": world * (f_fwd + f_bwd) / (ms_g * 1e-3) / 1e12})
-            del graph
+            try:
+                side = torch.cuda.Stream()
+                side.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(side):
+                    train_step()
+                torch.cuda.current_stream().wait_stream(side)
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    train_step()
+            except RuntimeError as e:   # reported, never fatal to the bench line
+                line["step_graph_error"] = str(e).splitlines()[0][:200]
+            else:
+                for _ in range(warmup):
+                    graph.replay()
+                ms_g, _, _ = timed(graph.replay, steps)
+                ms_g /= steps
+                line.update({"step_graph_ms": ms_g,
+                             "step_graph_tflops": world * (f_fwd + f_bwd) / (ms_g * 1e-3) / 1e12})
+                del graph
         # bytes of one forward (qkv read, out written, lse written) against HBM
         byt = w.layers * w.tokens() * w.heads * (3 * 64 + 64 + 4)
         line["fwd_gbs"] = byt / (ms_f * 1e-3) / 1e9
