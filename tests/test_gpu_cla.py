@@ -112,6 +112,7 @@ def _cla_bwd_case(B, H, W, C, seed):
     (1, 8, 16, 32),       # one tile, every pixel at the border
     (1, 16, 32, 96),      # three heads, a partial 64-channel group
     (2, 32, 48, 192),     # six heads (two point-wise accumulators), several tiles
+    (1, 16, 32, 160),     # five heads: a partial last 64-channel chunk and two M blocks
 ])
 def test_cla_bwd_parity(B, H, W, C):
     _cla_bwd_case(B, H, W, C, seed=C + 7)
